@@ -1,0 +1,191 @@
+/*
+ * ai_index.h - C ABI of the causal IVF top-k key selection library
+ * (libai_index.so, sm_100a).
+ *
+ * What it computes.  For every query of a chunked causal prefill, the top-k
+ * keys under the DSA indexer score
+ *     I(q, s) = sum_h w_h * ReLU(q_h . k_s),
+ * selected through a causal inverted-file index over the indexer keys, as
+ * described on the pages titled "AttentionIndex: Accelerating Learned Sparse
+ * Attention with a Causal Inverted-File Index" (paper-daily.com explainer;
+ * kurate.org review).  Sections cited below are those of the explainer.
+ *
+ * Conventions for every call.
+ *  - Pointers named *_dev are CUDA device pointers owned by the caller; the
+ *    library never frees them.  Pointers named *_host are host memory.
+ *  - All work is enqueued on the handle's main stream (given at create time)
+ *    and is asynchronous unless stated otherwise; call ai_sync() to wait
+ *    and to collect device-side error flags.
+ *  - Return value: AI_OK (0) or a negative AI_ERR_* code; ai_last_error()
+ *    gives a message for the calling thread.  A call that fails leaves the
+ *    index unchanged unless stated otherwise.
+ *  - Layouts are row-major and dense: keys [n, d], queries [T, H, d],
+ *    head weights [T, H] float32, outputs [T, k] int32.
+ *  - One handle is one (request, layer) index; handles are independent and
+ *    must not be used from two threads at once.
+ */
+#ifndef AI_INDEX_H_
+#define AI_INDEX_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ errors */
+#define AI_OK 0
+#define AI_ERR_ARG (-1)          /* invalid argument, shape or dtype            */
+#define AI_ERR_OOM (-2)          /* device allocation failed, or max_keys hit  */
+#define AI_ERR_CAUSALITY (-3)    /* a query position beyond the appended keys  */
+#define AI_ERR_DEVICE_CHECK (-4) /* a kernel flagged an out-of-range id/offset */
+#define AI_ERR_TIMEOUT (-5)      /* a bounded device wait or host wait ran out */
+#define AI_ERR_CUDA (-6)         /* a CUDA runtime call failed                 */
+#define AI_ERR_STATE (-7)        /* call not valid in the current state        */
+
+/* ------------------------------------------------------------ dtypes */
+#define AI_FP32 0     /* float32                                              */
+#define AI_BF16 1     /* bfloat16 bits (uint16)                               */
+#define AI_FP8E4M3 2  /* OCP FP8 E4M3 codes (uint8) + one float32 scale per key */
+
+typedef struct ai_index* ai_handle;
+
+/* Index configuration.  Field names follow the pages' notation.           */
+typedef struct ai_config {
+  int32_t d;                   /* key / query head dimension                 */
+  int32_t H;                   /* indexer heads                              */
+  int32_t key_dtype;           /* AI_FP32 | AI_BF16 | AI_FP8E4M3             */
+  int32_t q_dtype;             /* AI_FP32 (only with AI_FP32 keys) | AI_BF16 */
+  int32_t n_sinks;             /* S: first keys, always candidates, never clustered */
+  int32_t window;              /* W: open keys sealed together               */
+  int32_t clusters_per_window; /* m                                          */
+  int32_t cluster_cap;         /* size cap at seal; 0 -> ceil(W / m)         */
+  int32_t refit_period;        /* R (multiple of W); 0 = never refit         */
+  int32_t refit_new_seeds;     /* seeds per refit; 0 -> R * m / W            */
+  int32_t refit_seed_window;   /* seeds come from the last keys; 0 -> R      */
+  int32_t seal_iters;          /* k-means passes at seal; 0 -> 10            */
+  int32_t async_refit;         /* 1: refit runs on an internal side stream   */
+  int32_t max_query_chunk;     /* largest T passed to route/exhaustive calls */
+  int32_t max_budget;          /* largest C passed to ai_route_refine        */
+  int32_t max_k;               /* largest k                                  */
+  int64_t max_keys;            /* capacity of the key store                  */
+  uint64_t seed;               /* seed of the refit seed draws (SplitMix64)  */
+  const float* encoder_weights_host; /* NULL: plain mean representatives.   */
+  /* Else the correction encoder's float32 weights, packed in this order:
+   * A [d,d], a [d], B1 [d, 3d+1], b1 [d], B2 [d,d], b2 [d] (copied at create). */
+} ai_config;
+
+/* Create an index.  `cuda_stream` is the main stream (cudaStream_t, may be
+ * NULL for the legacy default stream).  Allocates the key store and all
+ * device scratch sized from the config.  Errors: AI_ERR_ARG, AI_ERR_OOM,
+ * AI_ERR_CUDA.  On success *out is a new handle.                           */
+int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out);
+
+/* Free a handle and everything it owns (waits for its streams first).     */
+int ai_index_destroy(ai_handle h);
+
+/* Insert (explainer, "索引怎么边算边建？" item 1).  Appends n keys to the
+ * append-only store; they are candidates of every later query at once (the
+ * open window).  keys_dev: [n, d] in the key dtype (fp8: codes);
+ * scales_dev: [n] float32 per-key scales for AI_FP8E4M3, else NULL.
+ * Also publishes a pending refit first (see ai_refit).  Errors: AI_ERR_ARG,
+ * AI_ERR_OOM (store full).                                                */
+int ai_append_keys(ai_handle h, const void* keys_dev, const float* scales_dev, int64_t n);
+
+/* Seal (explainer, "索引怎么边算边建？" item 2).  Clusters every complete
+ * W-window of open keys into m size-capped k-means clusters and appends
+ * them; each seal creates a version whose open window starts after the
+ * sealed keys.  Whenever the number of sealed keys reaches a multiple of R
+ * a refit is started (see ai_refit).  *version_out (nullable) receives the
+ * newest version number.                                                  */
+int ai_seal(ai_handle h, int64_t* version_out);
+
+/* Refit (explainer, "索引怎么边算边建？" item 3).  One warm-started assign +
+ * update pass over all sealed keys [S, n_r): previous refit centres plus
+ * new seeds drawn from the last keys, Hamerly bounds, member means.  Runs
+ * on the side stream when async_refit = 1.  The result becomes the index
+ * base at the next ai_append_keys or ai_publish call (a version with
+ * watermark n_r).  n_new_seeds / seed_window: 0 -> config values.         */
+int ai_refit(ai_handle h, int32_t n_new_seeds, int32_t seed_window, int64_t* version_out);
+
+/* Make a pending refit the index base now (waits on the side stream from
+ * the main stream, not from the host).  No-op without a pending refit.     */
+int ai_publish(ai_handle h);
+
+/* Route + refine (explainer, "查询时怎么挑候选？").  For the T queries at
+ * positions pos0 .. pos0+T-1: each query t uses the newest version whose
+ * keys all lie in its prefix, scores every visible cluster representative,
+ * fills C candidate slots with the sinks, the open window [n_v, t] and
+ * whole member lists in rank order (score desc, cluster id asc; the last
+ * list is truncated), rescores the candidates exactly and writes the top k
+ * ids by (score desc, id asc) to out_dev[T, k] in candidate order, padded
+ * with -1.  q_dev: [T, H, d] in q_dtype; w_dev: [T, H] float32;
+ * out_scores_dev: [T, k] float32 or NULL.  Errors: AI_ERR_ARG (T, k, C
+ * beyond the create-time maxima), AI_ERR_CAUSALITY (pos0 + T - 1 >=
+ * appended keys).                                                          */
+int ai_route_refine(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
+                    int32_t T, int32_t k, int32_t C, int32_t* out_dev, float* out_scores_dev);
+
+/* Exhaustive selection (explainer, "它到底在解决什么问题？": the indexer
+ * scores every key s <= t).  Same arguments and output order rules as
+ * ai_route_refine (ids ascending).  The in-library baseline.              */
+int ai_select_exhaustive(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
+                         int32_t T, int32_t k, int32_t* out_dev, float* out_scores_dev);
+
+/* Wait for all work of the handle (both streams) and report device-side
+ * error flags: AI_ERR_DEVICE_CHECK or AI_ERR_TIMEOUT (flags are cleared).  */
+int ai_sync(ai_handle h);
+
+/* Message of the last error on this thread ("" if none).                  */
+const char* ai_last_error(void);
+
+/* -------------------------------------------------------- inspection */
+typedef struct ai_stats {
+  int64_t n_keys;        /* appended keys                                   */
+  int64_t n_sealed;      /* sealed windows                                  */
+  int64_t n_clusters;    /* clusters in the published array                 */
+  int64_t n_versions;    /* versions in the published table                 */
+  int64_t n_refits;      /* refits started                                  */
+  int64_t refit_pending; /* 1 if a refit awaits publication                 */
+  int64_t base_watermark;/* n_r of the published base (0 = none)            */
+  int64_t last_refit_scanned; /* keys fully scanned by the last finished refit */
+} ai_stats;
+int ai_get_stats(ai_handle h, ai_stats* out);
+
+/* Copy the published index to host memory (synchronous).  Any pointer may
+ * be NULL.  offsets_host [n_clusters + 1] (member offsets, relative),
+ * members_host [offsets[n_clusters]], reps_bf16_host [n_clusters, d],
+ * centroids_host [n_clusters, d] float64, version_nc_host / version_nv_host
+ * [n_versions] (visible clusters, open-window start).                      */
+int ai_export_index(ai_handle h, int32_t* offsets_host, int32_t* members_host,
+                    uint16_t* reps_bf16_host, double* centroids_host, int64_t* version_nc_host,
+                    int64_t* version_nv_host);
+
+/* Debug: the candidate lists [T, C] (-1 padded) and cluster scores
+ * [T, n_clusters] that ai_route_refine would use for these queries.        */
+int ai_debug_candidates(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
+                        int32_t T, int32_t C, int32_t* cand_dev, float* cluster_scores_dev);
+
+/* Debug: the full indexer score matrix out_dev[T, n_keys] (float32, -inf
+ * where key position > query position) computed by the exhaustive kernels. */
+int ai_debug_scores(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0, int32_t T,
+                    float* out_dev);
+
+/* Checkpoint / rollback of the index state (host counters, version table,
+ * active cluster buffer and per-key refit bounds).  Rollback forgets keys
+ * appended after the checkpoint (they must be appended again).  Fails with
+ * AI_ERR_STATE while a refit is pending at checkpoint time.               */
+int ai_checkpoint(ai_handle h);
+int ai_rollback(ai_handle h);
+
+/* fp8 store helper: per-key scale = amax / 448 and E4M3 codes (round to
+ * nearest even, saturating) from bf16 keys [n, d].  Enqueued on
+ * cuda_stream.                                                            */
+int ai_quantize_fp8(const uint16_t* keys_bf16_dev, int64_t n, int32_t d, uint8_t* codes_dev,
+                    float* scales_dev, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AI_INDEX_H_ */

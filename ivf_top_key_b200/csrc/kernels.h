@@ -1,0 +1,155 @@
+// Internal launchers of the causal IVF top-k library (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace aiidx {
+
+// ---------------------------------------------------------- score matrices
+struct ScoreArgs {
+  int nA;                  // rows of A
+  int T;                   // queries
+  const float* w;          // [T, H] head weights
+  const float* row_scale;  // [nA] per-row positive scale or nullptr
+  float* out;              // out[q * ld_out + a]
+  int64_t ld_out;
+  int a_tiles_per_cta;
+  int causal;              // mask a_pos0 + a > q_pos0 + q to -inf
+  int64_t a_pos0;
+  int64_t q_pos0;
+  int* err;
+};
+int scores_smem_bytes();
+cudaError_t launch_scores_tc(const CUtensorMap& mapA, const CUtensorMap& mapB, int H,
+                             const ScoreArgs& args, int a_tiles_per_cta, cudaStream_t st);
+cudaError_t launch_scores_simt(const void* A, int a_dtype, const void* Q, int q_is_bf16, int d,
+                               int H, const ScoreArgs& args, cudaStream_t st);
+
+// --------------------------------------------------------- route + refine
+constexpr int kMaxSegs = 64;
+struct VersionSeg {
+  int64_t first_pos;  // first query position that uses this version
+  int64_t n_v;        // open-window start (clustered keys are [S, n_v))
+  int32_t nC;         // visible clusters (a prefix of the cluster array)
+  int32_t pad;
+};
+struct VersionTable {
+  int n;
+  int pad;
+  VersionSeg seg[kMaxSegs];
+};
+
+struct RefineArgs {
+  const void* keys;          // key store [N, d] (fp32 / bf16 / fp8 codes)
+  const float* key_scale;    // fp8 per-key scale, else nullptr
+  int key_dtype;
+  const void* q;             // [T, H, d] (fp32 or bf16)
+  int q_is_bf16;
+  const float* w;            // [T, H]
+  const float* route;        // [T, ld_route] cluster scores
+  int64_t ld_route;
+  const int32_t* offsets;    // CSR offsets [nC + 1]
+  const int32_t* members;    // CSR members
+  int64_t pos0;
+  int T, H, d, k, C, n_sinks;
+  int32_t* out;              // [T, k]
+  float* out_scores;         // [T, k] or nullptr
+  int32_t* cand_out;         // debug: [T, C] candidate lists or nullptr
+  int* err;
+};
+size_t refine_smem_bytes(int C, int H, int d, bool tc);
+cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, bool tc, int num_sms,
+                          cudaStream_t st);
+
+// ------------------------------------------------------- exhaustive top-k
+struct RowTopkArgs {
+  const float* scores;  // [T, ld]
+  int64_t ld;
+  int T;
+  int64_t q_pos0;       // query i sees keys [0, q_pos0 + i]
+  int64_t n_keys;       // keys in the store
+  int k;
+  int32_t* out;         // [T, k] (row stride k)
+  float* out_scores;    // or nullptr
+  int* err;
+};
+cudaError_t launch_row_topk(const RowTopkArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------------ seal
+struct SealArgs {
+  const void* keys;
+  const float* key_scale;
+  int key_dtype;
+  int d, W, m, cap, iters;
+  int64_t first_key;        // window j covers keys [first_key + j W, + W)
+  int n_windows;
+  int32_t* members;         // output: window j writes members[mem_base + j W ...]
+  int64_t mem_base;
+  int32_t* offsets;         // output: offsets[cl_base + j m + c] (start of each cluster)
+  int64_t cl_base;
+  double* centroids;        // [cl_base + j m + c][d]
+  uint16_t* reps;           // bf16 [.., d]
+  int* err;
+};
+size_t seal_smem_bytes(int W, int m, int d);
+cudaError_t launch_seal(const SealArgs& a, cudaStream_t st);
+
+// ----------------------------------------------------------------- refit
+struct RefitArgs {
+  const void* keys;
+  const float* key_scale;
+  int key_dtype;
+  int d;
+  int64_t S;             // first clustered key
+  int64_t n_r;           // refit covers keys [S, n_r)
+  int64_t n_old;         // keys [S, n_old) carry bounds from the previous refit
+  int K_prev;            // centroids carried from the previous refit
+  int K;                 // K_prev + seeds
+  const int64_t* seed_ids;  // [K - K_prev] (device)
+  const double* prev_centroids;  // [K_prev, d] (device, may alias nothing)
+  double* cent;          // [K, d] working centroids (output: updated)
+  float* cent32;         // [K, d] fp32 copy for screening
+  double* cent_old;      // [K, d] centroids before update (for drift)
+  int32_t* assign;       // [N] per key (index = key id)
+  float* ub;             // [N] upper bound to own centre
+  float* lb;             // [N] lower bound to every other centre
+  int32_t* counts;       // [K]
+  int32_t* offsets;      // [K + 1] output CSR
+  int32_t* members;      // [n_r - S] output CSR members
+  uint16_t* reps;        // [K, d] bf16
+  double* drift;         // [K]
+  float* seed_lb;        // [K_prev] min distance from old centre to any seed
+  int32_t* tile_counts;  // scratch [ntiles * K]
+  int32_t* scan_list;    // scratch [n_r - S] keys needing a full scan
+  int32_t* n_scan;       // scratch [1]
+  int* err;
+};
+cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
+                         int32_t* host_nscan /*nullable: read back count*/);
+int64_t refit_tile_size();
+
+// --------------------------------------------------------------- encoder
+struct EncoderArgs {
+  const void* keys;
+  const float* key_scale;
+  int key_dtype;
+  int d;
+  const int32_t* offsets;  // cluster c members offsets[c] .. offsets[c+1]
+  const int32_t* members;
+  const double* centroids; // [.., d]
+  int cl_begin, cl_end;    // clusters to (re)compute
+  const float* wts;        // packed A [d,d], a [d], B1 [d, 3d+1], b1 [d], B2 [d,d], b2 [d]
+  uint16_t* reps;          // bf16 output
+  int* err;
+};
+cudaError_t launch_encoder(const EncoderArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- formats
+cudaError_t launch_quantize_fp8(const uint16_t* keys_bf16, int64_t n, int d, uint8_t* codes,
+                                float* scales, cudaStream_t st);
+cudaError_t launch_fp8_codes_to_bf16(const uint8_t* codes, int64_t n, int d, uint16_t* out,
+                                     cudaStream_t st);
+
+}  // namespace aiidx

@@ -1,0 +1,461 @@
+// Refit: one warm-started assign + update pass over the whole clustered
+// prefix, with Hamerly bounds.
+//
+// AttentionIndex explainer (paper-daily.com), section "索引怎么边算边建？",
+// item 3 and the paragraph after it: every R tokens the whole prefix is
+// regrouped, starting from the previous centres plus a few new centres taken
+// from recent keys; each key keeps an upper bound to its own centre and a
+// lower bound to the others, and only new keys and keys whose bounds no
+// longer guarantee their cluster are compared against all centres; one
+// round of assignment and update, run on a side CUDA stream.  The kurate.org
+// review ("Core Contribution", item 1) names the bounds Elkan/Hamerly-style.
+//
+// The result equals plain nearest-centre assignment (ties to the lower
+// centre id) followed by a mean update: the bounds only skip comparisons
+// whose outcome they already prove.  Bounds are kept conservative in fp32
+// (rounded outward, with a relative margin), distances are screened in fp32
+// and every near tie is decided again in float64.
+//
+// Steps (all on the stream given):
+//   init     centres = previous refit centres ++ seed keys (float64)
+//   seed_lb  for each previous centre a: min over seeds of ||c_a - s||
+//   test     Hamerly test for keys with bounds; failures and new keys are
+//            queued for a full scan
+//   scan     fp32 distances to all centres (tiled SIMT), best and second
+//   recheck  float64 argmin for keys whose best two are within the margin
+//   count / tile counts / scan / scatter: CSR by cluster, members in
+//            ascending key id (deterministic, no float atomics)
+//   update   float64 member means in CSR order, drift, bf16 representatives
+//   bounds   u += drift(own), l -= max drift
+#include "common.cuh"
+#include "kernels.h"
+
+namespace aiidx {
+namespace {
+
+constexpr int64_t kTileKeys = 4096;  // keys per CSR tile
+constexpr float kRel = 1e-4f;         // relative margin of fp32 distances
+
+__device__ __forceinline__ double kf64(const RefitArgs& a, int64_t s, int i) {
+  double v = key_elem(a.keys, a.key_dtype, s, a.d, i);
+  if (a.key_dtype == KD_FP8) v *= static_cast<double>(a.key_scale[s]);
+  return v;
+}
+__device__ __forceinline__ float kf32(const RefitArgs& a, int64_t s, int i) {
+  float v = key_elem(a.keys, a.key_dtype, s, a.d, i);
+  if (a.key_dtype == KD_FP8) v *= a.key_scale[s];  // screening only; near ties are redone in fp64
+  return v;
+}
+
+__global__ void k_init(RefitArgs a) {
+  const int64_t n = static_cast<int64_t>(a.K) * a.d;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(e / a.d), i = static_cast<int>(e % a.d);
+    double v = j < a.K_prev ? a.prev_centroids[e] : kf64(a, a.seed_ids[j - a.K_prev], i);
+    a.cent[e] = v;
+    a.cent_old[e] = v;
+    a.cent32[e] = static_cast<float>(v);
+  }
+}
+
+// one warp per previous centre
+__global__ void k_seed_lb(RefitArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= a.K_prev) return;
+  const int ns = a.K - a.K_prev;
+  double best = 1e300;
+  for (int sidx = 0; sidx < ns; ++sidx) {
+    double acc = 0.0;
+    for (int i = lane; i < a.d; i += 32) {
+      const double df = a.cent[static_cast<int64_t>(warp) * a.d + i] -
+                        a.cent[static_cast<int64_t>(a.K_prev + sidx) * a.d + i];
+      acc = fma(df, df, acc);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    best = fmin(best, acc);
+  }
+  if (lane == 0) a.seed_lb[warp] = __double2float_rd(sqrt(best) * (1.0 - 1e-6));
+}
+
+// Hamerly test.  One thread per key in [S, n_r).
+__global__ void k_test(RefitArgs a) {
+  const int64_t x = a.S + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (x >= a.n_r) return;
+  bool scan = true;
+  if (x < a.n_old && a.K_prev > 0) {
+    const int ca = a.assign[x];
+    float u = a.ub[x];
+    float l = a.lb[x];
+    if (a.K > a.K_prev) l = fminf(l, __fsub_rd(a.seed_lb[ca], u));
+    if (u < l) {
+      scan = false;
+    } else {
+      // tighten u to the exact distance and retest
+      double acc = 0.0;
+      for (int i = 0; i < a.d; ++i) {
+        const double df = kf64(a, x, i) - a.cent[static_cast<int64_t>(ca) * a.d + i];
+        acc = fma(df, df, acc);
+      }
+      u = __double2float_ru(sqrt(acc) * (1.0 + 1e-6));
+      if (u < l) {
+        scan = false;
+        a.ub[x] = u;
+        a.lb[x] = l;
+      }
+    }
+  }
+  if (scan) {
+    const int pos = atomicAdd(a.n_scan, 1);
+    a.scan_list[pos] = static_cast<int32_t>(x);
+  }
+}
+
+// Full scan in fp32: block = 64 keys x all centres in tiles of 64.
+// Thread (r, c) of a 16 x 16 grid covers keys 4r..4r+3 and centres
+// 4c..4c+3 of each tile.
+constexpr int kSK = 64, kSC = 64, kSD = 32;
+__global__ void __launch_bounds__(256) k_scan(RefitArgs a, int32_t* recheck, int32_t* n_recheck) {
+  __shared__ float xs[kSK][kSD + 1];
+  __shared__ float cs[kSC][kSD + 1];
+  const int n = *a.n_scan;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  for (int kb = blockIdx.x * kSK; kb < n; kb += gridDim.x * kSK) {
+  float best[4], second[4];
+  int bid[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    best[r] = INFINITY;
+    second[r] = INFINITY;
+    bid[r] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < a.K; c0 += kSC) {
+    float acc[4][4] = {};
+    for (int d0 = 0; d0 < a.d; d0 += kSD) {
+      for (int e = threadIdx.x; e < kSK * kSD; e += blockDim.x) {
+        const int r = e / kSD, i = e % kSD;
+        const int kk = kb + r;
+        xs[r][i] = (kk < n && d0 + i < a.d) ? kf32(a, a.scan_list[kk], d0 + i) : 0.f;
+      }
+      for (int e = threadIdx.x; e < kSC * kSD; e += blockDim.x) {
+        const int r = e / kSD, i = e % kSD;
+        const int cc = c0 + r;
+        cs[r][i] = (cc < a.K && d0 + i < a.d) ? a.cent32[static_cast<int64_t>(cc) * a.d + d0 + i] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int i = 0; i < kSD; ++i) {
+        float xv[4], cv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) xv[r] = xs[tr * 4 + r][i];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cv[c] = cs[tc * 4 + c][i];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float df = xv[r] - cv[c];
+            acc[r][c] = fmaf(df, df, acc[r][c]);
+          }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int cc = c0 + tc * 4 + c;
+      if (cc >= a.K) continue;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float v = acc[r][c];
+        if (v < best[r] || (v == best[r] && cc < bid[r])) {
+          second[r] = best[r];
+          best[r] = v;
+          bid[r] = cc;
+        } else if (v < second[r]) {
+          second[r] = v;
+        }
+      }
+    }
+  }
+  // merge across the 16 threads of a row (consecutive lanes)
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best[r], o);
+      const float os = __shfl_xor_sync(0xffffffffu, second[r], o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bid[r], o);
+      if (ob < best[r] || (ob == best[r] && oi < bid[r])) {
+        second[r] = fminf(best[r], os);
+        best[r] = ob;
+        bid[r] = oi;
+      } else {
+        second[r] = fminf(second[r], ob);
+      }
+    }
+  }
+  if (tc == 0) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int kk = kb + tr * 4 + r;
+      if (kk >= n) continue;
+      const int32_t x = a.scan_list[kk];
+      a.assign[x] = bid[r];
+      if (second[r] - best[r] <= kRel * second[r] + 1e-30f) {
+        const int p = atomicAdd(n_recheck, 1);
+        recheck[p] = x;
+      }
+      a.ub[x] = __fmul_ru(sqrtf(best[r]), 1.f + kRel);
+      a.lb[x] = __fmul_rd(sqrtf(second[r]), 1.f - kRel);
+    }
+  }
+  __syncthreads();
+  }
+}
+
+// float64 decision for near ties: one block per key.
+__global__ void __launch_bounds__(256) k_recheck(RefitArgs a, const int32_t* recheck,
+                                                 const int32_t* n_recheck) {
+  __shared__ double xs[256];
+  __shared__ double rb[8], rs[8];
+  __shared__ int ri[8];
+  const int nr = *n_recheck;
+  for (int idx = blockIdx.x; idx < nr; idx += gridDim.x) {
+  const int32_t x = recheck[idx];
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.d; i += blockDim.x) xs[i] = kf64(a, x, i);
+  __syncthreads();
+  double best = INFINITY, second = INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = threadIdx.x; c < a.K; c += blockDim.x) {
+    double acc = 0.0;
+    for (int i = 0; i < a.d; ++i) {
+      const double df = xs[i] - a.cent[static_cast<int64_t>(c) * a.d + i];
+      acc = fma(df, df, acc);
+    }
+    if (acc < best || (acc == best && c < bi)) {
+      second = best;
+      best = acc;
+      bi = c;
+    } else if (acc < second) {
+      second = acc;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const double os = __shfl_xor_sync(0xffffffffu, second, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob < best || (ob == best && oi < bi)) {
+      second = fmin(best, os);
+      best = ob;
+      bi = oi;
+    } else {
+      second = fmin(second, ob);
+    }
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    rb[w] = best;
+    rs[w] = second;
+    ri[w] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int j = 1; j < (blockDim.x >> 5); ++j) {
+      if (rb[j] < best || (rb[j] == best && ri[j] < bi)) {
+        second = fmin(best, rs[j]);
+        best = rb[j];
+        bi = ri[j];
+      } else {
+        second = fmin(second, rb[j]);
+      }
+    }
+    a.assign[x] = bi;
+    a.ub[x] = __double2float_ru(sqrt(best) * (1.0 + 1e-6));
+    a.lb[x] = __double2float_rd(sqrt(second) * (1.0 - 1e-6));
+  }
+  __syncthreads();
+  }
+}
+
+__global__ void k_zero_counts(RefitArgs a) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < a.K; j += gridDim.x * blockDim.x)
+    a.counts[j] = 0;
+}
+
+__global__ void k_count(RefitArgs a) {
+  const int64_t x = a.S + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (x >= a.n_r) return;
+  const int c = a.assign[x];
+  if (c < 0 || c >= a.K) {
+    atomicOr(a.err, DEV_ERR_RANGE);
+    return;
+  }
+  atomicAdd(&a.counts[c], 1);
+}
+
+// exclusive scan of counts -> offsets (single block)
+__global__ void __launch_bounds__(1024) k_offsets(RefitArgs a) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int base = 0; base < a.K; base += blockDim.x) {
+    const int j = base + threadIdx.x;
+    const int v = j < a.K ? a.counts[j] : 0;
+    int incl = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int s = warp_sums[lane];
+      int si = s;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, si, o);
+        if (lane >= o) si += n;
+      }
+      warp_sums[lane] = si - s;
+    }
+    __syncthreads();
+    if (j < a.K) a.offsets[j] = carry + warp_sums[w] + incl - v;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry += warp_sums[w] + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) a.offsets[a.K] = carry;
+}
+
+// per-tile cluster counts: one warp per tile, keys walked in order
+__global__ void k_tile_counts(RefitArgs a) {
+  extern __shared__ int cnt[];
+  const int tile = blockIdx.x;
+  const int lane = threadIdx.x;
+  for (int j = lane; j < a.K; j += 32) cnt[j] = 0;
+  __syncwarp();
+  const int64_t x0 = a.S + tile * kTileKeys;
+  const int64_t x1 = min(a.n_r, x0 + kTileKeys);
+  for (int64_t xb = x0; xb < x1; xb += 32) {
+    const int64_t x = xb + lane;
+    const bool v = x < x1;
+    const int c = v ? a.assign[x] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    if (v && __ffs(peers) - 1 == lane) cnt[c] += __popc(peers);
+    __syncwarp();
+  }
+  for (int j = lane; j < a.K; j += 32) a.tile_counts[static_cast<int64_t>(tile) * a.K + j] = cnt[j];
+}
+
+// tile_counts[t][j] <- offsets[j] + sum of counts of earlier tiles
+__global__ void k_tile_base(RefitArgs a, int ntiles) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.K) return;
+  int run = a.offsets[j];
+  for (int t = 0; t < ntiles; ++t) {
+    int32_t* p = a.tile_counts + static_cast<int64_t>(t) * a.K + j;
+    const int v = *p;
+    *p = run;
+    run += v;
+  }
+}
+
+__global__ void k_scatter(RefitArgs a) {
+  extern __shared__ int base[];
+  const int tile = blockIdx.x;
+  const int lane = threadIdx.x;
+  for (int j = lane; j < a.K; j += 32) base[j] = a.tile_counts[static_cast<int64_t>(tile) * a.K + j];
+  __syncwarp();
+  const int64_t x0 = a.S + tile * kTileKeys;
+  const int64_t x1 = min(a.n_r, x0 + kTileKeys);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int64_t xb = x0; xb < x1; xb += 32) {
+    const int64_t x = xb + lane;
+    const bool v = x < x1;
+    const int c = v ? a.assign[x] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    if (v) a.members[base[c] + __popc(peers & lt)] = static_cast<int32_t>(x);
+    __syncwarp();
+    if (v && __ffs(peers) - 1 == lane) base[c] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// one warp per cluster: float64 mean in member order, drift, bf16 rep
+__global__ void k_update(RefitArgs a, unsigned long long* max_drift_bits) {
+  const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (j >= a.K) return;
+  const int o0 = a.offsets[j], o1 = a.offsets[j + 1];
+  double dr = 0.0;
+  for (int i = lane; i < a.d; i += 32) {
+    const int64_t e = static_cast<int64_t>(j) * a.d + i;
+    double v = a.cent[e];
+    if (o1 > o0) {
+      double sum = 0.0;
+      for (int p = o0; p < o1; ++p) sum += kf64(a, a.members[p], i);
+      v = sum / static_cast<double>(o1 - o0);
+    }
+    const double df = v - a.cent_old[e];
+    dr = fma(df, df, dr);
+    a.cent[e] = v;
+    a.reps[e] = f64_to_bf16_rne(v);
+  }
+  for (int o = 16; o > 0; o >>= 1) dr += __shfl_xor_sync(0xffffffffu, dr, o);
+  if (lane == 0) {
+    const double drift = sqrt(dr) * (1.0 + 1e-6);
+    a.drift[j] = drift;
+    atomicMax(max_drift_bits, static_cast<unsigned long long>(__double_as_longlong(drift)));
+  }
+}
+
+__global__ void k_bounds(RefitArgs a, const unsigned long long* max_drift_bits) {
+  const int64_t x = a.S + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (x >= a.n_r) return;
+  const double md = __longlong_as_double(static_cast<long long>(*max_drift_bits));
+  const int c = a.assign[x];
+  a.ub[x] = __fadd_ru(a.ub[x], __double2float_ru(a.drift[c]));
+  a.lb[x] = __fsub_rd(a.lb[x], __double2float_ru(md));
+}
+
+}  // namespace
+
+int64_t refit_tile_size() { return kTileKeys; }
+
+cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
+                         int32_t* host_nscan) {
+  const int64_t n = a.n_r - a.S;
+  if (n <= 0 || a.K <= 0) return cudaSuccess;
+  const int64_t ntiles = (n + kTileKeys - 1) / kTileKeys;
+  if (ntiles > max_tiles) return cudaErrorInvalidValue;
+  if (static_cast<size_t>(a.K) * 4 > 200 * 1024) return cudaErrorInvalidValue;
+  // scratch words after n_scan: [1] n_recheck, [2..3] max drift bits
+  int32_t* n_recheck = a.n_scan + 1;
+  unsigned long long* mdb = reinterpret_cast<unsigned long long*>(a.n_scan + 2);
+  cudaMemsetAsync(a.n_scan, 0, 16, st);
+  const int64_t ce = static_cast<int64_t>(a.K) * a.d;
+  k_init<<<static_cast<unsigned>((ce + 255) / 256 < 4096 ? (ce + 255) / 256 : 4096), 256, 0, st>>>(a);
+  if (a.K_prev > 0 && a.K > a.K_prev) k_seed_lb<<<(a.K_prev * 32 + 255) / 256, 256, 0, st>>>(a);
+  const unsigned gk = static_cast<unsigned>((n + 255) / 256);
+  k_test<<<gk, 256, 0, st>>>(a);
+  // the scan list length is only known on the device: fixed grids that stride
+  const int64_t sblocks = (n + kSK - 1) / kSK;
+  k_scan<<<static_cast<unsigned>(sblocks < 1184 ? sblocks : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
+  // recheck list lives after the scan list (capacity n)
+  k_recheck<<<static_cast<unsigned>(n < 1184 ? n : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
+  k_zero_counts<<<(a.K + 255) / 256, 256, 0, st>>>(a);
+  k_count<<<gk, 256, 0, st>>>(a);
+  k_offsets<<<1, 1024, 0, st>>>(a);
+  const size_t sm = static_cast<size_t>(a.K) * 4;
+  cudaFuncSetAttribute(k_tile_counts, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  k_tile_counts<<<static_cast<unsigned>(ntiles), 32, sm, st>>>(a);
+  k_tile_base<<<(a.K + 255) / 256, 256, 0, st>>>(a, static_cast<int>(ntiles));
+  k_scatter<<<static_cast<unsigned>(ntiles), 32, sm, st>>>(a);
+  k_update<<<static_cast<unsigned>((static_cast<int64_t>(a.K) * 32 + 255) / 256), 256, 0, st>>>(a, mdb);
+  k_bounds<<<gk, 256, 0, st>>>(a, mdb);
+  if (host_nscan) cudaMemcpyAsync(host_nscan, a.n_scan, 8, cudaMemcpyDeviceToHost, st);
+  return cudaGetLastError();
+}
+
+}  // namespace aiidx

@@ -1,0 +1,186 @@
+// Block-wide selection helpers: ordered compaction and radix select.
+//
+// Used by the per-query top-k (candidate scores in shared memory), the
+// exhaustive row top-k (scores in global memory) and the size-weighted
+// cluster threshold of the candidate fill.
+#pragma once
+
+#include "common.cuh"
+
+namespace aiidx {
+
+struct BlockScratch {
+  uint32_t hist[256];     // radix histogram (counts or weights)
+  int warp_tot[40];       // per-warp totals for ordered compaction
+  int bcast[8];           // broadcast slots
+};
+
+// Exclusive prefix of `pred` over the block in thread order.  Returns this
+// thread's rank among the threads with pred set; *total receives the count.
+// Every thread of the block must call it.
+__device__ __forceinline__ int block_rank(bool pred, int* total, BlockScratch& bs) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, pred);
+  const int in_warp = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) bs.warp_tot[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < nwarps ? bs.warp_tot[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane < nwarps) bs.warp_tot[lane] = incl - v;  // exclusive
+    if (lane == 31) bs.bcast[7] = incl;
+  }
+  __syncthreads();
+  const int r = bs.warp_tot[warp] + in_warp;
+  *total = bs.bcast[7];
+  __syncthreads();
+  return r;
+}
+
+// Radix select over n items with 32-bit keys: find theta, the key of the
+// k-th largest item among those with pred(i), with weights wt(i) (the
+// k-th unit of weight).  Returns theta and *above = weight strictly above
+// theta.  If the total weight is <= k, returns 0 and *above = total.
+// key(i), pred(i), wt(i) are functors; all threads call it.
+template <class KeyF, class PredF, class WtF>
+__device__ uint32_t radix_select(int n, KeyF key, PredF pred, WtF wt, uint64_t k, uint64_t* above,
+                                 BlockScratch& bs, uint64_t* tot_out = nullptr) {
+  uint32_t prefix = 0, mask = 0;
+  uint64_t need = k;
+  uint64_t above_acc = 0;
+  // total weight
+  __shared__ unsigned long long s_tot;
+  if (threadIdx.x == 0) s_tot = 0;
+  __syncthreads();
+  {
+    unsigned long long loc = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      if (pred(i)) loc += wt(i);
+    for (int o = 16; o > 0; o >>= 1) loc += __shfl_xor_sync(0xffffffffu, loc, o);
+    if ((threadIdx.x & 31) == 0 && loc) atomicAdd(&s_tot, loc);
+  }
+  __syncthreads();
+  const uint64_t total = s_tot;
+  if (tot_out) *tot_out = total;
+  if (total <= k) {
+    *above = total;
+    __syncthreads();
+    return 0;
+  }
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) bs.hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      if (!pred(i)) continue;
+      const uint32_t kk = key(i);
+      if ((kk & mask) != prefix) continue;
+      atomicAdd(&bs.hist[(kk >> shift) & 255u], static_cast<uint32_t>(wt(i)));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // scan digits from 255 down; lane l owns digits 255-8l .. 248-8l
+      const int lane = threadIdx.x;
+      uint64_t loc[8];
+      uint64_t lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        loc[j] = bs.hist[255 - (lane * 8 + j)];
+        lsum += loc[j];
+      }
+      uint64_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        uint64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      uint64_t run = incl - lsum;  // weight of digits above this lane's range
+      int found = -1;
+      uint64_t before = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (found < 0 && run + loc[j] >= need && run < need) {
+          found = 255 - (lane * 8 + j);
+          before = run;
+        }
+        run += loc[j];
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+      const int src = __ffs(who) - 1;
+      const int dg = __shfl_sync(0xffffffffu, found, src);
+      const uint64_t bf = __shfl_sync(0xffffffffu, before, src);
+      if (lane == 0) {
+        bs.bcast[0] = dg;
+        reinterpret_cast<unsigned long long*>(&bs.bcast[2])[0] = bf;
+      }
+    }
+    __syncthreads();
+    const uint32_t dg = static_cast<uint32_t>(bs.bcast[0]);
+    const uint64_t bf = reinterpret_cast<unsigned long long*>(&bs.bcast[2])[0];
+    need -= bf;
+    above_acc += bf;
+    prefix |= dg << shift;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  *above = above_acc;
+  return prefix;
+}
+
+// Top-k of n items (score(i), id(i)) by (score desc, id asc).  Writes the
+// selected ids (and scores) in item order, then pads with -1 / -inf up to
+// k.  All threads call it.
+template <class ScoreF, class IdF>
+__device__ void topk_select_emit(int n, ScoreF score, IdF id, int k, int32_t* out, float* outs,
+                                 BlockScratch& bs) {
+  auto skey = [&](int i) -> uint32_t { return f2key(score(i)); };
+  auto all = [&](int) -> bool { return true; };
+  auto one = [&](int) -> uint32_t { return 1u; };
+  uint64_t above = 0, tot = 0;
+  const uint32_t theta = radix_select(n, skey, all, one, static_cast<uint64_t>(k), &above, bs, &tot);
+  const bool take_all = tot <= static_cast<uint64_t>(k);
+  uint32_t theta_id = 0;
+  bool ties_all = true;
+  if (!take_all) {
+    const uint64_t need_eq = k - above;
+    auto idkey = [&](int i) -> uint32_t { return ~static_cast<uint32_t>(id(i)); };
+    auto tie = [&](int i) -> bool { return skey(i) == theta; };
+    uint64_t above2 = 0, tot2 = 0;
+    theta_id = radix_select(n, idkey, tie, one, need_eq, &above2, bs, &tot2);
+    ties_all = tot2 <= need_eq;
+  }
+  int written = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    bool p = false;
+    float sv = 0.f;
+    if (i < n) {
+      sv = score(i);
+      if (take_all) {
+        p = true;
+      } else {
+        const uint32_t kk = f2key(sv);
+        p = kk > theta || (kk == theta && (ties_all || (~static_cast<uint32_t>(id(i))) >= theta_id));
+      }
+    }
+    int total;
+    const int r = block_rank(p, &total, bs);
+    if (p && written + r < k) {
+      out[written + r] = id(i);
+      if (outs) outs[written + r] = sv;
+    }
+    written += total;
+  }
+  for (int j = min(written, k) + threadIdx.x; j < k; j += blockDim.x) {
+    out[j] = -1;
+    if (outs) outs[j] = -INFINITY;
+  }
+  __syncthreads();
+}
+
+}  // namespace aiidx

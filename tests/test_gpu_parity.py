@@ -1,0 +1,211 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64 CPU
+oracle, on seeded synthetic prefills.  Sizes span several 128-row tiles and
+ragged tails; the large workloads run scaled down here (full sizes are
+checked on sampled queries in test_gpu_fullsize.py)."""
+import collections
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ai_oracle as O
+from synth import workloads as S
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+
+def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_refit=True,
+                 seed_q=0):
+    """Chunked prefill on both sides; compare index state after every chunk
+    and route+refine / exhaustive results on (sampled) queries."""
+    gpu, orc = P.make_pair(wl, encoder=encoder, async_refit=async_refit)
+    rng = np.random.default_rng(1234 + seed_q)
+    stats = collections.Counter()
+    for c in range(wl.n_chunks):
+        p0, p1 = c * wl.T, (c + 1) * wl.T
+        kd, ks, kv = P.keys_inputs(wl, p0, p1)
+        gpu.append_keys(kd, ks)
+        orc.append(kv)
+        gpu.seal()
+        orc.seal()
+        gpu.sync()
+        P.check_index_equal(gpu, orc)
+        qd, wd, qv, wv = P.query_inputs(wl, p0, p1)
+        out = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
+        osc = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
+        gpu.route_refine(qd, wd, p0, wl.k, wl.budget, out=out, out_scores=osc)
+        cand, _ = gpu.debug_candidates(qd, wd, p0, wl.budget, with_scores=False)
+        gpu.sync()
+        idx = np.arange(wl.T) if sample is None else np.unique(np.concatenate(
+            [[0, wl.T - 1], rng.choice(wl.T, size=min(sample, wl.T), replace=False)]))
+        ids = out.cpu().numpy()[idx]
+        scs = osc.cpu().numpy()[idx]
+        cnd = cand.cpu().numpy()[idx]
+        P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], ids, scs, cnd, wl.k,
+                        wl.budget, stats)
+        if check_exhaustive:
+            eo = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
+            es = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
+            gpu.select_exhaustive(qd, wd, p0, wl.k, out=eo, out_scores=es)
+            gpu.sync()
+            eo, es = eo.cpu().numpy()[idx], es.cpu().numpy()[idx]
+            for j, i in enumerate(idx):
+                t = p0 + i
+                want, want_sc = orc.exhaustive(qv[i], wv[i], t, wl.k)
+                got = eo[j]
+                assert np.array_equal(got >= 0, np.arange(wl.k) < min(wl.k, t + 1))
+                assert np.all(np.diff(got[got >= 0]) > 0), "exhaustive ids must ascend"
+                if set(got[got >= 0].tolist()) != set(want[want >= 0].tolist()):
+                    theta = want_sc[(want >= 0).sum() - 1]
+                    for s in np.setxor1d(got[got >= 0], want[want >= 0]):
+                        sc = O.indexer_score(qv[i], wv[i], orc.keys[[s]])[0]
+                        tl = P.score_tol(qv[i], wv[i], orc.keys[[s]])[0]
+                        assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: exhaustive swap {s}"
+                    stats["exh_near_tie"] += 1
+                else:
+                    stats["exh_equal"] += 1
+                vs = got >= 0
+                exact = O.indexer_score(qv[i], wv[i], orc.keys[got[vs]])
+                tol = P.score_tol(qv[i], wv[i], orc.keys[got[vs]])
+                assert np.all(np.abs(es[j][vs] - exact) <= tol + 1e-6)
+    gpu.close()
+    return stats
+
+
+def test_tiny_fp32_full_prefill_every_query():
+    wl = S.WORKLOADS["tiny_fp32_L4k"]
+    st = _run_prefill(wl)
+    assert st["cand_equal"] + st["cand_near_tie"] == wl.L
+    assert st["cand_near_tie"] <= 0.01 * wl.L, st
+
+
+def test_glm_bf16_scaled_sampled():
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=20480, T=2048, refit_period=8192,
+                  budget=3000, k=256, M=256)
+    st = _run_prefill(wl, sample=48)
+    assert st["cand_near_tie"] <= 0.02 * (st["cand_equal"] + st["cand_near_tie"]), st
+
+
+def test_v4flash_fp8_scaled_sampled():
+    wl = S.scaled(S.WORKLOADS["v4flash_fp8_L256k"], L=12288, T=2048, refit_period=4096,
+                  budget=2500, k=200, M=256)
+    st = _run_prefill(wl, sample=32)
+    assert st["cand_equal"] > 0, st
+
+
+def test_synchronous_refit_matches_oracle():
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=10240, T=2048, refit_period=4096,
+                  budget=2048, k=128, M=128)
+    _run_prefill(wl, sample=16, async_refit=False, check_exhaustive=False)
+
+
+def test_encoder_correction_random_and_zero():
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k_encoder"], L=8192, T=2048, refit_period=4096,
+                  budget=2048, k=128, M=128)
+    enc = S.encoder_weights(wl)
+    _run_prefill(wl, sample=16, encoder=enc, check_exhaustive=False)
+    # zero output layer: representatives identical to plain IVF, bit for bit
+    zero = S.encoder_weights(wl, zero_out=True)
+    g0, _ = P.make_pair(wl, encoder=zero)
+    g1, _ = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        kd, ks, _ = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        for g in (g0, g1):
+            g.append_keys(kd, ks)
+            g.seal()
+    g0.sync()
+    g1.sync()
+    a, b = g0.export_index(), g1.export_index()
+    assert np.array_equal(a["reps_bf16"], b["reps_bf16"])
+    assert np.array_equal(a["members"], b["members"])
+
+
+def test_quantize_fp8_bit_exact():
+    g = np.random.default_rng(11)
+    x = (g.standard_normal((1000, 128)) * g.uniform(0.01, 30, size=(1000, 1)))
+    x[7] = 0.0
+    bits = S.to_bf16_bits(x)
+    kb = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    from ivf_top_key_b200 import quantize_fp8
+    codes, scales = quantize_fp8(kb)
+    torch.cuda.synchronize()
+    got = codes.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    oc, osc = O.quantize_fp8_keys(S.bf16_bits_to_f64(bits).astype(np.float32))
+    assert np.array_equal(scales.cpu().numpy(), osc)
+    assert np.array_equal(got, oc)
+
+
+@pytest.mark.parametrize("H,dtype,n,T", [(32, "bf16", 1000, 20), (64, "bf16", 700, 9),
+                                         (64, "fp8", 1300, 13), (4, "fp32", 333, 7)])
+def test_score_matrix(H, dtype, n, T):
+    """Exhaustive score matrix (tensor-core and SIMT paths) vs float64,
+    with the causal mask; ragged key and query counts."""
+    d = 32 if dtype == "fp32" else 128
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=n, T=T, d=d, H=H, M=64, key_dtype=dtype,
+                  q_dtype="fp32" if dtype == "fp32" else "bf16", window=256, refit_period=0,
+                  budget=512, k=16)
+    gpu, orc = P.make_pair(wl, max_keys=n)
+    kd, ks, kv = P.keys_inputs(wl, 0, n)
+    gpu.append_keys(kd, ks)
+    orc.append(kv)
+    pos0 = n - T - 3
+    qd, wd, qv, wv = P.query_inputs(wl, 0, T)
+    sc = gpu.debug_scores(qd, wd, pos0).cpu().numpy()
+    for i in range(T):
+        t = pos0 + i
+        exact = O.indexer_score(qv[i], wv[i], kv[:t + 1])
+        tol = P.score_tol(qv[i], wv[i], kv[:t + 1])
+        assert np.all(np.abs(sc[i, :t + 1] - exact) <= tol + 1e-6)
+        assert np.all(np.isneginf(sc[i, t + 1:]))
+    gpu.close()
+
+
+def test_errors_are_reported():
+    from ivf_top_key_b200 import AiError
+    wl = S.scaled(S.WORKLOADS["tiny_fp32_L4k"], L=1024)
+    gpu, _ = P.make_pair(wl)
+    kd, ks, _ = P.keys_inputs(wl, 0, 512)
+    gpu.append_keys(kd, ks)
+    qd, wd, _, _ = P.query_inputs(wl, 0, 512)
+    with pytest.raises(AiError, match="CAUSALITY"):
+        gpu.route_refine(qd, wd, 1, wl.k, wl.budget)
+    with pytest.raises(AiError, match="ARG"):
+        gpu.route_refine(qd, wd, 0, wl.k + 1, wl.budget)
+    with pytest.raises(AiError, match="ARG"):
+        gpu.route_refine(qd, wd, 0, wl.k, wl.budget + 1)
+    big = torch.zeros((2000, wl.d), dtype=torch.float32, device="cuda")
+    with pytest.raises(AiError, match="OOM"):
+        gpu.append_keys(big)
+    gpu.route_refine(qd, wd, 0, wl.k, wl.budget)
+    gpu.sync()
+    gpu.close()
+
+
+def test_checkpoint_rollback_repeats_a_chunk_exactly():
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=8192, T=2048, refit_period=4096,
+                  budget=2048, k=128, M=128)
+    gpu, _ = P.make_pair(wl)
+    for c in range(3):
+        kd, ks, _ = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+    gpu.publish()
+    gpu.checkpoint()
+    kd, ks, _ = P.keys_inputs(wl, 3 * wl.T, 4 * wl.T)
+    qd, wd, _, _ = P.query_inputs(wl, 3 * wl.T, 4 * wl.T)
+    outs = []
+    for rep in range(2):
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+        out = gpu.route_refine(qd, wd, 3 * wl.T, wl.k, wl.budget)
+        gpu.publish()
+        gpu.sync()
+        outs.append((out.cpu().numpy(), gpu.export_index()))
+        gpu.rollback()
+    assert np.array_equal(outs[0][0], outs[1][0])
+    assert np.array_equal(outs[0][1]["members"], outs[1][1]["members"])
+    gpu.close()
