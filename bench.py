@@ -1,0 +1,542 @@
+"""Benchmark: selected query-tokens/s of causal IVF route+refine on B200.
+
+One step = the whole hot path over the last R/T prefill chunks of the
+workload (one refit period): per chunk, append its keys, seal its windows
+(the refit they trigger runs on the side stream) and route + refine its
+queries; then publish the refit.  The index state before those chunks is
+restored (checkpoint/rollback) between steps, and L2 is flushed between
+steps.  Inputs are seeded synthetic data of the workload's shapes.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload glm_bf16_L128k]
+
+N > 1 runs under torch.distributed.run: every rank holds an independent
+request (its own seed) and runs the same step; no collective is on the data
+path (weak scaling).  `--impl reference` times the float64 CPU oracle on the
+host cores (rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth import workloads as S  # noqa: E402
+
+METRIC = "selected query-tokens/s at 128K-1M prefix (route+refine) & recall vs exhaustive"
+UNIT = "query-tokens/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="glm_bf16_L128k", choices=sorted(S.WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-sample", type=int, default=48, help="queries timed per oracle step")
+    return p.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def chunks_per_step(wl):
+    """A step spans one refit period (R / T chunks) so that it holds the
+    refit the method runs every R tokens."""
+    return max(1, wl.refit_period // wl.T) if wl.refit_period else 1
+
+
+def config_block(wl, n):
+    return {"workload": wl.name, "chunks_per_step": chunks_per_step(wl),
+            "queries_per_step": chunks_per_step(wl) * wl.T, "prefix_tokens": wl.L, "chunk_queries": wl.T, "heads": wl.H,
+            "head_dim": wl.d, "key_dtype": wl.key_dtype, "k": wl.k, "budget_C": wl.budget,
+            "window_W": wl.window, "clusters_per_window": wl.clusters_per_window,
+            "refit_period_R": wl.refit_period, "sinks": wl.n_sinks,
+            "step": "last R/T chunks: per chunk append + seal (+side-stream refit) + route/refine; then publish",
+            "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{n}"}
+
+
+def wl_for_rank(name, rank):
+    return S.scaled(S.WORKLOADS[name], seed=rank)
+
+
+# ------------------------------------------------------------- inputs --
+
+def bf16_dev(x, device):
+    import torch
+    bits = S.to_bf16_bits(x)
+    return torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def chunk_keys_dev(wl, p0, p1, device):
+    import torch
+    kf = S.keys_f64(wl, p0, p1)
+    if wl.key_dtype == "fp32":
+        return torch.from_numpy(kf.astype(np.float32)).to(device), None
+    kb = bf16_dev(kf, device)
+    if wl.key_dtype == "bf16":
+        return kb, None
+    from ivf_top_key_b200 import quantize_fp8
+    return quantize_fp8(kb)
+
+
+def queries_dev(wl, p0, p1, device):
+    import torch
+    q, w = S.queries_f64(wl, p0, p1)
+    wd = torch.from_numpy(w.astype(np.float32)).to(device)
+    if wl.q_dtype == "fp32":
+        return torch.from_numpy(q.astype(np.float32)).to(device), wd
+    return bf16_dev(q, device), wd
+
+
+# ------------------------------------------------------------- clocks --
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ roofline --
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def traffic_from_profile(kernel_src: str, profile_md: str):
+    """DRAM bytes per launch recorded by an ncu capture summary, if the
+    kernel source has not changed since (sha256 prefix recorded there)."""
+    try:
+        txt = open(profile_md).read()
+        src = open(kernel_src, "rb").read()
+    except OSError:
+        return None
+    h = hashlib.sha256(src).hexdigest()[:16]
+    m_h = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+    m_t = re.search(r"dram_bytes_per_launch_fullsize:\s*([0-9.eE+]+)", txt)
+    if not m_h or not m_t or m_h.group(1) != h:
+        return None
+    return float(m_t.group(1))
+
+
+# ------------------------------------------------------------ our arm --
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from ivf_top_key_b200 import AttentionIndex, C as capi
+    wl = wl_for_rank(args.workload, rank)
+    T, L = wl.T, wl.L
+    ncs = chunks_per_step(wl)
+    p_first = L - ncs * T          # first position of the timed chunks
+    pos0 = L - T                   # last chunk (recall is measured on it)
+    idx = AttentionIndex(d=wl.d, H=wl.H, key_dtype=wl.key_dtype, q_dtype=wl.q_dtype,
+                         n_sinks=wl.n_sinks, window=wl.window,
+                         clusters_per_window=wl.clusters_per_window,
+                         refit_period=wl.refit_period, refit_new_seeds=0,
+                         refit_seed_window=0, seal_iters=wl.seal_iters, async_refit=True,
+                         max_query_chunk=T, max_budget=wl.budget, max_k=wl.k, max_keys=L,
+                         seed=wl.seed)
+    # prefix before the timed chunks (untimed setup)
+    for c in range(wl.n_chunks - ncs):
+        kd, ks = chunk_keys_dev(wl, c * T, (c + 1) * T, dev)
+        idx.append_keys(kd, ks)
+        idx.seal()
+    idx.publish()
+    idx.sync()
+    idx.checkpoint()
+    chunks = []
+    for c in range(ncs):
+        a = p_first + c * T
+        kd, ks = chunk_keys_dev(wl, a, a + T, dev)
+        qd, wd = queries_dev(wl, a, a + T, dev)
+        chunks.append((a, kd, ks, qd, wd))
+    kd, ks, qd, wd = chunks[-1][1:]
+    out = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for a, kd_, ks_, qd_, wd_ in chunks:
+            idx.append_keys(kd_, ks_)
+            idx.seal()
+            idx.route_refine(qd_, wd_, a, wl.k, wl.budget, out=out)
+        idx.publish()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        idx.rollback()
+        step()
+    idx.sync()
+    idx.profile_read()
+    idx.profile(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = capi.ai_kernel_launches()
+    with Clocks(local) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            idx.rollback()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    launches = capi.ai_kernel_launches() - launches0
+    idx.profile(False)
+    phases = idx.profile_read()
+    idx.sync()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(np.sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    units = T * ncs                # query tokens per step
+    value = world * units * args.steps / (total_ms / 1e3)
+
+    # recall vs the in-library exhaustive selection (after the last step)
+    exh = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    idx.select_exhaustive(qd, wd, pos0, wl.k, out=exh)
+    e1.record(stream)
+    idx.sync()
+    exh_ms = e0.elapsed_time(e1)
+    rows = torch.arange(T, device=dev, dtype=torch.int64)[:, None] * (L + 1)
+    sel_c = (out.to(torch.int64) + rows)[out >= 0]
+    exh_c = (exh.to(torch.int64) + rows)[exh >= 0]
+    recall = float(torch.isin(exh_c, sel_c).sum().item() / max(1, exh_c.numel()))
+
+    # roofline of the dominant kernel (live phase events)
+    peaks, peak_kind = measured_peaks()
+    st = idx.stats()
+    nC = st["n_clusters"]
+    esz = {"bf16": 2, "fp8": 1, "fp32": 4}[wl.key_dtype]
+    row_bytes = wl.d * esz + (4 if wl.key_dtype == "fp8" else 0)
+    refine_ms, refine_n = phases["refine"]
+    route_ms, route_n = phases["route"]
+    # algorithmic bytes per refine launch: gathered candidate rows, query,
+    # weights, cluster-score row, CSR offsets, output ids
+    qbytes = wl.H * wl.d * (2 if wl.q_dtype == "bf16" else 4)
+    refine_bytes = T * (wl.budget * row_bytes + qbytes + wl.H * 4 + nC * 8 + wl.k * 4)
+    # (nC: clusters of the final chunk's index; per launch = one chunk of T queries)
+    route_flops = 2.0 * T * wl.H * wl.d * nC
+    dom = max(phases.items(), key=lambda kv: kv[1][0])[0]
+    roofline = None
+    if refine_n:
+        avg = refine_ms / refine_n / 1e3
+        ach = refine_bytes / avg / 1e9
+        traffic = traffic_from_profile(os.path.join(ROOT, "ivf_top_key_b200", "csrc", "route_refine.cu"),
+                                       os.path.join(ROOT, "profiles", f"refine_{wl.name}.md"))
+        roofline = {"kernel": "k_refine_tc (candidate fill + gathered rescore + top-k)",
+                    "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                    "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                    "algorithmic_bytes_per_launch": refine_bytes,
+                    "avg_launch_ms": round(refine_ms / refine_n, 4)}
+    route_roof = None
+    if route_n:
+        avg = route_ms / route_n / 1e3
+        tf = route_flops / avg / 1e12
+        route_roof = {"kernel": "k_scores_tc (route GEMM)", "bound": "tensor",
+                      "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": round(tf / peaks["bf16_tflops"], 4),
+                      "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                      "avg_launch_ms": round(route_ms / route_n, 4)}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        for a, kd_, ks_, qd_, wd_ in chunks:
+            host.append((a, kd_.cpu().pin_memory(), ks_.cpu().pin_memory() if ks_ is not None else None,
+                         qd_.cpu().pin_memory(), wd_.cpu().pin_memory(),
+                         torch.empty((T, wl.k), dtype=torch.int32).pin_memory()))
+        kd2, qd2, wd2 = torch.empty_like(kd), torch.empty_like(qd), torch.empty_like(wd)
+        sd2 = torch.empty_like(ks) if ks is not None else None
+        out2 = torch.empty_like(out)
+
+        def e2e_step():
+            for a, kh, sh, qh, wh, oh in host:
+                kd2.copy_(kh, non_blocking=True)
+                if sh is not None:
+                    sd2.copy_(sh, non_blocking=True)
+                qd2.copy_(qh, non_blocking=True)
+                wd2.copy_(wh, non_blocking=True)
+                idx.append_keys(kd2, sd2)
+                idx.seal()
+                idx.route_refine(qd2, wd2, a, wl.k, wl.budget, out=out2)
+                oh.copy_(out2, non_blocking=True)
+            idx.publish()
+
+        for _ in range(max(1, args.warmup)):
+            idx.rollback()
+            e2e_step()
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            idx.rollback()
+            ee[i][0].record(stream)
+            e2e_step()
+            ee[i][1].record(stream)
+        torch.cuda.synchronize()
+        e_ms = float(np.sum([a.elapsed_time(b) for a, b in ee]))
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(kh.numel() * kh.element_size() + qh.numel() * qh.element_size() +
+                  wh.numel() * wh.element_size() + (sh.numel() * 4 if sh is not None else 0)
+                  for _, kh, sh, qh, wh, _ in host)
+        d2h = sum(oh.numel() * 4 for *_, oh in host)
+        e2e = {"value": world * units * args.steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / args.steps}
+
+    idx.close()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(wl, args.cpu_sample)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.key_dtype, "data": "synthetic (seeded Gaussian-mixture keys/queries)",
+            "config": config_block(wl, world),
+            "recall_vs_exhaustive": round(recall, 4),
+            "exhaustive": {"value": round(T / (exh_ms / 1e3), 1), "unit": UNIT,
+                           "ms_per_chunk": exh_ms, "note": "in-library exhaustive selection of the final chunk",
+                           "route_refine_speedup": round(value / world / (T / (exh_ms / 1e3)), 2)},
+            "roofline": roofline, "roofline_route_gemm": route_roof,
+            "phases_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
+            "dominant_phase": dom,
+            "gpu_launches": int(launches), "gpu_launches_per_step": launches / args.steps,
+            "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+            "wall_s_timed_region": round(t_wall, 3),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------- oracle arm --
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_prefix(wl):
+    from oracle import ai_oracle as O
+    orc = O.OracleIndex(d=wl.d, n_sinks=wl.n_sinks, window=wl.window,
+                        clusters_per_window=wl.clusters_per_window,
+                        refit_period=wl.refit_period, refit_new_seeds=wl.refit_new_seeds,
+                        refit_seed_window=wl.refit_seed_window, seal_iters=wl.seal_iters,
+                        seed=wl.seed)
+    keys = oracle_keys(wl, 0, wl.L)
+    for c in range(wl.n_chunks - chunks_per_step(wl)):
+        orc.append(keys[c * wl.T:(c + 1) * wl.T])
+        orc.seal()
+    orc.publish()
+    return orc, keys
+
+
+def oracle_keys(wl, p0, p1):
+    from oracle import ai_oracle as O
+    kf = S.keys_f64(wl, p0, p1)
+    if wl.key_dtype == "fp32":
+        return kf.astype(np.float32).astype(np.float64)
+    vals = S.bf16_bits_to_f64(S.to_bf16_bits(kf))
+    if wl.key_dtype == "bf16":
+        return vals
+    codes, sc = O.quantize_fp8_keys(vals.astype(np.float32))
+    return codes * sc.astype(np.float64)[:, None]
+
+
+def oracle_queries(wl, p0, p1):
+    q, w = S.queries_f64(wl, p0, p1)
+    w = w.astype(np.float32).astype(np.float64)
+    if wl.q_dtype == "fp32":
+        return q.astype(np.float32).astype(np.float64), w
+    return S.bf16_bits_to_f64(S.to_bf16_bits(q)), w
+
+
+def oracle_step(orc0, keys, wl, sample_idx, qv, wv):
+    """One oracle step over the timed chunks: maintenance (append, seal,
+    refit) of every chunk plus route+refine of a sample of their queries.
+    sample_idx indexes the queries of the timed chunks.  Returns
+    (maintenance seconds, seconds per query)."""
+    import copy
+    orc = copy.deepcopy(orc0)
+    ncs = chunks_per_step(wl)
+    p_first = wl.L - ncs * wl.T
+    t_m = t_q = 0.0
+    nq = 0
+    for c in range(ncs):
+        a = p_first + c * wl.T
+        t0 = time.perf_counter()
+        orc.append(keys[a:a + wl.T])
+        orc.seal()
+        t_m += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        for i in sample_idx:
+            if c * wl.T <= i < (c + 1) * wl.T:
+                orc.route_refine(qv[i], wv[i], p_first + int(i), wl.k, wl.budget)
+                nq += 1
+        t_q += time.perf_counter() - t0
+    return t_m, t_q / max(nq, 1)
+
+
+def oracle_baseline(wl, n_sample):
+    orc, keys = _oracle_prefix(wl)
+    nq = chunks_per_step(wl) * wl.T
+    qv, wv = oracle_queries(wl, wl.L - nq, wl.L)
+    rng = np.random.default_rng(0)
+    sample = np.sort(rng.choice(nq, size=min(n_sample, nq), replace=False))
+    t_m, t_q = oracle_step(orc, keys, wl, sample, qv, wv)
+    step_s = t_m + nq * t_q
+    return {"value": round(nq / step_s, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": (f"last {nq} queries of {wl.name} (one step): full maintenance (append, "
+                       f"seal, refit) timed ({t_m:.2f} s) + {len(sample)} sampled queries' "
+                       f"route+refine ({t_q * 1e3:.1f} ms each), extrapolated to the step")}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    wl = wl_for_rank(args.workload, 0)
+    orc, keys = _oracle_prefix(wl)
+    nq = chunks_per_step(wl) * wl.T
+    qv, wv = oracle_queries(wl, wl.L - nq, wl.L)
+    rng = np.random.default_rng(0)
+    n = max(4, min(args.cpu_sample, nq) // 4)
+    for _ in range(args.warmup):
+        oracle_step(orc, keys, wl, rng.choice(nq, size=2, replace=False), qv, wv)
+    tot = 0.0
+    t_ms, t_qs = [], []
+    for _ in range(args.steps):
+        sample = np.sort(rng.choice(nq, size=n, replace=False))
+        t_m, t_q = oracle_step(orc, keys, wl, sample, qv, wv)
+        t_ms.append(t_m)
+        t_qs.append(t_q)
+        tot += t_m + nq * t_q
+    value = nq * args.steps / tot
+    cores = _threads()
+    sample_desc = (f"per step: maintenance of the last {nq} positions of {wl.name} "
+                   f"(mean {np.mean(t_ms):.2f} s) + {n} sampled queries' route+refine "
+                   f"(mean {np.mean(t_qs) * 1e3:.1f} ms each), extrapolated to the step")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Gaussian-mixture keys/queries)",
+        "config": config_block(wl, world), "impl": "reference",
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample_desc,
+                         "value": round(value, 2), "unit": UNIT},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

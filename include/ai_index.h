@@ -178,6 +178,25 @@ int ai_debug_scores(ai_handle h, const void* q_dev, const float* w_dev, int64_t 
 int ai_checkpoint(ai_handle h);
 int ai_rollback(ai_handle h);
 
+/* ----------------------------------------------------------- profiling */
+/* Phase timing with CUDA events recorded on the stream each phase runs on
+ * (refit: the side stream when async).  Off by default.                    */
+#define AI_PHASE_ROUTE 0       /* cluster-score GEMM                          */
+#define AI_PHASE_REFINE 1      /* candidate fill + rescore + top-k kernel     */
+#define AI_PHASE_SEAL 2        /* seal k-means (+ encoder)                    */
+#define AI_PHASE_REFIT 3       /* refit kernels (+ encoder)                   */
+#define AI_PHASE_PUBLISH 4     /* wait for the refit + tail copy              */
+#define AI_PHASE_EXH_SCORES 5  /* exhaustive score GEMM                       */
+#define AI_PHASE_EXH_TOPK 6    /* exhaustive row top-k                        */
+#define AI_N_PHASES 7
+int ai_profile_enable(ai_handle h, int enable);
+/* Waits for the handle's streams, then writes the summed milliseconds and
+ * the number of timed launches per phase (arrays of AI_N_PHASES, nullable)
+ * since the last read, and resets them.                                   */
+int ai_profile_read(ai_handle h, double* ms_out, int64_t* launches_out);
+/* Number of kernels this library has launched in the process.             */
+long long ai_kernel_launches(void);
+
 /* fp8 store helper: per-key scale = amax / 448 and E4M3 codes (round to
  * nearest even, saturating) from bf16 keys [n, d].  Enqueued on
  * cuda_stream.                                                            */

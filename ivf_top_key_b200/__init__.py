@@ -106,6 +106,13 @@ class AttentionIndex:
         out = torch.empty((q.shape[0], n), dtype=torch.float32, device=q.device)
         return C.ai_debug_scores(self.h, q, w, pos0, out)
 
+    def profile(self, enable: bool = True):
+        C.ai_profile_enable(self.h, enable)
+
+    def profile_read(self) -> dict:
+        """{phase: (milliseconds, timed launches)} since the last read."""
+        return C.ai_profile_read(self.h)
+
     def checkpoint(self):
         C.ai_checkpoint(self.h)
 

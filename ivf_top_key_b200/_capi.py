@@ -28,8 +28,10 @@ EXPORTED = [
     "ai_index_create", "ai_index_destroy", "ai_append_keys", "ai_seal", "ai_refit",
     "ai_publish", "ai_route_refine", "ai_select_exhaustive", "ai_sync", "ai_last_error",
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
-    "ai_checkpoint", "ai_rollback", "ai_quantize_fp8",
+    "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
+    "ai_kernel_launches",
 ]
+PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
 
 
 class AiConfig(ctypes.Structure):
@@ -80,11 +82,15 @@ def _load():
         "ai_checkpoint": [vp],
         "ai_rollback": [vp],
         "ai_quantize_fp8": [vp, i64, i32, vp, vp, vp],
+        "ai_profile_enable": [vp, ctypes.c_int],
+        "ai_profile_read": [vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
         f.argtypes = args
         f.restype = ctypes.c_int
+    lib.ai_kernel_launches.argtypes = []
+    lib.ai_kernel_launches.restype = ctypes.c_longlong
     lib.ai_last_error.argtypes = []
     lib.ai_last_error.restype = ctypes.c_char_p
     return lib
@@ -204,6 +210,22 @@ def ai_quantize_fp8(keys_bf16, codes, scales, stream=None):
     _check(_lib.ai_quantize_fp8(_ptr(keys_bf16), keys_bf16.shape[0], keys_bf16.shape[1],
                                 _ptr(codes), _ptr(scales), _stream(stream)))
     return codes, scales
+
+
+def ai_profile_enable(h, enable: bool = True):
+    _check(_lib.ai_profile_enable(h, int(enable)))
+
+
+def ai_profile_read(h) -> dict:
+    import numpy as np
+    ms = np.zeros(len(PHASES), dtype=np.float64)
+    n = np.zeros(len(PHASES), dtype=np.int64)
+    _check(_lib.ai_profile_read(h, ms.ctypes.data_as(ctypes.c_void_p), n.ctypes.data_as(ctypes.c_void_p)))
+    return {p: (float(ms[i]), int(n[i])) for i, p in enumerate(PHASES)}
+
+
+def ai_kernel_launches() -> int:
+    return int(_lib.ai_kernel_launches())
 
 
 def ai_last_error() -> str:

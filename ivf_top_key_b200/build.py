@@ -1,6 +1,7 @@
 """Build libai_index.so (sm_100a) in-tree with nvcc.
 
-Usage: python -m ivf_top_key_b200.build [--force]
+Usage: python ivf_top_key_b200/build.py [--force]
+(run by path: importing the package loads the library this script builds)
 """
 from __future__ import annotations
 

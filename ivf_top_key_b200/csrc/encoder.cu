@@ -95,6 +95,7 @@ cudaError_t launch_encoder(const EncoderArgs& a, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   if (a.d > 1024) return cudaErrorInvalidValue;
   const size_t smem = static_cast<size_t>(a.d * 3 + 3 * a.d + 1) * 8;
+  count_launch();
   k_encoder<<<n, a.d, smem, st>>>(a);
   return cudaGetLastError();
 }

@@ -27,7 +27,15 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <atomic>
+
 using namespace aiidx;
+
+namespace aiidx {
+static std::atomic<long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+long long kernel_launches() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace aiidx
 
 namespace {
 
@@ -129,6 +137,11 @@ struct Buffer {
   std::vector<Version> versions;
 };
 
+struct ProfRec {
+  int phase;
+  cudaEvent_t a, b;
+};
+
 struct Checkpoint {
   bool valid = false;
   int64_t n_keys = 0, n_windows = 0, n_refits = 0, refit_n_old = 0, n_codes_bf16 = 0;
@@ -186,6 +199,12 @@ struct ai_index {
   int* err_dev = nullptr;
   int* err_host = nullptr;         // pinned
   float* enc_wts = nullptr;
+  // phase timing (CUDA events on the launching stream)
+  bool prof = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> ev_pool;
+  double prof_ms[AI_N_PHASES] = {};
+  int64_t prof_n[AI_N_PHASES] = {};
   // checkpoint copies of the per-key bounds
   Checkpoint ck;
   int32_t* ck_assign = nullptr;
@@ -196,6 +215,29 @@ struct ai_index {
 namespace {
 
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+cudaEvent_t pool_event(ai_index* h) {
+  if (!h->ev_pool.empty()) {
+    cudaEvent_t e = h->ev_pool.back();
+    h->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Open / close a timed phase on stream st (no-op unless profiling is on).
+int prof_begin(ai_index* h, int phase, cudaStream_t st) {
+  if (!h->prof) return -1;
+  ProfRec r{phase, pool_event(h), pool_event(h)};
+  cudaEventRecord(r.a, st);
+  h->recs.push_back(r);
+  return static_cast<int>(h->recs.size()) - 1;
+}
+void prof_end(ai_index* h, int idx, cudaStream_t st) {
+  if (idx >= 0) cudaEventRecord(h->recs[idx].b, st);
+}
 
 bool tc_route(const ai_index* h) {
   return h->cfg.q_dtype == AI_BF16 && h->cfg.d == 128 && (h->cfg.H == 32 || h->cfg.H == 64);
@@ -230,9 +272,13 @@ int route_scores(ai_index* h, const void* q, const float* w, int T, int64_t nC) 
     const int64_t atiles = (nC + 127) / 128;
     int64_t apc = (atiles * qtiles + 4 * h->num_sms - 1) / (4 * h->num_sms);
     apc = std::max<int64_t>(1, std::min(apc, atiles));
+    const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
+    prof_end(h, pi, h->main);
   } else {
+    const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
     CK(launch_scores_simt(b.reps, KD_BF16, q, h->cfg.q_dtype == AI_BF16, h->cfg.d, h->cfg.H, sa, h->main));
+    prof_end(h, pi, h->main);
   }
   return AI_OK;
 }
@@ -269,6 +315,7 @@ int check_queries(const ai_index* h, const void* q, const float* w, int64_t pos0
 
 int publish(ai_index* h) {
   if (!h->pending) return AI_OK;
+  const int pp = prof_begin(h, AI_PHASE_PUBLISH, h->main);
   CK(cudaStreamWaitEvent(h->main, h->ev_refit, 0));
   Buffer& A = h->buf[h->active];
   Buffer& B = h->buf[h->pending_buf];
@@ -297,6 +344,7 @@ int publish(ai_index* h) {
     CK(cudaMemcpyAsync(B.members + B.n_members, A.members + src_mem0, tail_w * W * sizeof(int32_t),
                        cudaMemcpyDeviceToDevice, h->main));
     const int n = static_cast<int>(nc + 1);
+    count_launch();
     k_shift_offsets<<<(n + 255) / 256, 256, 0, h->main>>>(A.offsets + c0, B.offsets + K, n,
                                                            static_cast<int32_t>(B.n_members - src_mem0));
     CK(cudaGetLastError());
@@ -305,6 +353,7 @@ int publish(ai_index* h) {
     B.nC = K + nc;
     B.n_members += tail_w * W;
   }
+  prof_end(h, pp, h->main);
   h->active = h->pending_buf;
   h->pending = false;
   return AI_OK;
@@ -363,6 +412,7 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
   ra.scan_list = h->scan_list;
   ra.n_scan = h->scan_words;
   ra.err = h->err_dev;
+  const int pr = prof_begin(h, AI_PHASE_REFIT, st);
   CK(launch_refit(ra, h->max_tiles, st, h->nscan_host));
   if (h->enc_wts) {
     EncoderArgs ea{};
@@ -380,6 +430,7 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
     ea.err = h->err_dev;
     CK(launch_encoder(ea, st));
   }
+  prof_end(h, pr, st);
   CK(cudaEventRecord(h->ev_refit, st));
   h->pending = true;
   h->pending_buf = target;
@@ -412,6 +463,7 @@ int seal_group(ai_index* h, int64_t w0, int64_t nw) {
   sa.centroids = A.centroids;
   sa.reps = A.reps;
   sa.err = h->err_dev;
+  const int ps = prof_begin(h, AI_PHASE_SEAL, h->main);
   CK(launch_seal(sa, h->main));
   if (h->enc_wts) {
     EncoderArgs ea{};
@@ -429,6 +481,7 @@ int seal_group(ai_index* h, int64_t w0, int64_t nw) {
     ea.err = h->err_dev;
     CK(launch_encoder(ea, h->main));
   }
+  prof_end(h, ps, h->main);
   for (int64_t w = w0; w < w0 + nw; ++w) {
     A.nC += m;
     A.n_members += W;
@@ -478,10 +531,14 @@ int exhaustive_scores(ai_index* h, const void* q, const float* w, int64_t pos0, 
     const int64_t atiles = (nA + 127) / 128;
     int64_t apc = (atiles * qtiles + 4 * h->num_sms - 1) / (4 * h->num_sms);
     apc = std::max<int64_t>(1, std::min(apc, atiles));
+    const int pe = prof_begin(h, AI_PHASE_EXH_SCORES, h->main);
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
+    prof_end(h, pe, h->main);
   } else {
+    const int pe = prof_begin(h, AI_PHASE_EXH_SCORES, h->main);
     const int kd = h->cfg.key_dtype == AI_FP8E4M3 ? KD_FP8 : (h->cfg.key_dtype == AI_BF16 ? KD_BF16 : KD_FP32);
     CK(launch_scores_simt(h->keys, kd, q, h->cfg.q_dtype == AI_BF16, h->cfg.d, h->cfg.H, sa, h->main));
+    prof_end(h, pe, h->main);
   }
   return AI_OK;
 }
@@ -495,7 +552,8 @@ const char* ai_last_error(void) { return g_err.c_str(); }
 int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   if (!cfg || !out) return fail(AI_ERR_ARG, "null config or output");
   const ai_config& c = *cfg;
-  if (c.d <= 0 || c.d > 1024 || c.H <= 0 || c.H > 64) return fail(AI_ERR_ARG, "bad d or H");
+  if (c.d <= 0 || c.d > 1024 || c.d % 8 != 0 || c.H <= 0 || c.H > 64)
+    return fail(AI_ERR_ARG, "bad d (a multiple of 8 up to 1024) or H (1..64)");
   if (c.key_dtype < 0 || c.key_dtype > 2) return fail(AI_ERR_ARG, "bad key dtype");
   if (!(c.q_dtype == AI_BF16 || (c.q_dtype == AI_FP32 && c.key_dtype == AI_FP32)))
     return fail(AI_ERR_ARG, "queries must be bf16 (or fp32 with fp32 keys)");
@@ -628,6 +686,11 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->ck_assign);
   cudaFree(h->ck_ub);
   cudaFree(h->ck_lb);
+  for (auto& r : h->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->ev_pool) cudaEventDestroy(e);
   if (h->ev_main) cudaEventDestroy(h->ev_main);
   if (h->ev_refit) cudaEventDestroy(h->ev_refit);
   if (h->side) cudaStreamDestroy(h->side);
@@ -733,7 +796,9 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
     CK(cudaMallocAsync(reinterpret_cast<void**>(&tmp_out), static_cast<size_t>(T) * k * 4, h->main));
     ra.out = tmp_out;
   }
+  const int pf = prof_begin(h, AI_PHASE_REFINE, h->main);
   CK(launch_refine(ra, vt, tc_keys(h), h->num_sms, h->main));
+  prof_end(h, pf, h->main);
   if (tmp_out) CK(cudaFreeAsync(tmp_out, h->main));
   return AI_OK;
 }
@@ -779,7 +844,9 @@ int ai_select_exhaustive(ai_handle h, const void* q_dev, const float* w_dev, int
     ta.out = out_dev + b0 * k;
     ta.out_scores = out_scores_dev ? out_scores_dev + b0 * k : nullptr;
     ta.err = h->err_dev;
+    const int pt = prof_begin(h, AI_PHASE_EXH_TOPK, h->main);
     CK(launch_row_topk(ta, h->main));
+    prof_end(h, pt, h->main);
   }
   return AI_OK;
 }
@@ -790,6 +857,7 @@ int ai_debug_scores(ai_handle h, const void* q_dev, const float* w_dev, int64_t 
   int rc = check_queries(h, q_dev, w_dev, pos0, T, 1);
   if (rc) return rc;
   const int64_t n = static_cast<int64_t>(T) * h->n_keys;
+  count_launch();
   k_fill<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 65535)), 256, 0, h->main>>>(out_dev, n, -INFINITY);
   CK(cudaGetLastError());
   return exhaustive_scores(h, q_dev, w_dev, pos0, T, out_dev, h->n_keys);
@@ -909,6 +977,37 @@ int ai_rollback(ai_handle h) {
   CK(cudaStreamWaitEvent(h->side, h->ev_main, 0));
   return AI_OK;
 }
+
+int ai_profile_enable(ai_handle h, int enable) {
+  if (!h) return fail(AI_ERR_ARG, "null handle");
+  h->prof = enable != 0;
+  return AI_OK;
+}
+
+int ai_profile_read(ai_handle h, double* ms_out, int64_t* launches_out) {
+  if (!h) return fail(AI_ERR_ARG, "null handle");
+  CK(cudaStreamSynchronize(h->main));
+  CK(cudaStreamSynchronize(h->side));
+  for (auto& r : h->recs) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      h->prof_ms[r.phase] += ms;
+      h->prof_n[r.phase] += 1;
+    }
+    h->ev_pool.push_back(r.a);
+    h->ev_pool.push_back(r.b);
+  }
+  h->recs.clear();
+  for (int i = 0; i < AI_N_PHASES; ++i) {
+    if (ms_out) ms_out[i] = h->prof_ms[i];
+    if (launches_out) launches_out[i] = h->prof_n[i];
+    h->prof_ms[i] = 0.0;
+    h->prof_n[i] = 0;
+  }
+  return AI_OK;
+}
+
+long long ai_kernel_launches(void) { return aiidx::kernel_launches(); }
 
 int ai_quantize_fp8(const uint16_t* keys_bf16_dev, int64_t n, int32_t d, uint8_t* codes_dev,
                     float* scales_dev, void* cuda_stream) {

@@ -7,6 +7,10 @@
 
 namespace aiidx {
 
+// Kernel launches made by this library (all handles, all streams).
+void count_launch();
+long long kernel_launches();
+
 // ---------------------------------------------------------- score matrices
 struct ScoreArgs {
   int nA;                  // rows of A

@@ -41,6 +41,7 @@ cudaError_t launch_quantize_fp8(const uint16_t* keys_bf16, int64_t n, int d, uin
                                 float* scales, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const int64_t threads = n * 32;
+  count_launch();
   k_quantize<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(keys_bf16, n, d, codes, scales);
   return cudaGetLastError();
 }
@@ -51,6 +52,7 @@ cudaError_t launch_fp8_codes_to_bf16(const uint8_t* codes, int64_t n, int d, uin
   if (e <= 0) return cudaSuccess;
   int64_t blocks = (e + 255) / 256;
   if (blocks > 65535 * 8) blocks = 65535 * 8;
+  count_launch();
   k_codes_to_bf16<<<static_cast<unsigned>(blocks), 256, 0, st>>>(codes, e, out);
   return cudaGetLastError();
 }

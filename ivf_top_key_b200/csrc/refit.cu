@@ -434,25 +434,40 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   unsigned long long* mdb = reinterpret_cast<unsigned long long*>(a.n_scan + 2);
   cudaMemsetAsync(a.n_scan, 0, 16, st);
   const int64_t ce = static_cast<int64_t>(a.K) * a.d;
+  count_launch();
   k_init<<<static_cast<unsigned>((ce + 255) / 256 < 4096 ? (ce + 255) / 256 : 4096), 256, 0, st>>>(a);
-  if (a.K_prev > 0 && a.K > a.K_prev) k_seed_lb<<<(a.K_prev * 32 + 255) / 256, 256, 0, st>>>(a);
+  if (a.K_prev > 0 && a.K > a.K_prev) {
+    count_launch();
+    k_seed_lb<<<(a.K_prev * 32 + 255) / 256, 256, 0, st>>>(a);
+  }
   const unsigned gk = static_cast<unsigned>((n + 255) / 256);
+  count_launch();
   k_test<<<gk, 256, 0, st>>>(a);
   // the scan list length is only known on the device: fixed grids that stride
   const int64_t sblocks = (n + kSK - 1) / kSK;
+  count_launch();
   k_scan<<<static_cast<unsigned>(sblocks < 1184 ? sblocks : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
   // recheck list lives after the scan list (capacity n)
+  count_launch();
   k_recheck<<<static_cast<unsigned>(n < 1184 ? n : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
+  count_launch();
   k_zero_counts<<<(a.K + 255) / 256, 256, 0, st>>>(a);
+  count_launch();
   k_count<<<gk, 256, 0, st>>>(a);
+  count_launch();
   k_offsets<<<1, 1024, 0, st>>>(a);
   const size_t sm = static_cast<size_t>(a.K) * 4;
   cudaFuncSetAttribute(k_tile_counts, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
   cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  count_launch();
   k_tile_counts<<<static_cast<unsigned>(ntiles), 32, sm, st>>>(a);
+  count_launch();
   k_tile_base<<<(a.K + 255) / 256, 256, 0, st>>>(a, static_cast<int>(ntiles));
+  count_launch();
   k_scatter<<<static_cast<unsigned>(ntiles), 32, sm, st>>>(a);
+  count_launch();
   k_update<<<static_cast<unsigned>((static_cast<int64_t>(a.K) * 32 + 255) / 256), 256, 0, st>>>(a, mdb);
+  count_launch();
   k_bounds<<<gk, 256, 0, st>>>(a, mdb);
   if (host_nscan) cudaMemcpyAsync(host_nscan, a.n_scan, 8, cudaMemcpyDeviceToHost, st);
   return cudaGetLastError();

@@ -479,9 +479,11 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, bool tc, 
     const int grid = a.T < num_sms ? a.T : num_sms;
     if (a.H == 32) {
       cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      count_launch();
       k_refine_tc<32><<<grid, kTcThreads, smem, st>>>(a, vt);
     } else if (a.H == 64) {
       cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      count_launch();
       k_refine_tc<64><<<grid, kTcThreads, smem, st>>>(a, vt);
     } else {
       return cudaErrorInvalidValue;
@@ -492,6 +494,7 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, bool tc, 
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_refine_simt, kSimtThreads, smem);
     if (per_sm < 1) per_sm = 1;
     const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
+    count_launch();
     k_refine_simt<<<grid, kSimtThreads, smem, st>>>(a, vt);
   }
   return cudaGetLastError();

@@ -270,9 +270,11 @@ cudaError_t launch_scores_tc(const CUtensorMap& mapA, const CUtensorMap& mapB, i
   dim3 grid((n_atiles + a_tiles_per_cta - 1) / a_tiles_per_cta, (a.T + QPT - 1) / QPT);
   if (H == 32) {
     cudaFuncSetAttribute(k_scores_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    count_launch();
     k_scores_tc<32><<<grid, kThreads, kSmemBytes, st>>>(mapA, mapB, a);
   } else if (H == 64) {
     cudaFuncSetAttribute(k_scores_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    count_launch();
     k_scores_tc<64><<<grid, kThreads, kSmemBytes, st>>>(mapA, mapB, a);
   } else {
     return cudaErrorInvalidValue;
@@ -293,6 +295,7 @@ cudaError_t launch_scores_simt(const void* A, int a_dtype, const void* Q, int q_
   }
   if (last <= 0 || args.T <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>((last + kSimtRows - 1) / kSimtRows), (args.T + kSimtQ - 1) / kSimtQ);
+  count_launch();
   k_scores_simt<<<grid, 256, smem, st>>>(A, a_dtype, Q, q_is_bf16, d, H, args);
   return cudaGetLastError();
 }

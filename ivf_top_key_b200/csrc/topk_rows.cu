@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(1024) k_row_topk(RowTopkArgs a) {
 
 cudaError_t launch_row_topk(const RowTopkArgs& a, cudaStream_t st) {
   if (a.T <= 0) return cudaSuccess;
+  count_launch();
   k_row_topk<<<a.T, 1024, 0, st>>>(a);
   return cudaGetLastError();
 }

@@ -21,8 +21,8 @@ def test_header_declares_the_core_calls():
 
 
 def test_library_exports_every_declared_symbol():
-    from ivf_top_key_b200 import build
-    lib_path = build.build()
+    import __graft_entry__
+    lib_path = __graft_entry__._build_module().build()
     lib = ctypes.CDLL(lib_path)
     missing = [n for n in declared_symbols() if not hasattr(lib, n)]
     assert not missing, missing
