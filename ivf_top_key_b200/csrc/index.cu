@@ -796,8 +796,21 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
     CK(cudaMallocAsync(reinterpret_cast<void**>(&tmp_out), static_cast<size_t>(T) * k * 4, h->main));
     ra.out = tmp_out;
   }
+  CUtensorMap kmap, qmap;
+  const CUtensorMap* kmp = nullptr;
+  const CUtensorMap* qmp = nullptr;
+  if (tc_keys(h)) {
+    // bf16 rows gathered by TMA (box 64 x 1); fp8 rows are loaded by threads
+    // (the map then points at the queries and is not read)
+    const bool ok_k = h->cfg.key_dtype == AI_BF16 ? make_map(&kmap, h->keys, h->n_keys, 1)
+                                                  : make_map(&kmap, q, static_cast<int64_t>(T) * h->cfg.H, 1);
+    if (!ok_k || !make_map(&qmap, q, static_cast<int64_t>(T) * h->cfg.H, h->cfg.H))
+      return fail(AI_ERR_CUDA, "tensor map encoding failed (key store / queries)");
+    kmp = &kmap;
+    qmp = &qmap;
+  }
   const int pf = prof_begin(h, AI_PHASE_REFINE, h->main);
-  CK(launch_refine(ra, vt, tc_keys(h), h->num_sms, h->main));
+  CK(launch_refine(ra, vt, kmp, qmp, h->num_sms, h->main));
   prof_end(h, pf, h->main);
   if (tmp_out) CK(cudaFreeAsync(tmp_out, h->main));
   return AI_OK;

@@ -67,55 +67,145 @@ __device__ __forceinline__ void version_of(const VersionTable& vt, int64_t t, in
 }
 
 // Phase 1: candidate list of query qi (position t).  Returns its length.
+//
+// Sinks and the open window come first.  Then clusters in rank order
+// (score desc, id asc) until C slots are filled, the last one truncated.
+// Only the clusters that can reach the budget are ranked: a weighted
+// 2048-bin histogram of the cluster scores over [min, max] (weights =
+// cluster sizes) finds the bin where the size-weighted count from the top
+// crosses the remaining budget; clusters in that bin or above are sorted
+// exactly and the fill stops at C.
+constexpr int kNB1 = 2048;
+struct P1Smem {
+  uint32_t hist[kNB1];
+  float fred[32];
+  unsigned long long wred[16];
+  int scal[4];
+};
+
 __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, int64_t n_v,
                                 int32_t* cand, uint64_t* sortbuf, int32_t* pref,
                                 BlockScratch& bs) {
   const int C = a.C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
   const int n_s = static_cast<int>(min64(a.n_sinks, t + 1));
   const int64_t open_lo = max64(n_v, a.n_sinks);
   const int64_t n_open64 = open_lo <= t ? t + 1 - open_lo : 0;
   const int fixed = static_cast<int>(min64(C, n_s + n_open64));
-  for (int i = threadIdx.x; i < fixed; i += blockDim.x)
+  for (int i = tid; i < fixed; i += blockDim.x)
     cand[i] = i < n_s ? i : static_cast<int32_t>(open_lo + (i - n_s));
   const int rem = C - fixed;
   if (rem <= 0 || nC == 0) {
     __syncthreads();
     return fixed;
   }
+  // scratch after the sort buffer and prefix array
+  P1Smem& ps = *reinterpret_cast<P1Smem*>(
+      (reinterpret_cast<uintptr_t>(pref + kSortCap + 1) + 15) & ~uintptr_t(15));
   const float* rs = a.route + static_cast<int64_t>(qi) * a.ld_route;
   const int32_t* off = a.offsets;
-  auto size = [&](int c) -> uint32_t { return static_cast<uint32_t>(off[c + 1] - off[c]); };
-  auto key = [&](int c) -> uint32_t { return f2key(rs[c]); };
-  auto pred = [&](int c) -> bool { return off[c + 1] > off[c]; };
-  uint64_t above = 0, tot = 0;
-  const uint32_t theta = radix_select(nC, key, pred, size, static_cast<uint64_t>(rem), &above, bs, &tot);
-  const bool take_all = tot <= static_cast<uint64_t>(rem);
+  // pass A: score range and total size of the non-empty clusters
+  float vmin = INFINITY, vmax = -INFINITY;
+  unsigned long long wsum = 0;
+  for (int c = tid; c < nC; c += blockDim.x) {
+    const int sz = off[c + 1] - off[c];
+    if (sz > 0) {
+      const float v = rs[c];
+      vmin = fminf(vmin, v);
+      vmax = fmaxf(vmax, v);
+      wsum += static_cast<unsigned long long>(sz);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  }
+  if (lane == 0) {
+    ps.fred[warp] = vmin;
+    ps.fred[16 + warp] = vmax;
+    ps.wred[warp] = wsum;
+  }
+  for (int i = tid; i < kNB1; i += blockDim.x) ps.hist[i] = 0;
+  __syncthreads();
+  vmin = INFINITY;
+  vmax = -INFINITY;
+  wsum = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    vmin = fminf(vmin, ps.fred[w]);
+    vmax = fmaxf(vmax, ps.fred[16 + w]);
+    wsum += ps.wred[w];
+  }
+  const bool take_all = wsum <= static_cast<unsigned long long>(rem);
+  const float scale = vmax > vmin ? static_cast<float>(kNB1) / (vmax - vmin) : 0.f;
+  auto binof = [&](float v) -> int {
+    const int b = static_cast<int>((v - vmin) * scale);
+    return b < kNB1 - 1 ? b : kNB1 - 1;
+  };
+  int bstar = 0;
+  if (!take_all) {
+    // pass B: size-weighted histogram; the bin where the weight from the top
+    // reaches the remaining budget
+    for (int c = tid; c < nC; c += blockDim.x) {
+      const int sz = off[c + 1] - off[c];
+      if (sz > 0) atomicAdd(&ps.hist[binof(rs[c])], static_cast<uint32_t>(sz));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns bins [64 l, 64 l + 64), scanned from the top
+      uint32_t lsum = 0;
+      for (int b = 0; b < 64; ++b) lsum += ps.hist[lane * 64 + b];
+      uint32_t incl = lsum;  // suffix sum over lanes >= l
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+      }
+      uint32_t cum = incl - lsum;  // weight in bins above this lane's range
+      int found = -1;
+      for (int b = lane * 64 + 63; b >= lane * 64; --b) {
+        const uint32_t h = ps.hist[b];
+        if (found < 0 && cum < static_cast<uint32_t>(rem) && static_cast<uint32_t>(rem) <= cum + h) found = b;
+        cum += h;
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+      const int fb = __shfl_sync(0xffffffffu, found, who ? __ffs(who) - 1 : 0);
+      if (lane == 0) ps.scal[0] = who ? fb : 0;
+    }
+    __syncthreads();
+    bstar = ps.scal[0];
+  }
+  // pass C: clusters at or above the boundary bin, in id order
   int nsel = 0;
   for (int base = 0; base < nC; base += blockDim.x) {
-    const int c = base + threadIdx.x;
-    const bool p = c < nC && pred(c) && (take_all || key(c) >= theta);
+    const int c = base + tid;
+    bool p = false;
+    float v = 0.f;
+    if (c < nC && off[c + 1] > off[c]) {
+      v = rs[c];
+      p = take_all || binof(v) >= bstar;
+    }
     int total;
     const int r = block_rank(p, &total, bs);
     if (p && nsel + r < kSortCap)
-      sortbuf[nsel + r] = (static_cast<uint64_t>(~key(c)) << 32) | static_cast<uint32_t>(c);
+      sortbuf[nsel + r] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(c);
     nsel += total;
   }
   if (nsel > kSortCap) {
-    if (threadIdx.x == 0) atomicOr(a.err, DEV_ERR_CAPACITY);
+    if (tid == 0) atomicOr(a.err, DEV_ERR_CAPACITY);
     nsel = kSortCap;
   }
   int np = 1;
   while (np < nsel) np <<= 1;
-  for (int i = nsel + threadIdx.x; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
+  for (int i = nsel + tid; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
   __syncthreads();
   bitonic_sort_u64(sortbuf, np);
   // exclusive prefix of member counts in rank order
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < nsel; base += 32) {
       const int r = base + lane;
-      const int v = r < nsel ? static_cast<int>(size(static_cast<int>(sortbuf[r] & 0xffffffffu))) : 0;
+      const int v = r < nsel ? off[(sortbuf[r] & 0xffffffffu) + 1] - off[sortbuf[r] & 0xffffffffu] : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -128,17 +218,19 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     if (lane == 0) pref[nsel] = carry;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  for (int r = warp; r < nsel; r += nwarps) {
-    const int slot0 = fixed + pref[r];
-    if (slot0 >= C) continue;
-    const int c = static_cast<int>(sortbuf[r] & 0xffffffffu);
-    const int o = off[c];
-    const int n = min(static_cast<int>(size(c)), C - slot0);
-    for (int j = lane; j < n; j += 32) cand[slot0 + j] = a.members[o + j];
-  }
   const int len = static_cast<int>(min64(C, static_cast<int64_t>(fixed) + pref[nsel]));
+  // flat fill: slot -> rank r (binary search over pref) -> member
+  for (int slot = fixed + tid; slot < len; slot += blockDim.x) {
+    const int x = slot - fixed;
+    int lo = 0, hi = nsel - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pref[mid] <= x) lo = mid;
+      else hi = mid - 1;
+    }
+    const int c = static_cast<int>(sortbuf[lo] & 0xffffffffu);
+    cand[slot] = a.members[off[c] + (x - pref[lo])];
+  }
   __syncthreads();
   return len;
 }
@@ -169,7 +261,7 @@ struct Layout {
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ inline size_t region_bytes(int H, int d, bool tc) {
-  size_t p1 = static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4;
+  size_t p1 = static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4 + sizeof(P1Smem) + 16;
   size_t p2 = tc ? static_cast<size_t>(kStages) * kTile * 256 + static_cast<size_t>(H) * 256
                  : static_cast<size_t>(H) * d * 4;
   return align_up(p1 > p2 ? p1 : p2, 1024);
@@ -242,32 +334,6 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
 }
 
 // ---------------------------------------------------------- tcgen05 kernel
-// Gather one 128-row tile of candidate keys into the swizzled bf16 layout.
-// Thread r (0..127) of the gather warps; rows handled per warp: 32.
-__device__ __forceinline__ void gather_tile_bf16(const RefineArgs& a, const int32_t* cand, int n,
-                                                 int slot0, int64_t t, uint8_t* stage) {
-  const int gt = threadIdx.x;  // 0..127
-  const int gw = gt >> 5, lane = gt & 31;
-  const int chunk = lane & 15;
-  const uint16_t* keys = reinterpret_cast<const uint16_t*>(a.keys);
-#pragma unroll 4
-  for (int p = 0; p < 16; ++p) {
-    const int row = gw * 32 + 2 * p + (lane >> 4);
-    const int slot = slot0 + row;
-    int32_t id = slot < n ? cand[slot] : -1;
-    if (id > t) {
-      atomicOr(a.err, DEV_ERR_RANGE);
-      id = -1;
-    }
-    uint8_t* dst = stage + (chunk >> 3) * (kTile * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
-    const void* src = id >= 0 ? static_cast<const void*>(keys + static_cast<int64_t>(id) * 128 + chunk * 8)
-                              : static_cast<const void*>(keys);
-    const uint32_t sz = id >= 0 ? 16u : 0u;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(sz)
-                 : "memory");
-  }
-}
-
 __device__ __forceinline__ void gather_tile_fp8(const RefineArgs& a, const int32_t* cand, int n,
                                                 int slot0, int64_t t, uint8_t* stage) {
   const int gt = threadIdx.x;
@@ -309,106 +375,392 @@ __device__ __forceinline__ void gather_tile_fp8(const RefineArgs& a, const int32
   }
 }
 
+// ------------------------------------------------- top-k by the epilogue warps
+// The 128 epilogue threads hold the candidate scores in TMEM: thread
+// (quarter q, lane l) owns row r = 32 q + l, i.e. slots j * 128 + r, in
+// columns scol + j.  Selection: a 2048-bin linear histogram over
+// [min, max] locates the bin of the k-th score; the bin's items are sorted
+// to get the exact threshold; rare overflow and tie cases use a radix
+// select over the same items.  Ties at the threshold go to the lower key id.
+constexpr int kNB = 2048;     // histogram bins
+constexpr int kCapB = 2048;   // items of the threshold bin sorted in smem
+
+struct P3Smem {
+  uint32_t hist[kNB];
+  uint64_t buf[kCapB];
+  float fred[8];
+  int ired[8];
+  int scal[8];
+  unsigned long long cnt;
+};
+
+struct P3Ctx {
+  uint32_t tcol;   // TMEM address of this thread's first score column
+  int row, ntiles, n;
+  const int32_t* cand;
+};
+
+template <class F>
+__device__ __forceinline__ void p3_for_each(const P3Ctx& c, F f) {
+  for (int c0 = 0; c0 < c.ntiles; c0 += 16) {
+    float v[16];
+    tmem_ld16(c.tcol + c0, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int j = c0 + u;
+      const int slot = j * 128 + c.row;
+      if (j < c.ntiles && slot < c.n) f(v[u], slot);
+    }
+  }
+}
+
+// Exclusive prefix over the 128 epilogue threads (et = 0..127).
+__device__ __forceinline__ int p3_scan(int v, int et, int* total, P3Smem& ps) {
+  const int lane = et & 31, w = et >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ps.ired[w] = incl;
+  named_bar(1, 128);
+  int before = 0, tot = 0;
+  for (int i = 0; i < 4; ++i) {
+    if (i < w) before += ps.ired[i];
+    tot += ps.ired[i];
+  }
+  named_bar(1, 128);
+  *total = tot;
+  return before + incl - v;
+}
+
+// Radix select over the items passing pred: the value of key(v, slot) of
+// the need-th largest item, and how many items lie strictly above it.
+template <class Pred, class Key>
+__device__ uint32_t p3_radix(const P3Ctx& c, int et, Pred pred, Key key, int need, int* above,
+                             int* eq, P3Smem& ps) {
+  uint32_t prefix = 0, mask = 0;
+  int needr = need, ab = 0, last = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = et; i < 256; i += 128) ps.hist[i] = 0;
+    named_bar(1, 128);
+    p3_for_each(c, [&](float v, int slot) {
+      if (!pred(v, slot)) return;
+      const uint32_t kk = key(v, slot);
+      if ((kk & mask) == prefix) atomicAdd(&ps.hist[(kk >> shift) & 255u], 1u);
+    });
+    named_bar(1, 128);
+    if (et == 0) {
+      int cum = 0, dg = 0;
+      for (int d = 255; d >= 0; --d) {
+        const int h = static_cast<int>(ps.hist[d]);
+        if (cum < needr && needr <= cum + h) {
+          dg = d;
+          ps.scal[5] = h;
+          break;
+        }
+        cum += h;
+      }
+      ps.scal[3] = dg;
+      ps.scal[4] = cum;
+    }
+    named_bar(1, 128);
+    const uint32_t dg = static_cast<uint32_t>(ps.scal[3]);
+    needr -= ps.scal[4];
+    ab += ps.scal[4];
+    last = ps.scal[5];
+    prefix |= dg << shift;
+    mask |= 255u << shift;
+    named_bar(1, 128);
+  }
+  *above = ab;
+  *eq = last;
+  return prefix;
+}
+
+__device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3Smem& ps) {
+  const int k = a.k;
+  int32_t* out = a.out + static_cast<int64_t>(qi) * k;
+  float* outs = a.out_scores ? a.out_scores + static_cast<int64_t>(qi) * k : nullptr;
+  // range of the valid scores
+  float vmin = INFINITY, vmax = -INFINITY;
+  p3_for_each(c, [&](float v, int) {
+    vmin = fminf(vmin, v);
+    vmax = fmaxf(vmax, v);
+  });
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  }
+  if ((et & 31) == 0) {
+    ps.fred[et >> 5] = vmin;
+    ps.fred[4 + (et >> 5)] = vmax;
+  }
+  named_bar(1, 128);
+  vmin = fminf(fminf(ps.fred[0], ps.fred[1]), fminf(ps.fred[2], ps.fred[3]));
+  vmax = fmaxf(fmaxf(ps.fred[4], ps.fred[5]), fmaxf(ps.fred[6], ps.fred[7]));
+  named_bar(1, 128);
+  const bool take_all = c.n <= k;
+  float theta = -INFINITY;
+  int theta_id = 0x7fffffff;
+  bool ties_all = true;
+  if (!take_all) {
+    const float scale = vmax > vmin ? static_cast<float>(kNB) / (vmax - vmin) : 0.f;
+    auto binof = [&](float v) -> int {
+      const int b = static_cast<int>((v - vmin) * scale);
+      return b < kNB - 1 ? b : kNB - 1;
+    };
+    for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
+    if (et == 0) ps.cnt = 0;
+    named_bar(1, 128);
+    p3_for_each(c, [&](float v, int) { atomicAdd(&ps.hist[binof(v)], 1u); });
+    named_bar(1, 128);
+    // bin holding the k-th largest: thread et owns bins [16 et, 16 et + 16)
+    int tsum = 0;
+    for (int b = 0; b < 16; ++b) tsum += static_cast<int>(ps.hist[16 * et + b]);
+    int tot;
+    const int before = p3_scan(tsum, et, &tot, ps);
+    int cum = tot - before - tsum;  // items in bins above this thread's range
+    for (int b = 16 * et + 15; b >= 16 * et; --b) {
+      const int h = static_cast<int>(ps.hist[b]);
+      if (cum < k && k <= cum + h) {
+        ps.scal[0] = b;
+        ps.scal[1] = cum;
+        ps.scal[2] = h;
+      }
+      cum += h;
+    }
+    named_bar(1, 128);
+    const int bstar = ps.scal[0], above_b = ps.scal[1], nb = ps.scal[2];
+    const int need = k - above_b;
+    int above_in = 0, eq = 0;
+    uint32_t tkey;
+    if (nb <= kCapB) {
+      p3_for_each(c, [&](float v, int slot) {
+        if (binof(v) == bstar) {
+          const unsigned long long pos = atomicAdd(&ps.cnt, 1ull);
+          ps.buf[pos] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(slot);
+        }
+      });
+      named_bar(1, 128);
+      int np = 1;
+      while (np < nb) np <<= 1;
+      for (int i = nb + et; i < np; i += 128) ps.buf[i] = ~0ull;
+      named_bar(1, 128);
+      for (int kk = 2; kk <= np; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+          for (int i = et; i < np; i += 128) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const uint64_t x = ps.buf[i], y = ps.buf[ixj];
+              if ((x > y) == ((i & kk) == 0)) {
+                ps.buf[i] = y;
+                ps.buf[ixj] = x;
+              }
+            }
+          }
+          named_bar(1, 128);
+        }
+      }
+      tkey = ~static_cast<uint32_t>(ps.buf[need - 1] >> 32);
+      if (et == 0) {
+        int i0 = need - 1;
+        while (i0 > 0 && ~static_cast<uint32_t>(ps.buf[i0 - 1] >> 32) == tkey) --i0;
+        int i1 = need - 1;
+        while (i1 + 1 < nb && ~static_cast<uint32_t>(ps.buf[i1 + 1] >> 32) == tkey) ++i1;
+        ps.scal[6] = i0;
+        ps.scal[7] = i1 - i0 + 1;
+      }
+      named_bar(1, 128);
+      above_in = ps.scal[6];
+      eq = ps.scal[7];
+    } else {
+      tkey = p3_radix(
+          c, et, [&](float v, int) { return binof(v) == bstar; },
+          [&](float v, int) { return f2key(v); }, need, &above_in, &eq, ps);
+    }
+    theta = key2f(tkey);
+    const int need_eq = k - above_b - above_in;
+    if (eq > need_eq) {
+      ties_all = false;
+      int ab2 = 0, eq2 = 0;
+      const uint32_t idk = p3_radix(
+          c, et, [&](float v, int) { return v == theta; },
+          [&](float, int slot) { return ~static_cast<uint32_t>(c.cand[slot]); }, need_eq, &ab2, &eq2,
+          ps);
+      theta_id = static_cast<int>(~idk);
+    }
+  }
+  // emission: thread-major order, deterministic
+  auto sel = [&](float v, int slot) {
+    return take_all || v > theta || (v == theta && (ties_all || c.cand[slot] <= theta_id));
+  };
+  int mine = 0;
+  p3_for_each(c, [&](float v, int slot) { mine += sel(v, slot) ? 1 : 0; });
+  int total;
+  int pos = p3_scan(mine, et, &total, ps);
+  p3_for_each(c, [&](float v, int slot) {
+    if (sel(v, slot)) {
+      if (pos < k) {
+        out[pos] = c.cand[slot];
+        if (outs) outs[pos] = v;
+      }
+      ++pos;
+    }
+  });
+  for (int j = min(total, k) + et; j < k; j += 128) {
+    out[j] = -1;
+    if (outs) outs[j] = -INFINITY;
+  }
+}
+
+// Layout of the tensor-core kernel (one region reused by the three phases).
+constexpr int kStages2 = 2;
+__host__ __device__ inline size_t tc_region_bytes() {
+  size_t p1 = static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4 + sizeof(P1Smem) + 16;
+  size_t p2 = static_cast<size_t>(kStages2) * kTile * 256;
+  size_t p3 = sizeof(P3Smem);
+  size_t m = p1 > p2 ? p1 : p2;
+  return align_up(m > p3 ? m : p3, 1024);
+}
+__host__ __device__ inline size_t tc_smem_bytes(int C, int H) {
+  return 1024 + tc_region_bytes() + static_cast<size_t>(H) * 256 + align_up(static_cast<size_t>(C) * 4, 16) +
+         align_up(static_cast<size_t>(H) * 4, 16) + (2 * kStages2 + 5) * 8 + 16;
+}
+__host__ __device__ inline int tc_tmem_cols(int C, int H) {
+  const int sc = ((C + 127) / 128 + 15) / 16 * 16;
+  int need = 2 * H + sc, cols = 32;
+  while (cols < need) cols <<= 1;
+  return cols;
+}
+
 template <int H>
-__global__ void __launch_bounds__(kTcThreads, 1) k_refine_tc(RefineArgs a, VersionTable vt) {
+__global__ void __launch_bounds__(kTcThreads, 2)
+    k_refine_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                RefineArgs a, VersionTable vt) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ BlockScratch bs;
-  Layout L = carve(smem_raw, a.C, H, 128, true);
-  uint64_t* full = L.bars;
-  uint64_t* empty = L.bars + kStages;
-  uint64_t* tfull = L.bars + 2 * kStages;
-  uint64_t* tempty = L.bars + 2 * kStages + 2;
-  uint8_t* stages = L.region;
-  uint8_t* qtile = L.region + kStages * kTile * 256;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* region = base;
+  uint8_t* qtile = region + tc_region_bytes();
+  int32_t* cand = reinterpret_cast<int32_t*>(qtile + H * 256);
+  float* wsh = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(cand) + align_up(static_cast<size_t>(a.C) * 4, 16));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(wsh) + align_up(H * 4, 16));
+  uint64_t* qfull = bars + 2 * kStages2 + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages2 + 5);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages2;
+  uint64_t* tfull = bars + 2 * kStages2;
+  uint64_t* tempty = bars + 2 * kStages2 + 2;
+  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(region);
+  int32_t* pref = reinterpret_cast<int32_t*>(region + static_cast<size_t>(kSortCap) * 8);
+  P3Smem& ps = *reinterpret_cast<P3Smem*>(region);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kTmemCols = 2 * H;
+  const int tcols = tc_tmem_cols(a.C, H);
+  const bool fp8 = a.key_dtype == KD_FP8;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 128);
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], fp8 ? 128 : 4);
       mbar_init(&empty[s], 1);
     }
     for (int c = 0; c < 2; ++c) {
       mbar_init(&tfull[c], 1);
       mbar_init(&tempty[c], 128);
     }
-    *L.abort = 0;
+    mbar_init(qfull, 1);
+    *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 4) {
-    tmem_alloc(L.tmem, kTmemCols);
+    tmem_alloc(tmem_holder, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *L.tmem;
-  uint32_t g = 0;  // tiles processed by this CTA so far (for barrier parity)
+  const uint32_t tmem_base = *tmem_holder;
+  uint32_t g = 0;      // tiles processed so far by this CTA (barrier parity)
+  uint32_t qiter = 0;  // queries processed so far by this CTA
 
-  for (int qi = blockIdx.x; qi < a.T; qi += gridDim.x) {
+  for (int qi = blockIdx.x; qi < a.T; qi += gridDim.x, ++qiter) {
     const int64_t t = a.pos0 + qi;
+    // the query's heads (UMMA B operand) arrive by TMA while the
+    // candidate list is built
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(qfull, H * 256);
+      tma_load_2d(qtile, &qmap, 0, qi * H, qfull);
+      tma_load_2d(qtile + H * 128, &qmap, 64, qi * H, qfull);
+    }
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref, bs);
+    const int n = build_candidates(a, qi, t, nC, n_v, cand, sortbuf, pref, bs);
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
-        a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? L.cand[i] : -1;
+        a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cand[i] : -1;
     }
-    // query heads -> swizzled UMMA B tile (H rows x 128 bf16), weights -> smem
-    const uint16_t* qg = reinterpret_cast<const uint16_t*>(a.q) + static_cast<int64_t>(qi) * H * 128;
-    for (int i = threadIdx.x; i < H * 16; i += blockDim.x) {
-      const int h = i >> 4, chunk = i & 15;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + h * 128) + chunk);
-      uint8_t* dst = qtile + (chunk >> 3) * (H * 128) + h * 128 + (((chunk & 7) ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = v;
-    }
-    for (int h = threadIdx.x; h < H; h += blockDim.x) L.wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
+    for (int h = threadIdx.x; h < H; h += blockDim.x) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
     fence_proxy_async_smem();
     __syncthreads();
 
     const int ntiles = (n + kTile - 1) / kTile;
-    if (warp < 4) {
-      // ------------------------------------------------------------ gather
-      if (a.key_dtype == KD_BF16) {
-        for (int j = 0; j < ntiles; ++j) {
-          const uint32_t gj = g + j;
-          const int s = gj % kStages;
-          if (gj >= kStages && !mbar_wait(&empty[s], ((gj / kStages) & 1) ^ 1, a.err, L.abort)) break;
-          gather_tile_bf16(a, L.cand, n, j * kTile, t, stages + s * (kTile * 256));
-          cp_async_commit();
-          if (j >= kStages - 1) {
-            cp_async_wait<kStages - 1>();
-            fence_proxy_async_smem();
-            mbar_arrive(&full[(g + j - (kStages - 1)) % kStages]);
+    if (!fp8 && warp < 4) {
+      // ------------------------------------------- TMA gather4 producers
+      // Four warps share a tile (32 rows each): a single issuing warp
+      // limits gather4 throughput, so the issue is spread out.
+      for (int j = 0; j < ntiles; ++j) {
+        const uint32_t gj = g + j;
+        const int s = gj % kStages2;
+        if (gj >= kStages2 && !mbar_wait(&empty[s], ((gj / kStages2) & 1) ^ 1, a.err, abort_flag)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], kTile * 256 / 4);
+        __syncwarp();
+        if (lane < 16) {
+          const int rl = warp * 32 + (lane & 7) * 4;  // first of this lane's 4 rows
+          int r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int slot = j * kTile + rl + i;
+            int id = slot < n ? cand[slot] : 0;
+            if (id < 0 || id > t) {
+              atomicOr(a.err, DEV_ERR_RANGE);
+              id = 0;
+            }
+            r[i] = id;
           }
-        }
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        for (int j = max(0, ntiles - (kStages - 1)); j < ntiles; ++j) mbar_arrive(&full[(g + j) % kStages]);
-      } else {
-        for (int j = 0; j < ntiles; ++j) {
-          const uint32_t gj = g + j;
-          const int s = gj % kStages;
-          if (gj >= kStages && !mbar_wait(&empty[s], ((gj / kStages) & 1) ^ 1, a.err, L.abort)) break;
-          gather_tile_fp8(a, L.cand, n, j * kTile, t, stages + s * (kTile * 256));
-          fence_proxy_async_smem();
-          mbar_arrive(&full[s]);
+          const int half = lane >> 3;
+          uint8_t* dst = region + s * (kTile * 256) + half * (kTile * 128) + rl * 128;
+          tma_gather4(dst, &kmap, half * 64, r[0], r[1], r[2], r[3], &full[s]);
         }
       }
+    } else if (fp8 && warp < 4) {
+      // --------------------------------------- fp8 rows widened to bf16
+      for (int j = 0; j < ntiles; ++j) {
+        const uint32_t gj = g + j;
+        const int s = gj % kStages2;
+        if (gj >= kStages2 && !mbar_wait(&empty[s], ((gj / kStages2) & 1) ^ 1, a.err, abort_flag)) break;
+        gather_tile_fp8(a, cand, n, j * kTile, t, region + s * (kTile * 256));
+        fence_proxy_async_smem();
+        mbar_arrive(&full[s]);
+      }
     } else if (warp == 4) {
-      // -------------------------------------------------------- UMMA issue
+      // ------------------------------------------------------ UMMA issue
       if (lane == 0) {
         constexpr uint32_t idesc = idesc_bf16_f32(kTile, H);
         const uint32_t sb = smem_u32(qtile);
-        for (int j = 0; j < ntiles; ++j) {
+        // wait for this query's head tile (every query, so phases stay paired)
+        const bool qok = mbar_wait(qfull, qiter & 1, a.err, abort_flag);
+        for (int j = 0; qok && j < ntiles; ++j) {
           const uint32_t gj = g + j;
-          const int s = gj % kStages;
+          const int s = gj % kStages2;
           const int acc = gj & 1;
-          if (!mbar_wait(&full[s], (gj / kStages) & 1, a.err, L.abort)) break;
-          if (gj >= 2 && !mbar_wait(&tempty[acc], ((gj >> 1) & 1) ^ 1, a.err, L.abort)) break;
+          if (!mbar_wait(&full[s], (gj / kStages2) & 1, a.err, abort_flag)) break;
+          if (gj >= 2 && !mbar_wait(&tempty[acc], ((gj >> 1) & 1) ^ 1, a.err, abort_flag)) break;
           tc_fence_after();
-          const uint32_t sa = smem_u32(stages + s * (kTile * 256));
+          const uint32_t sa = smem_u32(region + s * (kTile * 256));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
@@ -419,15 +771,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_refine_tc(RefineArgs a, Versi
           umma_commit(&tfull[acc]);
         }
       }
-    } else {
-      // ---------------------------------------------------------- epilogue
+    } else if (warp >= 5) {
+      // ------------------------------------------ epilogue -> TMEM scores
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
       for (int j = 0; j < ntiles; ++j) {
         const uint32_t gj = g + j;
         const int acc = gj & 1;
-        if (!mbar_wait(&tfull[acc], (gj >> 1) & 1, a.err, L.abort)) break;
+        if (!mbar_wait(&tfull[acc], (gj >> 1) & 1, a.err, abort_flag)) break;
         tc_fence_after();
         float sc = 0.f;
 #pragma unroll
@@ -436,55 +788,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_refine_tc(RefineArgs a, Versi
           tmem_ld32(tmem_base + acc * H + c * 32 + lane_off, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < 32; ++h) sc = fmaf(L.wsh[c * 32 + h], fmaxf(v[h], 0.f), sc);
+          for (int h = 0; h < 32; ++h) sc = fmaf(wsh[c * 32 + h], fmaxf(v[h], 0.f), sc);
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
         const int slot = j * kTile + row;
-        if (slot < n) {
-          if (a.key_scale) sc *= a.key_scale[L.cand[slot]];
-          L.score[slot] = sc;
-        }
+        if (fp8 && slot < n) sc *= a.key_scale[cand[slot]];
+        tmem_st1(tmem_base + 2 * H + j + lane_off, sc);
       }
+      tmem_st_wait();
     }
     g += ntiles;
     __syncthreads();
+    if (*abort_flag) break;
     fence_proxy_async_smem();  // the region is rewritten by generic stores next
-    if (*L.abort) break;
-    topk_emit(a, qi, L.score, L.cand, n, bs);
+    // ----------------------------------------------------------- top-k
+    if (warp >= 5) {
+      const int quarter = warp & 3;
+      P3Ctx c;
+      c.row = quarter * 32 + lane;
+      c.tcol = tmem_base + 2 * H + (static_cast<uint32_t>(quarter * 32) << 16);
+      c.ntiles = ntiles;
+      c.n = n;
+      c.cand = cand;
+      p3_topk(a, qi, c, threadIdx.x - 160, ps);
+    }
+    __syncthreads();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 4) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, tcols);
   }
 }
 
 }  // namespace
 
 size_t refine_smem_bytes(int C, int H, int d, bool tc) {
-  return 1024 + region_bytes(H, d, tc) + 2 * align_up(static_cast<size_t>(C) * 4, 16) +
+  if (tc) return tc_smem_bytes(C, H);
+  return 1024 + region_bytes(H, d, false) + 2 * align_up(static_cast<size_t>(C) * 4, 16) +
          align_up(static_cast<size_t>(H) * 4, 16) + (2 * kStages + 4) * 8 + 16;
 }
 
-cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, bool tc, int num_sms,
-                          cudaStream_t st) {
+cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUtensorMap* kmap,
+                          const CUtensorMap* qmap, int num_sms, cudaStream_t st) {
   if (a.T <= 0) return cudaSuccess;
+  const bool tc = kmap != nullptr && qmap != nullptr;
   const size_t smem = refine_smem_bytes(a.C, a.H, a.d, tc);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (tc) {
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
-    const int grid = a.T < num_sms ? a.T : num_sms;
+    // CTAs per SM bounded by shared memory and by TMEM (512 columns)
+    int per_sm = static_cast<int>((228 * 1024) / (smem + 2048));
+    const int tm = 512 / tc_tmem_cols(a.C, a.H);
+    per_sm = per_sm < tm ? per_sm : tm;
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
     if (a.H == 32) {
       cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       count_launch();
-      k_refine_tc<32><<<grid, kTcThreads, smem, st>>>(a, vt);
+      k_refine_tc<32><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);
     } else if (a.H == 64) {
       cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       count_launch();
-      k_refine_tc<64><<<grid, kTcThreads, smem, st>>>(a, vt);
+      k_refine_tc<64><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);
     } else {
       return cudaErrorInvalidValue;
     }

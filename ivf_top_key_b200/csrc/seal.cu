@@ -14,13 +14,14 @@
 // Members are stored per cluster in ascending key id; the representative is
 // the mean rounded once to bf16 (round to nearest even).
 //
-// One CTA (1024 threads) per window.  The W*m distances are sorted with a
-// shared-memory bitonic sort of (distance bits, pair index); the greedy walk
-// is done by one warp, 32 sorted pairs at a time: within a batch the first
-// live pair of each key is the only one that can win, pairs of one cluster
-// are ranked in order, and the batch is committed up to the first pair
-// refused for lack of room (which happens at most m times per pass), so the
-// result equals the sequential walk.
+// One CTA (1024 threads) per window.  The sequential greedy walk over the
+// W*m sorted pairs is reproduced exactly in at most m + 1 data-parallel
+// rounds: in a round every free key proposes its best pair among the
+// clusters that are not full; the proposals are sorted by (cluster, pair
+// order); the first cluster to fill is the one whose (cap - count)-th
+// proposal comes first in pair order; every proposal up to that pair is
+// final (nothing before it can be refused), that cluster is closed, and the
+// remaining keys propose again.  Pair order is (distance, key, cluster).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,16 +31,25 @@ namespace {
 constexpr int kThreads = 1024;
 
 struct SealSmem {
-  uint64_t* dkey;    // [NP] distance bits
-  uint16_t* pidx;    // [NP] pair index i*m + j
+  double* D;         // [W, m] squared distances
   double* cent;      // [m, d]
+  uint64_t* bk1;     // [m, NPW] proposal buckets: distance bits
+  uint16_t* bk2;     // [m, NPW] proposal buckets: key
+  int* wcnt;         // [m, 32] per-(cluster, warp) counts / offsets
+  int* bfill;        // [m] bucket sizes
+  int* bpass;        // [m]
   int16_t* assign;   // [W]
   int16_t* prev;     // [W]
-  uint8_t* taken;    // [W]
-  int* cnt;          // [m]
+  int* cnt;          // [m] members so far
+  int* tcnt;         // [m] (spare)
+  int* tstart;       // [m + 1] (spare)
   int* cstart;       // [m + 1] member list starts
   int16_t* mlist;    // [W] members, grouped by cluster, ascending
-  int* flag;         // [2]
+  uint64_t* fk1;     // [m] fill pair of each cluster: distance bits
+  uint32_t* fk2;     // [m] fill pair: (key << 16) | cluster
+  int* flag;         // [4]
+  int* red;          // [32] per-warp partial sums
+  unsigned long long* fullmask;
 };
 
 __device__ __forceinline__ double key_f64(const SealArgs& a, int64_t s, int i) {
@@ -74,37 +84,58 @@ __device__ __forceinline__ void load8(const SealArgs& a, int64_t row, int e0, do
   }
 }
 
-__device__ __forceinline__ bool pair_less(uint64_t d1, uint16_t p1, uint64_t d2, uint16_t p2) {
-  return d1 < d2 || (d1 == d2 && p1 < p2);
+// Pair order (distance, key, cluster): is (d1, i1, j1) <= (d2, i2, j2)?
+__device__ __forceinline__ bool pair_le(uint64_t d1, uint32_t i1, uint32_t j1, uint64_t d2,
+                                        uint32_t i2, uint32_t j2) {
+  if (d1 != d2) return d1 < d2;
+  if (i1 != i2) return i1 < i2;
+  return j1 <= j2;
 }
 
 __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
   extern __shared__ uint8_t raw[];
   const int W = a.W, m = a.m, d = a.d;
-  const int np_pairs = W * m;
-  int NP = 1;
-  while (NP < np_pairs) NP <<= 1;
+  int NPW = 1;
+  while (NPW < W) NPW <<= 1;
   SealSmem s;
   uint8_t* p = raw;
-  s.dkey = reinterpret_cast<uint64_t*>(p);
-  p += static_cast<size_t>(NP) * 8;
+  s.D = reinterpret_cast<double*>(p);
+  p += static_cast<size_t>(W) * m * 8;
   s.cent = reinterpret_cast<double*>(p);
   p += static_cast<size_t>(m) * d * 8;
-  s.pidx = reinterpret_cast<uint16_t*>(p);
-  p += static_cast<size_t>(NP) * 2;
+  s.bk1 = reinterpret_cast<uint64_t*>(p);
+  p += static_cast<size_t>(m) * NPW * 8;
+  s.fk1 = reinterpret_cast<uint64_t*>(p);
+  p += static_cast<size_t>(m) * 8;
+  s.fullmask = reinterpret_cast<unsigned long long*>(p);
+  p += 8;
+  s.wcnt = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m) * 32 * 4;
+  s.bfill = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m) * 4;
+  s.bpass = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m) * 4;
+  s.fk2 = reinterpret_cast<uint32_t*>(p);
+  p += static_cast<size_t>(m) * 4;
+  s.cnt = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m) * 4;
+  s.tcnt = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m) * 4;
+  s.tstart = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m + 1) * 4;
+  s.cstart = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(m + 1) * 4;
+  s.flag = reinterpret_cast<int*>(p);
+  p += 16;
+  s.red = reinterpret_cast<int*>(p);
+  p += 128;
   s.assign = reinterpret_cast<int16_t*>(p);
   p += static_cast<size_t>(W) * 2;
   s.prev = reinterpret_cast<int16_t*>(p);
   p += static_cast<size_t>(W) * 2;
-  s.taken = p;
-  p += (W + 15) / 16 * 16;
-  s.cnt = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.cstart = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m + 1) * 4;
   s.mlist = reinterpret_cast<int16_t*>(p);
-  p += static_cast<size_t>(W + 8) / 8 * 16;
-  s.flag = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(W) * 2;
+  s.bk2 = reinterpret_cast<uint16_t*>(p);
 
   const int win = blockIdx.x;
   const int64_t lo = a.first_key + static_cast<int64_t>(win) * W;
@@ -142,10 +173,7 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
             }
           }
         }
-        for (int j = 0; j < m; ++j) {
-          s.dkey[i * m + j] = static_cast<uint64_t>(__double_as_longlong(acc[j]));
-          s.pidx[i * m + j] = static_cast<uint16_t>(i * m + j);
-        }
+        for (int j = 0; j < m; ++j) s.D[i * m + j] = acc[j];
       } else {
         for (int j = 0; j < m; ++j) {
           double acc = 0.0;
@@ -158,72 +186,171 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
               acc = fma(df, df, acc);
             }
           }
-          s.dkey[i * m + j] = static_cast<uint64_t>(__double_as_longlong(acc));
-          s.pidx[i * m + j] = static_cast<uint16_t>(i * m + j);
+          s.D[i * m + j] = acc;
         }
       }
+      s.assign[i] = -1;
     }
-    for (int q = np_pairs + tid; q < NP; q += blockDim.x) {
-      s.dkey[q] = ~0ull;
-      s.pidx[q] = 0xFFFFu;
-    }
-    for (int i = tid; i < W; i += blockDim.x) s.taken[i] = 0;
     for (int j = tid; j < m; j += blockDim.x) s.cnt[j] = 0;
+    if (tid == 0) *s.fullmask = 0ull;
     __syncthreads();
-    // bitonic sort by (distance, pair index)
-    for (int k = 2; k <= NP; k <<= 1) {
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int q = tid; q < NP; q += blockDim.x) {
-          const int r = q ^ j;
-          if (r > q) {
-            const uint64_t d1 = s.dkey[q], d2 = s.dkey[r];
-            const uint16_t p1 = s.pidx[q], p2 = s.pidx[r];
-            const bool up = (q & k) == 0;
-            if (pair_less(d2, p2, d1, p1) == up) {
-              s.dkey[q] = d2;
-              s.dkey[r] = d1;
-              s.pidx[q] = p2;
-              s.pidx[r] = p1;
+
+    // greedy capacity assignment in rounds (see the file comment)
+    int n_free = W;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nwarps = blockDim.x >> 5;
+    for (int round = 0; round <= m && n_free > 0; ++round) {
+      const unsigned long long fullm = *s.fullmask;
+      // 1. proposals, bucketed by cluster without atomics: per-warp ballot
+      //    counts -> (cluster, warp) offsets -> scatter
+      for (int j = tid; j < m; j += blockDim.x) s.bfill[j] = 0;
+      __syncthreads();
+      for (int i0 = 0; i0 < W; i0 += blockDim.x) {
+        const int i = i0 + tid;
+        int bj = -1;
+        double bd = 0.0;
+        if (i < W && s.assign[i] < 0) {
+          for (int j = 0; j < m; ++j) {
+            if ((fullm >> j) & 1ull) continue;
+            const double v = s.D[i * m + j];
+            if (bj < 0 || v < bd) {
+              bj = j;
+              bd = v;
             }
           }
+        }
+        for (int j = 0; j < m; ++j) {
+          const unsigned bal = __ballot_sync(0xffffffffu, bj == j);
+          if (lane == 0) s.wcnt[j * nwarps + warp] = __popc(bal);
+        }
+        __syncthreads();
+        // exclusive offsets of (cluster j, warp w) within this pass
+        if (tid < m) {
+          int run = 0;
+          for (int w = 0; w < nwarps; ++w) {
+            const int c = s.wcnt[tid * nwarps + w];
+            s.wcnt[tid * nwarps + w] = run;
+            run += c;
+          }
+          s.bpass[tid] = run;
+        }
+        __syncthreads();
+        for (int j = 0; j < m; ++j) {
+          const unsigned bal = __ballot_sync(0xffffffffu, bj == j);
+          if (bj == j) {
+            const int slot = s.bfill[j] + s.wcnt[j * nwarps + warp] + __popc(bal & ((1u << lane) - 1u));
+            s.bk1[j * NPW + slot] = static_cast<uint64_t>(__double_as_longlong(bd));
+            s.bk2[j * NPW + slot] = static_cast<uint16_t>(i);
+          }
+        }
+        __syncthreads();
+        if (tid < m) s.bfill[tid] += s.bpass[tid];
+        __syncthreads();
+      }
+      // 2. one warp per open cluster: sort its bucket by (distance, key) and
+      //    take the proposal that would fill it
+      for (int j = warp; j < m; j += nwarps) {
+        const int nb = s.bfill[j];
+        const int need = a.cap - s.cnt[j];
+        uint64_t* k1 = s.bk1 + j * NPW;
+        uint16_t* k2 = s.bk2 + j * NPW;
+        if (lane == 0) {
+          s.fk1[j] = ~0ull;
+          s.fk2[j] = ~0u;
+        }
+        if (((fullm >> j) & 1ull) || nb < need || need <= 0) continue;
+        int np = 1;
+        while (np < nb) np <<= 1;
+        for (int q = nb + lane; q < np; q += 32) {
+          k1[q] = ~0ull;
+          k2[q] = 0xFFFFu;
+        }
+        __syncwarp();
+        for (int kk = 2; kk <= np; kk <<= 1) {
+          for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int q = lane; q < np; q += 32) {
+              const int r = q ^ jj;
+              if (r > q) {
+                const uint64_t a1 = k1[q], b1 = k1[r];
+                const uint16_t a2 = k2[q], b2 = k2[r];
+                const bool b_less = b1 < a1 || (b1 == a1 && b2 < a2);
+                if (b_less == ((q & kk) == 0)) {
+                  k1[q] = b1;
+                  k1[r] = a1;
+                  k2[q] = b2;
+                  k2[r] = a2;
+                }
+              }
+            }
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          s.fk1[j] = k1[need - 1];
+          s.fk2[j] = (static_cast<uint32_t>(k2[need - 1]) << 16) | static_cast<uint32_t>(j);
+        }
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int best = -1;
+        for (int j = 0; j < m; ++j) {
+          if (s.fk1[j] == ~0ull && s.fk2[j] == ~0u) continue;
+          if (best < 0 || pair_le(s.fk1[j], s.fk2[j] >> 16, s.fk2[j] & 0xFFFFu, s.fk1[best],
+                                  s.fk2[best] >> 16, s.fk2[best] & 0xFFFFu))
+            best = j;
+        }
+        s.flag[2] = best;
+      }
+      __syncthreads();
+      const int best = s.flag[2];
+      const uint64_t bk1 = best >= 0 ? s.fk1[best] : 0;
+      const uint32_t bi = best >= 0 ? (s.fk2[best] >> 16) : 0;
+      // 3. commit every proposal up to the filling pair (all if none)
+      for (int i = tid; i < W; i += blockDim.x) {
+        if (s.assign[i] >= 0) continue;
+        int bj = -1;
+        double bd = 0.0;
+        for (int j = 0; j < m; ++j) {
+          if ((fullm >> j) & 1ull) continue;
+          const double v = s.D[i * m + j];
+          if (bj < 0 || v < bd) {
+            bj = j;
+            bd = v;
+          }
+        }
+        if (bj >= 0 && (best < 0 || pair_le(static_cast<uint64_t>(__double_as_longlong(bd)), i, bj, bk1, bi,
+                                            static_cast<uint32_t>(best))))
+          s.assign[i] = static_cast<int16_t>(bj);
+      }
+      if (tid == 0 && best >= 0) *s.fullmask |= 1ull << best;
+      __syncthreads();
+      // member counts and keys still free (ballots, no shared atomics)
+      {
+        int mine = 0;
+        for (int i = tid; i < W; i += blockDim.x) mine += s.assign[i] < 0 ? 1 : 0;
+        for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+        if (lane == 0) s.red[warp] = mine;
+        for (int j = 0; j < m; ++j) {
+          int cj = 0;
+          for (int i0 = 0; i0 < W; i0 += blockDim.x) {
+            const int i = i0 + tid;
+            cj += __popc(__ballot_sync(0xffffffffu, i < W && s.assign[i] == j));
+          }
+          if (lane == 0) s.wcnt[j * nwarps + warp] = cj;
+        }
+        __syncthreads();
+        n_free = 0;
+        for (int w = 0; w < nwarps; ++w) n_free += s.red[w];
+        if (tid < m) {
+          int c = 0;
+          for (int w = 0; w < nwarps; ++w) c += s.wcnt[tid * nwarps + w];
+          s.cnt[tid] = c;
         }
         __syncthreads();
       }
     }
-    // greedy capacity assignment (warp 0)
-    if (tid < 32) {
-      const int lane = tid;
-      const unsigned lt = (1u << lane) - 1u;
-      int pos = 0, n_free = W;
-      while (pos < np_pairs && n_free > 0) {
-        const int q = pos + lane;
-        const bool valid = q < np_pairs;
-        const int pi = valid ? s.pidx[q] : 0;
-        const int i = pi / m, j = pi % m;
-        const bool live = valid && !s.taken[i] && s.cnt[j] < a.cap;
-        const unsigned mi = __match_any_sync(0xffffffffu, live ? i : -1 - lane);
-        const bool leader = live && (__ffs(mi) - 1 == lane);
-        const unsigned mj = __match_any_sync(0xffffffffu, leader ? j : -1 - lane);
-        const int rank = __popc(mj & lt);
-        const bool ok = leader && (s.cnt[j] + rank < a.cap);
-        const unsigned bad = __ballot_sync(0xffffffffu, leader && !ok);
-        const int limit = bad ? __ffs(bad) - 1 : 32;
-        const bool acc = ok && lane < limit;
-        const unsigned accj = __match_any_sync(0xffffffffu, acc ? j : -1 - lane);
-        __syncwarp();
-        if (acc) {
-          s.taken[i] = 1;
-          s.assign[i] = static_cast<int16_t>(j);
-          if (__ffs(accj) - 1 == lane) s.cnt[j] += __popc(accj);
-        }
-        n_free -= __popc(__ballot_sync(0xffffffffu, acc));
-        __syncwarp();
-        pos += bad ? limit + 1 : 32;
-      }
-      if (lane == 0) s.flag[1] = n_free;
-    }
-    __syncthreads();
-    if (tid == 0 && s.flag[1] != 0) atomicOr(a.err, DEV_ERR_CAPACITY);
+    if (tid == 0 && n_free != 0) atomicOr(a.err, DEV_ERR_CAPACITY);
+
     // member lists (ascending key order), one warp per cluster
     {
       const int warp = tid >> 5, lane = tid & 31;
@@ -247,24 +374,27 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         }
       }
       __syncthreads();
-      // update: float64 mean of the members in ascending key order
-      for (int j = warp; j < m; j += blockDim.x >> 5) {
+      // update: float64 mean of the members in ascending key order; the
+      // (cluster, 32-dim block) pairs are spread over all warps
+      const int nblk = (d + 31) / 32;
+      for (int wj = warp; wj < m * nblk; wj += blockDim.x >> 5) {
+        const int j = wj / nblk;
         const int b0 = s.cstart[j], b1 = s.cstart[j + 1];
         if (b1 == b0) continue;
-        for (int e = lane; e < d; e += 32) {
+        for (int e = (wj % nblk) * 32 + lane; e < d && e < (wj % nblk) * 32 + 32; e += 32) {
           double sum = 0.0;
-          int p = b0;
-          for (; p + 4 <= b1; p += 4) {
-            const double v0 = key_f64(a, lo + s.mlist[p], e);
-            const double v1 = key_f64(a, lo + s.mlist[p + 1], e);
-            const double v2 = key_f64(a, lo + s.mlist[p + 2], e);
-            const double v3 = key_f64(a, lo + s.mlist[p + 3], e);
+          int q = b0;
+          for (; q + 4 <= b1; q += 4) {
+            const double v0 = key_f64(a, lo + s.mlist[q], e);
+            const double v1 = key_f64(a, lo + s.mlist[q + 1], e);
+            const double v2 = key_f64(a, lo + s.mlist[q + 2], e);
+            const double v3 = key_f64(a, lo + s.mlist[q + 3], e);
             sum += v0;
             sum += v1;
             sum += v2;
             sum += v3;
           }
-          for (; p < b1; ++p) sum += key_f64(a, lo + s.mlist[p], e);
+          for (; q < b1; ++q) sum += key_f64(a, lo + s.mlist[q], e);
           s.cent[j * d + e] = sum / static_cast<double>(b1 - b0);
         }
       }
@@ -297,16 +427,19 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
 }  // namespace
 
 size_t seal_smem_bytes(int W, int m, int d) {
-  int NP = 1;
-  while (NP < W * m) NP <<= 1;
-  return static_cast<size_t>(NP) * 10 + static_cast<size_t>(m) * d * 8 + static_cast<size_t>(W) * 4 +
-         (W + 15) / 16 * 16 + static_cast<size_t>(m) * 4 + static_cast<size_t>(m + 1) * 4 +
-         static_cast<size_t>(W + 8) / 8 * 16 + 16;
+  int NPW = 1;
+  while (NPW < W) NPW <<= 1;
+  // D, centres, proposal buckets (m x NPW of u64 + u16), counters, key lists
+  return static_cast<size_t>(W) * m * 8 + static_cast<size_t>(m) * d * 8 +
+         static_cast<size_t>(m) * NPW * 10 + static_cast<size_t>(m) * 12 + 8 +
+         static_cast<size_t>(m) * 32 * 4 + static_cast<size_t>(m) * 8 +
+         static_cast<size_t>(m + 1) * 8 + 16 + 128 + static_cast<size_t>(W) * 6 +
+         static_cast<size_t>(m) * 32 + 256;
 }
 
 cudaError_t launch_seal(const SealArgs& a, cudaStream_t st) {
   if (a.n_windows <= 0) return cudaSuccess;
-  if (a.m > 64 || a.W * a.m > 65535 || a.W > 32767 || a.d % 8 != 0) return cudaErrorInvalidValue;
+  if (a.m > 64 || a.W > 65535 || a.d % 8 != 0) return cudaErrorInvalidValue;
   const size_t smem = seal_smem_bytes(a.W, a.m, a.d);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaFuncSetAttribute(k_seal, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
