@@ -203,6 +203,29 @@ long long ai_kernel_launches(void);
 int ai_quantize_fp8(const uint16_t* keys_bf16_dev, int64_t n, int32_t d, uint8_t* codes_dev,
                     float* scales_dev, void* cuda_stream);
 
+/* ----------------------------------------------- allocation-free variant */
+/* Exhaustive selection for callers that cannot allocate device memory (for
+ * example a server whose memory all comes from its own pre-reserved pool, or
+ * a latency-critical path that must not hit the implicit synchronisation of
+ * cudaMalloc / cudaFree).  No counterpart in the paper: it is a deployment
+ * convenience with the same results as ai_select_exhaustive on the same
+ * keys.  It needs no handle and calls no allocator: its only scratch is a
+ * fixed 16 MiB device array inside the library, present on every device
+ * that loads the library until the process exits.
+ *   keys_dev: [n_keys, d] keys owned by the caller: AI_BF16 (d = 128,
+ *     H in {32, 64}, bf16 queries) or AI_FP32 (fp32 queries); n_keys at
+ *     most 1,048,576 (AI_ERR_ARG beyond).
+ *   q_dev [T, H, d], w_dev [T, H], pos0, T, k, out_dev [T, k],
+ *   out_scores_dev [T, k] or NULL: as for ai_select_exhaustive.
+ * Enqueued on cuda_stream.  The first call on a device looks up the
+ * array's device address (make it before any stream capture).  All calls
+ * share the array: calls whose work overlaps on the GPU (other streams,
+ * other threads) race and must be serialised by the caller.              */
+int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_t n_keys,
+                                 int32_t d, int32_t H, const void* q_dev, const float* w_dev,
+                                 int64_t pos0, int32_t T, int32_t k, int32_t* out_dev,
+                                 float* out_scores_dev, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

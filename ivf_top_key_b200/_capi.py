@@ -29,7 +29,7 @@ EXPORTED = [
     "ai_publish", "ai_route_refine", "ai_select_exhaustive", "ai_sync", "ai_last_error",
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
-    "ai_kernel_launches",
+    "ai_kernel_launches", "ai_select_exhaustive_noalloc",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
 
@@ -84,6 +84,7 @@ def _load():
         "ai_quantize_fp8": [vp, i64, i32, vp, vp, vp],
         "ai_profile_enable": [vp, ctypes.c_int],
         "ai_profile_read": [vp, vp, vp],
+        "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -226,6 +227,16 @@ def ai_profile_read(h) -> dict:
 
 def ai_kernel_launches() -> int:
     return int(_lib.ai_kernel_launches())
+
+
+def ai_select_exhaustive_noalloc(keys, key_dtype: int, q, w, pos0: int, k: int, out,
+                                 out_scores=None, stream=None):
+    """Exhaustive selection without any device allocation (see the header)."""
+    n, d = keys.shape[0], keys.shape[1]
+    _check(_lib.ai_select_exhaustive_noalloc(_ptr(keys), key_dtype, n, d, q.shape[1], _ptr(q), _ptr(w),
+                                             pos0, q.shape[0], k, _ptr(out), _ptr(out_scores),
+                                             _stream(stream)))
+    return out
 
 
 def ai_last_error() -> str:

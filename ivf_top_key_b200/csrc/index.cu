@@ -31,15 +31,18 @@
 
 using namespace aiidx;
 
+namespace {
+thread_local std::string g_err;
+}  // namespace
+
 namespace aiidx {
 static std::atomic<long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 long long kernel_launches() { return g_launches.load(std::memory_order_relaxed); }
+void set_last_error(const char* msg) { g_err = msg; }
 }  // namespace aiidx
 
 namespace {
-
-thread_local std::string g_err;
 
 int fail(int code, const std::string& msg) {
   g_err = msg;
@@ -575,6 +578,7 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   const bool tck = tcr && c.key_dtype != AI_FP32;
   if (refine_smem_bytes(c.max_budget, c.H, c.d, tck) > 227 * 1024)
     return fail(AI_ERR_ARG, "max_budget too large for the per-query kernel");
+  if (tck && c.max_k > 2048) return fail(AI_ERR_ARG, "k above 2048 is not supported for bf16/fp8 keys");
 
   ai_index* h = new ai_index();
   h->cfg = c;

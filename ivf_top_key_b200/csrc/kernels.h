@@ -10,6 +10,8 @@ namespace aiidx {
 // Kernel launches made by this library (all handles, all streams).
 void count_launch();
 long long kernel_launches();
+// Message returned by ai_last_error() on this thread.
+void set_last_error(const char* msg);
 
 // ---------------------------------------------------------- score matrices
 struct ScoreArgs {
