@@ -29,7 +29,7 @@
 namespace aiidx {
 namespace {
 
-constexpr int kSortCap = 4096;
+constexpr int kSortCap = 2048;  // ranked clusters per query (size-capped at ~W/m keys each)
 constexpr int kTile = 128;
 constexpr int kStages = 3;
 constexpr int kTcThreads = 288;   // warps 0-3 gather, 4 UMMA, 5-8 epilogue
@@ -77,11 +77,51 @@ __device__ __forceinline__ void version_of(const VersionTable& vt, int64_t t, in
 // exactly and the fill stops at C.
 constexpr int kNB1 = 2048;
 struct P1Smem {
+  int32_t coff[kSortCap];  // member offset of each ranked cluster
   uint32_t hist[kNB1];
   float fred[32];
   unsigned long long wred[16];
   int scal[4];
 };
+
+// Warp 0 scans the weighted histogram ps.hist from the top for the bin
+// where the weight reaches `need`: its index and the weight above it.
+// All threads call it (it ends with a barrier).
+__device__ void p1_find_bin(P1Smem& ps, int need, int* bstar, int* above) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    uint32_t lsum = 0;
+    for (int b = 0; b < 64; ++b) lsum += ps.hist[lane * 64 + b];
+    uint32_t incl = lsum;  // sum over lanes >= this one
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += v;
+    }
+    uint32_t cum = incl - lsum;
+    int found = -1;
+    uint32_t ab = 0;
+    for (int b = lane * 64 + 63; b >= lane * 64; --b) {
+      const uint32_t h = ps.hist[b];
+      if (found < 0 && cum < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= cum + h) {
+        found = b;
+        ab = cum;
+      }
+      cum += h;
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = who ? __ffs(who) - 1 : 0;
+    const int fb = __shfl_sync(0xffffffffu, found, src);
+    const uint32_t fa = __shfl_sync(0xffffffffu, ab, src);
+    if (lane == 0) {
+      ps.scal[0] = who ? fb : 0;
+      ps.scal[2] = static_cast<int>(fa);
+    }
+  }
+  __syncthreads();
+  *bstar = ps.scal[0];
+  *above = ps.scal[2];
+  __syncthreads();
+}
 
 __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, int64_t n_v,
                                 int32_t* cand, uint64_t* sortbuf, int32_t* pref,
@@ -108,10 +148,11 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   // pass A: score range and total size of the non-empty clusters
   float vmin = INFINITY, vmax = -INFINITY;
   unsigned long long wsum = 0;
+#pragma unroll 4
   for (int c = tid; c < nC; c += blockDim.x) {
-    const int sz = off[c + 1] - off[c];
+    const int sz = __ldg(off + c + 1) - __ldg(off + c);
+    const float v = __ldg(rs + c);
     if (sz > 0) {
-      const float v = rs[c];
       vmin = fminf(vmin, v);
       vmax = fmaxf(vmax, v);
       wsum += static_cast<unsigned long long>(sz);
@@ -139,58 +180,89 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   }
   const bool take_all = wsum <= static_cast<unsigned long long>(rem);
   const float scale = vmax > vmin ? static_cast<float>(kNB1) / (vmax - vmin) : 0.f;
+  // bin positions use explicitly rounded operations (no FMA contraction), so
+  // every pass computes the same bin for the same score
+  auto pos1 = [&](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
   auto binof = [&](float v) -> int {
-    const int b = static_cast<int>((v - vmin) * scale);
+    const int b = static_cast<int>(pos1(v));
     return b < kNB1 - 1 ? b : kNB1 - 1;
   };
-  int bstar = 0;
+  int bstar = 0, bstar2 = 0;
+  auto bin2 = [&](float v) -> int {
+    const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), static_cast<float>(bstar)),
+                                             static_cast<float>(kNB1)));
+    return b < 0 ? 0 : (b < kNB1 - 1 ? b : kNB1 - 1);
+  };
   if (!take_all) {
     // pass B: size-weighted histogram; the bin where the weight from the top
     // reaches the remaining budget
-    for (int c = tid; c < nC; c += blockDim.x) {
-      const int sz = off[c + 1] - off[c];
-      if (sz > 0) atomicAdd(&ps.hist[binof(rs[c])], static_cast<uint32_t>(sz));
+    for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+      float v[4];
+      int sz[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * blockDim.x;
+        sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
+        v[u] = c < nC ? __ldg(rs + c) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (sz[u] > 0) atomicAdd(&ps.hist[binof(v[u])], static_cast<uint32_t>(sz[u]));
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins [64 l, 64 l + 64), scanned from the top
-      uint32_t lsum = 0;
-      for (int b = 0; b < 64; ++b) lsum += ps.hist[lane * 64 + b];
-      uint32_t incl = lsum;  // suffix sum over lanes >= l
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += v;
+    int above1 = 0;
+    p1_find_bin(ps, rem, &bstar, &above1);
+    // pass B2: the boundary bin split into kNB1 sub-bins (a long score tail
+    // leaves most clusters in few level-1 bins)
+    for (int i = tid; i < kNB1; i += blockDim.x) ps.hist[i] = 0;
+    __syncthreads();
+    for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+      float v[4];
+      int sz[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * blockDim.x;
+        sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
+        v[u] = c < nC ? __ldg(rs + c) : 0.f;
       }
-      uint32_t cum = incl - lsum;  // weight in bins above this lane's range
-      int found = -1;
-      for (int b = lane * 64 + 63; b >= lane * 64; --b) {
-        const uint32_t h = ps.hist[b];
-        if (found < 0 && cum < static_cast<uint32_t>(rem) && static_cast<uint32_t>(rem) <= cum + h) found = b;
-        cum += h;
-      }
-      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
-      const int fb = __shfl_sync(0xffffffffu, found, who ? __ffs(who) - 1 : 0);
-      if (lane == 0) ps.scal[0] = who ? fb : 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (sz[u] > 0 && binof(v[u]) == bstar) atomicAdd(&ps.hist[bin2(v[u])], static_cast<uint32_t>(sz[u]));
     }
     __syncthreads();
-    bstar = ps.scal[0];
+    int above2 = 0;
+    p1_find_bin(ps, rem - above1, &bstar2, &above2);
   }
-  // pass C: clusters at or above the boundary bin, in id order
-  int nsel = 0;
-  for (int base = 0; base < nC; base += blockDim.x) {
-    const int c = base + tid;
-    bool p = false;
-    float v = 0.f;
-    if (c < nC && off[c + 1] > off[c]) {
-      v = rs[c];
-      p = take_all || binof(v) >= bstar;
+  auto selected = [&](float v) -> bool {
+    if (take_all) return true;
+    const int b = binof(v);
+    if (b != bstar) return b > bstar;
+    return bin2(v) >= bstar2;
+  };
+  // pass C: clusters at or above the boundary bin (any order: sorted next)
+  if (tid == 0) ps.scal[1] = 0;
+  __syncthreads();
+  for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+    float v[4];
+    int sz[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * blockDim.x;
+      sz[u] = c < nC ? off[c + 1] - off[c] : 0;
+      v[u] = c < nC ? rs[c] : 0.f;
     }
-    int total;
-    const int r = block_rank(p, &total, bs);
-    if (p && nsel + r < kSortCap)
-      sortbuf[nsel + r] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(c);
-    nsel += total;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * blockDim.x;
+      if (sz[u] > 0 && selected(v[u])) {
+        const int pos = atomicAdd(&ps.scal[1], 1);
+        if (pos < kSortCap)
+          sortbuf[pos] = (static_cast<uint64_t>(~f2key(v[u])) << 32) | static_cast<uint32_t>(c);
+      }
+    }
   }
+  __syncthreads();
+  int nsel = ps.scal[1];
   if (nsel > kSortCap) {
     if (tid == 0) atomicOr(a.err, DEV_ERR_CAPACITY);
     nsel = kSortCap;
@@ -200,12 +272,21 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   for (int i = nsel + tid; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
   __syncthreads();
   bitonic_sort_u64(sortbuf, np);
-  // exclusive prefix of member counts in rank order
+  // member offsets and sizes of the ranked clusters (parallel loads), then
+  // the exclusive prefix of sizes in rank order
+  int32_t* coff = ps.coff;
+  for (int r = tid; r < nsel; r += blockDim.x) {
+    const int c = static_cast<int>(sortbuf[r] & 0xffffffffu);
+    const int o0 = off[c];
+    coff[r] = o0;
+    pref[r] = off[c + 1] - o0;
+  }
+  __syncthreads();
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < nsel; base += 32) {
       const int r = base + lane;
-      const int v = r < nsel ? off[(sortbuf[r] & 0xffffffffu) + 1] - off[sortbuf[r] & 0xffffffffu] : 0;
+      const int v = r < nsel ? pref[r] : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -219,17 +300,31 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   }
   __syncthreads();
   const int len = static_cast<int>(min64(C, static_cast<int64_t>(fixed) + pref[nsel]));
-  // flat fill: slot -> rank r (binary search over pref) -> member
-  for (int slot = fixed + tid; slot < len; slot += blockDim.x) {
-    const int x = slot - fixed;
-    int lo = 0, hi = nsel - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pref[mid] <= x) lo = mid;
-      else hi = mid - 1;
+  // flat fill: slot -> rank r (binary search over pref) -> member; four
+  // independent loads in flight per thread
+  for (int s0 = fixed + tid; s0 < len; s0 += 4 * blockDim.x) {
+    int src[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int slot = s0 + u * blockDim.x;
+      src[u] = -1;
+      if (slot < len) {
+        const int x = slot - fixed;
+        int lo = 0, hi = nsel - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (pref[mid] <= x) lo = mid;
+          else hi = mid - 1;
+        }
+        src[u] = coff[lo] + (x - pref[lo]);
+      }
     }
-    const int c = static_cast<int>(sortbuf[lo] & 0xffffffffu);
-    cand[slot] = a.members[off[c] + (x - pref[lo])];
+    int32_t mv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) mv[u] = src[u] >= 0 ? __ldg(a.members + src[u]) : 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (src[u] >= 0) cand[s0 + u * blockDim.x] = mv[u];
   }
   __syncthreads();
   return len;
@@ -383,7 +478,7 @@ __device__ __forceinline__ void gather_tile_fp8(const RefineArgs& a, const int32
 // to get the exact threshold; rare overflow and tie cases use a radix
 // select over the same items.  Ties at the threshold go to the lower key id.
 constexpr int kNB = 2048;     // histogram bins
-constexpr int kCapB = 2048;   // items of the threshold bin sorted in smem
+constexpr int kCapB = 2048;   // items of the threshold bin sorted in smem (>= k/2)
 
 struct P3Smem {
   uint32_t hist[kNB];
@@ -480,6 +575,31 @@ __device__ uint32_t p3_radix(const P3Ctx& c, int et, Pred pred, Key key, int nee
   return prefix;
 }
 
+// The bin of ps.hist (kNB bins, scanned from the top) holding the k-th
+// item: its index, the count above it, and its own count.  All 128
+// epilogue threads call it; thread et owns bins [16 et, 16 et + 16).
+__device__ void p3_find_bin(P3Smem& ps, int et, int k, int* bstar, int* above, int* nb) {
+  int tsum = 0;
+  for (int b = 0; b < 16; ++b) tsum += static_cast<int>(ps.hist[16 * et + b]);
+  int tot;
+  const int before = p3_scan(tsum, et, &tot, ps);
+  int cum = tot - before - tsum;
+  for (int b = 16 * et + 15; b >= 16 * et; --b) {
+    const int h = static_cast<int>(ps.hist[b]);
+    if (cum < k && k <= cum + h) {
+      ps.scal[0] = b;
+      ps.scal[1] = cum;
+      ps.scal[2] = h;
+    }
+    cum += h;
+  }
+  named_bar(1, 128);
+  *bstar = ps.scal[0];
+  *above = ps.scal[1];
+  *nb = ps.scal[2];
+  named_bar(1, 128);
+}
+
 __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3Smem& ps) {
   const int k = a.k;
   int32_t* out = a.out + static_cast<int64_t>(qi) * k;
@@ -508,46 +628,52 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   bool ties_all = true;
   if (!take_all) {
     const float scale = vmax > vmin ? static_cast<float>(kNB) / (vmax - vmin) : 0.f;
+    // explicitly rounded (never contracted): the same score always lands in
+    // the same bin in every pass
+    auto pos1 = [&](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
     auto binof = [&](float v) -> int {
-      const int b = static_cast<int>((v - vmin) * scale);
+      const int b = static_cast<int>(pos1(v));
       return b < kNB - 1 ? b : kNB - 1;
     };
+    // level 1 over [vmin, vmax]; level 2 splits the level-1 bin that holds
+    // the k-th score into kNB sub-bins (a long score tail leaves the bulk
+    // in few level-1 bins)
     for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
     if (et == 0) ps.cnt = 0;
     named_bar(1, 128);
     p3_for_each(c, [&](float v, int) { atomicAdd(&ps.hist[binof(v)], 1u); });
     named_bar(1, 128);
-    // bin holding the k-th largest: thread et owns bins [16 et, 16 et + 16)
-    int tsum = 0;
-    for (int b = 0; b < 16; ++b) tsum += static_cast<int>(ps.hist[16 * et + b]);
-    int tot;
-    const int before = p3_scan(tsum, et, &tot, ps);
-    int cum = tot - before - tsum;  // items in bins above this thread's range
-    for (int b = 16 * et + 15; b >= 16 * et; --b) {
-      const int h = static_cast<int>(ps.hist[b]);
-      if (cum < k && k <= cum + h) {
-        ps.scal[0] = b;
-        ps.scal[1] = cum;
-        ps.scal[2] = h;
-      }
-      cum += h;
-    }
+    int above_b = 0, bstar = 0, nb = 0;
+    p3_find_bin(ps, et, k, &bstar, &above_b, &nb);
+    const float b1f = static_cast<float>(bstar);
+    auto bin2 = [&](float v) -> int {
+      const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), b1f), static_cast<float>(kNB)));
+      return b < 0 ? 0 : (b < kNB - 1 ? b : kNB - 1);
+    };
+    for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
     named_bar(1, 128);
-    const int bstar = ps.scal[0], above_b = ps.scal[1], nb = ps.scal[2];
+    p3_for_each(c, [&](float v, int) {
+      if (binof(v) == bstar) atomicAdd(&ps.hist[bin2(v)], 1u);
+    });
+    named_bar(1, 128);
+    int bstar2 = 0, above2 = 0, nb2 = 0;
+    p3_find_bin(ps, et, k - above_b, &bstar2, &above2, &nb2);
+    above_b += above2;
+    auto in_b = [&](float v) -> bool { return binof(v) == bstar && bin2(v) == bstar2; };
     const int need = k - above_b;
     int above_in = 0, eq = 0;
     uint32_t tkey;
-    if (nb <= kCapB) {
+    if (nb2 <= kCapB) {
       p3_for_each(c, [&](float v, int slot) {
-        if (binof(v) == bstar) {
+        if (in_b(v)) {
           const unsigned long long pos = atomicAdd(&ps.cnt, 1ull);
           ps.buf[pos] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(slot);
         }
       });
       named_bar(1, 128);
       int np = 1;
-      while (np < nb) np <<= 1;
-      for (int i = nb + et; i < np; i += 128) ps.buf[i] = ~0ull;
+      while (np < nb2) np <<= 1;
+      for (int i = nb2 + et; i < np; i += 128) ps.buf[i] = ~0ull;
       named_bar(1, 128);
       for (int kk = 2; kk <= np; kk <<= 1) {
         for (int j = kk >> 1; j > 0; j >>= 1) {
@@ -569,7 +695,7 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
         int i0 = need - 1;
         while (i0 > 0 && ~static_cast<uint32_t>(ps.buf[i0 - 1] >> 32) == tkey) --i0;
         int i1 = need - 1;
-        while (i1 + 1 < nb && ~static_cast<uint32_t>(ps.buf[i1 + 1] >> 32) == tkey) ++i1;
+        while (i1 + 1 < nb2 && ~static_cast<uint32_t>(ps.buf[i1 + 1] >> 32) == tkey) ++i1;
         ps.scal[6] = i0;
         ps.scal[7] = i1 - i0 + 1;
       }
@@ -578,11 +704,11 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       eq = ps.scal[7];
     } else {
       tkey = p3_radix(
-          c, et, [&](float v, int) { return binof(v) == bstar; },
-          [&](float v, int) { return f2key(v); }, need, &above_in, &eq, ps);
+          c, et, [&](float v, int) { return in_b(v); }, [&](float v, int) { return f2key(v); }, need,
+          &above_in, &eq, ps);
     }
     theta = key2f(tkey);
-    const int need_eq = k - above_b - above_in;
+    const int need_eq = k - above_b - above_in;  // above_b spans both levels
     if (eq > need_eq) {
       ties_all = false;
       int ab2 = 0, eq2 = 0;
@@ -593,7 +719,8 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       theta_id = static_cast<int>(~idk);
     }
   }
-  // emission: thread-major order, deterministic
+  // emission: ids staged in shared memory in thread-major order, then
+  // written out coalesced (deterministic order)
   auto sel = [&](float v, int slot) {
     return take_all || v > theta || (v == theta && (ties_all || c.cand[slot] <= theta_id));
   };
@@ -601,19 +728,24 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   p3_for_each(c, [&](float v, int slot) { mine += sel(v, slot) ? 1 : 0; });
   int total;
   int pos = p3_scan(mine, et, &total, ps);
+  int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] ids
+  float* ssc = reinterpret_cast<float*>(ps.buf) + kCapB;       // [k] scores
   p3_for_each(c, [&](float v, int slot) {
     if (sel(v, slot)) {
       if (pos < k) {
-        out[pos] = c.cand[slot];
-        if (outs) outs[pos] = v;
+        sid[pos] = c.cand[slot];
+        ssc[pos] = v;
       }
       ++pos;
     }
   });
-  for (int j = min(total, k) + et; j < k; j += 128) {
-    out[j] = -1;
-    if (outs) outs[j] = -INFINITY;
+  named_bar(1, 128);
+  const int nw = min(total, k);
+  for (int j = et; j < k; j += 128) {
+    out[j] = j < nw ? sid[j] : -1;
+    if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
   }
+  named_bar(1, 128);
 }
 
 // Layout of the tensor-core kernel (one region reused by the three phases).

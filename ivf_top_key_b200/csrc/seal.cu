@@ -7,7 +7,8 @@
 // pages give no algorithm; the reading implemented here:
 //   init    c_j = x[floor((j + 1/2) W / m)]
 //   repeat  at most `iters` times, stopping when the assignment repeats:
-//           D_ij = ||x_i - c_j||^2 (float64)
+//           D_ij = ||x_i - c_j||^2 (float64; evaluated as
+//                  ||x||^2 - 2 x.c + ||c||^2, clamped at 0)
 //           visit all (i, j) pairs by (D asc, i asc, j asc); key i joins
 //           cluster j if i is still free and j has fewer than cap keys
 //           c_j = mean of its members (float64, ascending key order)
@@ -33,6 +34,7 @@ constexpr int kThreads = 1024;
 struct SealSmem {
   double* D;         // [W, m] squared distances
   double* cent;      // [m, d]
+  double* cc;        // [m] squared centre norms
   uint64_t* bk1;     // [m, NPW] proposal buckets: distance bits
   uint16_t* bk2;     // [m, NPW] proposal buckets: key
   int* wcnt;         // [m, 32] per-(cluster, warp) counts / offsets
@@ -51,6 +53,9 @@ struct SealSmem {
   int* red;          // [32] per-warp partial sums
   unsigned long long* fullmask;
 };
+
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __device__ __forceinline__ double key_f64(const SealArgs& a, int64_t s, int i) {
   double v = key_elem(a.keys, a.key_dtype, s, a.d, i);
@@ -103,6 +108,8 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
   p += static_cast<size_t>(W) * m * 8;
   s.cent = reinterpret_cast<double*>(p);
   p += static_cast<size_t>(m) * d * 8;
+  s.cc = reinterpret_cast<double*>(p);
+  p += static_cast<size_t>(m) * 8;
   s.bk1 = reinterpret_cast<uint64_t*>(p);
   p += static_cast<size_t>(m) * NPW * 8;
   s.fk1 = reinterpret_cast<uint64_t*>(p);
@@ -150,10 +157,19 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
   __syncthreads();
 
   for (int it = 0; it < a.iters; ++it) {
-    // distances: one key row per thread, read once in 8-element chunks,
-    // against all m centres (m <= 16 in registers, else one centre at a time)
+    // squared centre norms for this pass
+    for (int j = warp_id(); j < m; j += blockDim.x >> 5) {
+      double cc = 0.0;
+      for (int e = lane_id(); e < d; e += 32) cc = fma(s.cent[j * d + e], s.cent[j * d + e], cc);
+      for (int o = 16; o > 0; o >>= 1) cc += __shfl_xor_sync(0xffffffffu, cc, o);
+      if (lane_id() == 0) s.cc[j] = cc;
+    }
+    __syncthreads();
+    // distances ||x||^2 - 2 x.c + ||c||^2 (float64, clamped at 0): one key
+    // row per thread, read once, 32 elements per batch of loads
     for (int i = tid; i < W; i += blockDim.x) {
       const int64_t row = lo + i;
+      double xx = 0.0;
       if (m <= 16) {
         double acc[16];
 #pragma unroll
@@ -162,31 +178,33 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
           double x[8];
           load8(a, row, e0, x);
 #pragma unroll
+          for (int u = 0; u < 8; ++u) xx = fma(x[u], x[u], xx);
+#pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j < m) {
               const double* c = s.cent + j * d + e0;
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const double df = x[u] - c[u];
-                acc[j] = fma(df, df, acc[j]);
-              }
+              for (int u = 0; u < 8; ++u) acc[j] = fma(x[u], c[u], acc[j]);
             }
           }
         }
-        for (int j = 0; j < m; ++j) s.D[i * m + j] = acc[j];
+        for (int j = 0; j < m; ++j) s.D[i * m + j] = fmax(0.0, fma(-2.0, acc[j], xx) + s.cc[j]);
       } else {
+        for (int e0 = 0; e0 < d; e0 += 8) {
+          double x[8];
+          load8(a, row, e0, x);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) xx = fma(x[u], x[u], xx);
+        }
         for (int j = 0; j < m; ++j) {
           double acc = 0.0;
           for (int e0 = 0; e0 < d; e0 += 8) {
             double x[8];
             load8(a, row, e0, x);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const double df = x[u] - s.cent[j * d + e0 + u];
-              acc = fma(df, df, acc);
-            }
+            for (int u = 0; u < 8; ++u) acc = fma(x[u], s.cent[j * d + e0 + u], acc);
           }
-          s.D[i * m + j] = acc;
+          s.D[i * m + j] = fmax(0.0, fma(-2.0, acc, xx) + s.cc[j]);
         }
       }
       s.assign[i] = -1;
@@ -247,47 +265,41 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         if (tid < m) s.bfill[tid] += s.bpass[tid];
         __syncthreads();
       }
-      // 2. one warp per open cluster: sort its bucket by (distance, key) and
-      //    take the proposal that would fill it
-      for (int j = warp; j < m; j += nwarps) {
-        const int nb = s.bfill[j];
+      // 2. the proposal that would fill each open cluster: the need-th
+      //    smallest (distance, key) of its bucket, found by counting ranks
+      //    (all threads; one entry each, compared against its bucket)
+      if (tid == 0) {
+        int run = 0;
+        for (int j = 0; j < m; ++j) {
+          s.tstart[j] = run;
+          run += s.bfill[j];
+        }
+        s.tstart[m] = run;
+      }
+      for (int j = tid; j < m; j += blockDim.x) {
+        s.fk1[j] = ~0ull;
+        s.fk2[j] = ~0u;
+      }
+      __syncthreads();
+      for (int e = tid; e < s.tstart[m]; e += blockDim.x) {
+        int j = 0;
+        while (j + 1 < m && s.tstart[j + 1] <= e) ++j;
         const int need = a.cap - s.cnt[j];
-        uint64_t* k1 = s.bk1 + j * NPW;
-        uint16_t* k2 = s.bk2 + j * NPW;
-        if (lane == 0) {
-          s.fk1[j] = ~0ull;
-          s.fk2[j] = ~0u;
-        }
+        const int nb = s.bfill[j];
         if (((fullm >> j) & 1ull) || nb < need || need <= 0) continue;
-        int np = 1;
-        while (np < nb) np <<= 1;
-        for (int q = nb + lane; q < np; q += 32) {
-          k1[q] = ~0ull;
-          k2[q] = 0xFFFFu;
+        const uint64_t* k1 = s.bk1 + j * NPW;
+        const uint16_t* k2 = s.bk2 + j * NPW;
+        const int me = e - s.tstart[j];
+        const uint64_t a1 = k1[me];
+        const uint16_t a2 = k2[me];
+        int rank = 0;
+        for (int x = 0; x < nb; ++x) {
+          const uint64_t b1 = k1[x];
+          rank += (b1 < a1 || (b1 == a1 && k2[x] < a2)) ? 1 : 0;
         }
-        __syncwarp();
-        for (int kk = 2; kk <= np; kk <<= 1) {
-          for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            for (int q = lane; q < np; q += 32) {
-              const int r = q ^ jj;
-              if (r > q) {
-                const uint64_t a1 = k1[q], b1 = k1[r];
-                const uint16_t a2 = k2[q], b2 = k2[r];
-                const bool b_less = b1 < a1 || (b1 == a1 && b2 < a2);
-                if (b_less == ((q & kk) == 0)) {
-                  k1[q] = b1;
-                  k1[r] = a1;
-                  k2[q] = b2;
-                  k2[r] = a2;
-                }
-              }
-            }
-            __syncwarp();
-          }
-        }
-        if (lane == 0) {
-          s.fk1[j] = k1[need - 1];
-          s.fk2[j] = (static_cast<uint32_t>(k2[need - 1]) << 16) | static_cast<uint32_t>(j);
+        if (rank == need - 1) {
+          s.fk1[j] = a1;
+          s.fk2[j] = (static_cast<uint32_t>(a2) << 16) | static_cast<uint32_t>(j);
         }
       }
       __syncthreads();
@@ -434,7 +446,7 @@ size_t seal_smem_bytes(int W, int m, int d) {
          static_cast<size_t>(m) * NPW * 10 + static_cast<size_t>(m) * 12 + 8 +
          static_cast<size_t>(m) * 32 * 4 + static_cast<size_t>(m) * 8 +
          static_cast<size_t>(m + 1) * 8 + 16 + 128 + static_cast<size_t>(W) * 6 +
-         static_cast<size_t>(m) * 32 + 256;
+         static_cast<size_t>(m) * 32 + 256 + static_cast<size_t>(m) * 8;
 }
 
 cudaError_t launch_seal(const SealArgs& a, cudaStream_t st) {
