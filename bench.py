@@ -48,6 +48,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=48, help="queries timed per oracle step")
+    p.add_argument("--budget", type=int, default=0, help="candidate budget C (0: the workload's)")
+    p.add_argument("--refit-overlap", action="store_true",
+                   help="also time one refit (64 seeds from the last 16384 keys) alone, the route "
+                        "alone and both together, and report the hidden fraction")
     return p.parse_args()
 
 
@@ -72,8 +76,27 @@ def config_block(wl, n):
             "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{n}"}
 
 
-def wl_for_rank(name, rank):
-    return S.scaled(S.WORKLOADS[name], seed=rank)
+def wl_for_rank(name, rank, budget=0):
+    """Every rank runs an independent request: same shapes, its own seed."""
+    wl = S.scaled(S.WORKLOADS[name], seed=rank)
+    return S.scaled(wl, budget=budget) if budget else wl
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity without a group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's timed device time."""
+    return world * units_per_rank * steps / (max_total_ms / 1e3)
 
 
 # ------------------------------------------------------------- inputs --
@@ -200,7 +223,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     from ivf_top_key_b200 import AttentionIndex, C as capi
-    wl = wl_for_rank(args.workload, rank)
+    wl = wl_for_rank(args.workload, rank, args.budget)
     T, L = wl.T, wl.L
     ncs = chunks_per_step(wl)
     p_first = L - ncs * T          # first position of the timed chunks
@@ -211,7 +234,8 @@ def run_ours(args):
                          refit_period=wl.refit_period, refit_new_seeds=0,
                          refit_seed_window=0, seal_iters=wl.seal_iters, async_refit=True,
                          max_query_chunk=T, max_budget=wl.budget, max_k=wl.k, max_keys=L,
-                         seed=wl.seed)
+                         seed=wl.seed,
+                         encoder_weights=S.encoder_weights(wl) if wl.encoder == "random" else None)
     # prefix before the timed chunks (untimed setup)
     for c in range(wl.n_chunks - ncs):
         kd, ks = chunk_keys_dev(wl, c * T, (c + 1) * T, dev)
@@ -268,13 +292,9 @@ def run_ours(args):
     phases = idx.profile_read()
     idx.sync()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(np.sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(np.sum(step_ms)), dev)
     units = T * ncs                # query tokens per step
-    value = world * units * args.steps / (total_ms / 1e3)
+    value = weak_scaling_value(units, args.steps, world, total_ms)
 
     # recall vs the in-library exhaustive selection (after the last step)
     exh = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
@@ -288,6 +308,10 @@ def run_ours(args):
     sel_c = (out.to(torch.int64) + rows)[out >= 0]
     exh_c = (exh.to(torch.int64) + rows)[exh >= 0]
     recall = float(torch.isin(exh_c, sel_c).sum().item() / max(1, exh_c.numel()))
+
+    refit_overlap = None
+    if args.refit_overlap:
+        refit_overlap = measure_refit_overlap(idx, chunks, wl, out, stream)
 
     # roofline of the dominant kernel (live phase events)
     peaks, peak_kind = measured_peaks()
@@ -364,16 +388,12 @@ def run_ours(args):
             e2e_step()
             ee[i][1].record(stream)
         torch.cuda.synchronize()
-        e_ms = float(np.sum([a.elapsed_time(b) for a, b in ee]))
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(float(np.sum([a.elapsed_time(b) for a, b in ee])), dev)
         h2d = sum(kh.numel() * kh.element_size() + qh.numel() * qh.element_size() +
                   wh.numel() * wh.element_size() + (sh.numel() * 4 if sh is not None else 0)
                   for _, kh, sh, qh, wh, _ in host)
         d2h = sum(oh.numel() * 4 for *_, oh in host)
-        e2e = {"value": world * units * args.steps / (e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": weak_scaling_value(units, args.steps, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms / args.steps}
 
@@ -396,6 +416,7 @@ def run_ours(args):
             "phases_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
             "dominant_phase": dom,
             "gpu_launches": int(launches), "gpu_launches_per_step": launches / args.steps,
+            "refit_overlap": refit_overlap,
             "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
             "wall_s_timed_region": round(t_wall, 3),
         }
@@ -403,6 +424,54 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_refit_overlap(idx, chunks, wl, out, stream, reps=3):
+    """One warm-started refit over the whole prefix (64 new seeds from the
+    last 16384 keys) on the side stream, concurrent with routing the final
+    chunk: hidden = (t_refit + t_route - t_both) / t_refit, all from CUDA
+    events on the main stream (the refit is joined by ai_publish)."""
+    import torch
+    idx.rollback()
+    for a, kd_, ks_, qd_, wd_ in chunks:
+        idx.append_keys(kd_, ks_)
+        idx.seal()
+    idx.publish()
+    idx.sync()
+    idx.checkpoint()
+    a, _, _, qd, wd = chunks[-1]
+
+    def timed(fn):
+        best = []
+        for _ in range(reps):
+            idx.rollback()
+            idx.sync()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            idx.sync()
+            best.append(e0.elapsed_time(e1))
+        return float(np.median(best))
+
+    def refit_only():
+        idx.refit(64, 16384)
+        idx.publish()
+
+    def route_only():
+        idx.route_refine(qd, wd, a, wl.k, wl.budget, out=out)
+
+    def both():
+        idx.refit(64, 16384)
+        idx.route_refine(qd, wd, a, wl.k, wl.budget, out=out)
+        idx.publish()
+
+    t_refit, t_route, t_both = timed(refit_only), timed(route_only), timed(both)
+    st = idx.stats()
+    return {"t_refit_ms": t_refit, "t_route_ms": t_route, "t_both_ms": t_both,
+            "hidden_fraction": (t_refit + t_route - t_both) / t_refit if t_refit > 0 else None,
+            "keys": st["n_keys"], "clusters_after": st["n_clusters"],
+            "keys_fully_scanned": st["last_refit_scanned"]}
 
 
 # --------------------------------------------------------- oracle arm --
@@ -422,7 +491,8 @@ def _oracle_prefix(wl):
                         clusters_per_window=wl.clusters_per_window,
                         refit_period=wl.refit_period, refit_new_seeds=wl.refit_new_seeds,
                         refit_seed_window=wl.refit_seed_window, seal_iters=wl.seal_iters,
-                        seed=wl.seed)
+                        seed=wl.seed,
+                        encoder=S.encoder_weights(wl) if wl.encoder == "random" else None)
     keys = oracle_keys(wl, 0, wl.L)
     for c in range(wl.n_chunks - chunks_per_step(wl)):
         orc.append(keys[c * wl.T:(c + 1) * wl.T])
