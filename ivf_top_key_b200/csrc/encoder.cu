@@ -19,16 +19,25 @@
 namespace aiidx {
 namespace {
 
-__global__ void k_encoder(EncoderArgs a) {
+constexpr int kEncThreads = 128;
+constexpr int kBatch = 8;
+
+// One CTA per cluster, thread o owns output feature o (d <= 128).  A is
+// staged in shared memory with padded rows (conflict-free column walks);
+// members are transformed 8 at a time; the MLP rows are read coalesced by
+// whole warps.
+__global__ void __launch_bounds__(kEncThreads) k_encoder(EncoderArgs a) {
   const int c = a.cl_begin + blockIdx.x;
   if (c >= a.cl_end) return;
   const int d = a.d, o = threadIdx.x;
+  const int lane = o & 31, warp = o >> 5;
   const int F = 3 * d + 1;
   extern __shared__ double sh[];
-  double* key = sh;          // [d]
-  double* f = sh + d;        // [3d + 1]
-  double* hv = f + F;        // [d]
-  double* red = hv + d;      // [d] reduction scratch
+  double* keyb = sh;                      // [kBatch][d]
+  double* f = keyb + kBatch * d;          // [3d + 1]
+  double* hv = f + F;                     // [d]
+  double* red = hv + d;                   // [8]
+  float* As = reinterpret_cast<float*>(red + 8);  // [d][d + 1]
   const float* A = a.wts;
   const float* av = A + d * d;
   const float* B1 = av + d;
@@ -37,55 +46,94 @@ __global__ void k_encoder(EncoderArgs a) {
   const float* b2 = B2 + d * d;
   const int o0 = a.offsets[c], o1 = a.offsets[c + 1];
   const int n = o1 - o0;
-  const double mu = a.centroids[static_cast<int64_t>(c) * d + o];
+  const bool act = o < d;
+  const double mu = act ? a.centroids[static_cast<int64_t>(c) * d + o] : 0.0;
   if (n <= 0) {
-    a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu);
+    if (act) a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu);
     return;
   }
-  double psum = 0.0, pmax = 0.0;  // phi >= 0, so 0 is a valid start for the max
-  for (int p = o0; p < o1; ++p) {
-    const int64_t s = a.members[p];
+  for (int e = o; e < d * d; e += blockDim.x) As[(e / d) * (d + 1) + (e % d)] = A[e];
+  const double ao = act ? static_cast<double>(av[o]) : 0.0;
+  double psum = 0.0, pmax = 0.0;  // phi >= 0, so 0 starts the max
+  for (int p0 = o0; p0 < o1; p0 += kBatch) {
+    const int nb = min(kBatch, o1 - p0);
     __syncthreads();
-    double v = key_elem(a.keys, a.key_dtype, s, d, o);
-    if (a.key_dtype == KD_FP8) v *= static_cast<double>(a.key_scale[s]);
-    key[o] = v;
+    for (int e = o; e < nb * d; e += blockDim.x) {
+      const int r = e / d, i = e % d;
+      const int64_t s = a.members[p0 + r];
+      double v = key_elem(a.keys, a.key_dtype, s, d, i);
+      if (a.key_dtype == KD_FP8) v *= static_cast<double>(a.key_scale[s]);
+      keyb[r * d + i] = v;
+    }
     __syncthreads();
-    double z = static_cast<double>(av[o]);
-    for (int i = 0; i < d; ++i) z = fma(static_cast<double>(A[o * d + i]), key[i], z);
-    z = z > 0.0 ? z : 0.0;
-    psum += z;
-    pmax = z > pmax ? z : pmax;
+    if (act) {
+      double z[kBatch];
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) z[r] = ao;
+      for (int i = 0; i < d; ++i) {
+        const double w = static_cast<double>(As[o * (d + 1) + i]);
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) z[r] = fma(w, keyb[r * d + i], z[r]);
+      }
+      for (int r = 0; r < nb; ++r) {
+        const double ph = z[r] > 0.0 ? z[r] : 0.0;
+        psum += ph;
+        pmax = ph > pmax ? ph : pmax;
+      }
+    }
   }
   __syncthreads();
-  f[o] = psum / static_cast<double>(n);
-  f[d + o] = pmax;
-  f[2 * d + o] = mu;
+  if (act) {
+    f[o] = psum / static_cast<double>(n);
+    f[d + o] = pmax;
+    f[2 * d + o] = mu;
+  }
   if (o == 0) f[3 * d] = log(static_cast<double>(n));
   __syncthreads();
-  double h = static_cast<double>(b1[o]);
-  for (int j = 0; j < F; ++j) h = fma(static_cast<double>(B1[static_cast<int64_t>(o) * F + j]), f[j], h);
-  hv[o] = h > 0.0 ? h : 0.0;
+  // h = ReLU(B1 f + b1): one warp per output row, lanes over the row
+  for (int r = warp; r < d; r += blockDim.x >> 5) {
+    double acc = 0.0;
+    for (int j = lane; j < F; j += 32)
+      acc = fma(static_cast<double>(B1[static_cast<int64_t>(r) * F + j]), f[j], acc);
+    for (int s2 = 16; s2 > 0; s2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s2);
+    if (lane == 0) {
+      const double h = acc + static_cast<double>(b1[r]);
+      hv[r] = h > 0.0 ? h : 0.0;
+    }
+  }
   __syncthreads();
-  double z = static_cast<double>(b2[o]);
-  for (int j = 0; j < d; ++j) z = fma(static_cast<double>(B2[o * d + j]), hv[j], z);
-  const double t = tanh(z);
-  // ||t|| and ||mu||
-  red[o] = t * t;
+  // z = B2 h + b2, t = tanh(z)
+  for (int r = warp; r < d; r += blockDim.x >> 5) {
+    double acc = 0.0;
+    for (int j = lane; j < d; j += 32) acc = fma(static_cast<double>(B2[r * d + j]), hv[j], acc);
+    for (int s2 = 16; s2 > 0; s2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s2);
+    if (lane == 0) f[r] = tanh(acc + static_cast<double>(b2[r]));  // reuse f[0..d) for t
+  }
   __syncthreads();
-  double tn2 = 0.0;
-  for (int j = 0; j < d; ++j) tn2 += red[j];
+  const double t = act ? f[o] : 0.0;
+  // ||t|| and ||mu|| (block reductions)
+  double tt = t * t, mm = mu * mu;
+  for (int s2 = 16; s2 > 0; s2 >>= 1) {
+    tt += __shfl_xor_sync(0xffffffffu, tt, s2);
+    mm += __shfl_xor_sync(0xffffffffu, mm, s2);
+  }
+  if (lane == 0) {
+    red[warp] = tt;
+    red[4 + warp] = mm;
+  }
   __syncthreads();
-  red[o] = mu * mu;
-  __syncthreads();
-  double mn2 = 0.0;
-  for (int j = 0; j < d; ++j) mn2 += red[j];
+  double tn2 = 0.0, mn2 = 0.0;
+  for (int w = 0; w < (kEncThreads >> 5); ++w) {
+    tn2 += red[w];
+    mn2 += red[4 + w];
+  }
   const double tn = sqrt(tn2);
   double corr = 0.0;
   if (tn > 0.0) {
     const double bound = 0.25 * sqrt(mn2);
     corr = t * (bound / tn < 1.0 ? bound / tn : 1.0);
   }
-  a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu + corr);
+  if (act) a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu + corr);
 }
 
 }  // namespace
@@ -93,10 +141,14 @@ __global__ void k_encoder(EncoderArgs a) {
 cudaError_t launch_encoder(const EncoderArgs& a, cudaStream_t st) {
   const int n = a.cl_end - a.cl_begin;
   if (n <= 0) return cudaSuccess;
-  if (a.d > 1024) return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(a.d * 3 + 3 * a.d + 1) * 8;
+  if (a.d > kEncThreads) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(kBatch * a.d + 3 * a.d + 1 + a.d + 8) * 8 +
+                      static_cast<size_t>(a.d) * (a.d + 1) * 4;
+  const cudaError_t e = cudaFuncSetAttribute(k_encoder, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   count_launch();
-  k_encoder<<<n, a.d, smem, st>>>(a);
+  k_encoder<<<n, kEncThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -566,6 +566,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
     return fail(AI_ERR_ARG, "bad sinks / window / clusters per window");
   if (c.refit_period < 0 || (c.refit_period > 0 && c.refit_period % c.window != 0))
     return fail(AI_ERR_ARG, "refit period must be a multiple of the window");
+  if ((c.refit_period > 0 || c.encoder_weights_host) && c.d > 128)
+    return fail(AI_ERR_ARG, "refit and the correction encoder support d <= 128");
   if (c.max_keys <= 0 || c.max_keys >= (int64_t(1) << 31)) return fail(AI_ERR_ARG, "bad max_keys");
   if (c.max_query_chunk <= 0 || c.max_budget <= 0 || c.max_k <= 0) return fail(AI_ERR_ARG, "bad maxima");
   int cap = c.cluster_cap > 0 ? c.cluster_cap : (c.window + c.clusters_per_window - 1) / c.clusters_per_window;

@@ -111,104 +111,106 @@ __global__ void k_test(RefitArgs a) {
   }
 }
 
-// Full scan in fp32: block = 64 keys x all centres in tiles of 64.
-// Thread (r, c) of a 16 x 16 grid covers keys 4r..4r+3 and centres
-// 4c..4c+3 of each tile.
-constexpr int kSK = 64, kSC = 64, kSD = 32;
+// Full scan in fp32: block = 64 keys x all centres in tiles of 64.  The
+// block's 64 key rows are staged once in shared memory (fp32, padded rows);
+// centre tiles stream through in 32-column slices.  Thread (r, c) of a
+// 16 x 16 grid covers keys 4r..4r+3 and centres 4c..4c+3 of each tile.
+constexpr int kSK = 64, kSC = 64, kSD = 32, kMaxD = 128;
 __global__ void __launch_bounds__(256) k_scan(RefitArgs a, int32_t* recheck, int32_t* n_recheck) {
-  __shared__ float xs[kSK][kSD + 1];
+  __shared__ float xs[kSK][kMaxD + 1];
   __shared__ float cs[kSC][kSD + 1];
   const int n = *a.n_scan;
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   for (int kb = blockIdx.x * kSK; kb < n; kb += gridDim.x * kSK) {
-  float best[4], second[4];
-  int bid[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    best[r] = INFINITY;
-    second[r] = INFINITY;
-    bid[r] = 0x7fffffff;
-  }
-  for (int c0 = 0; c0 < a.K; c0 += kSC) {
-    float acc[4][4] = {};
-    for (int d0 = 0; d0 < a.d; d0 += kSD) {
-      for (int e = threadIdx.x; e < kSK * kSD; e += blockDim.x) {
-        const int r = e / kSD, i = e % kSD;
-        const int kk = kb + r;
-        xs[r][i] = (kk < n && d0 + i < a.d) ? kf32(a, a.scan_list[kk], d0 + i) : 0.f;
-      }
-      for (int e = threadIdx.x; e < kSC * kSD; e += blockDim.x) {
-        const int r = e / kSD, i = e % kSD;
-        const int cc = c0 + r;
-        cs[r][i] = (cc < a.K && d0 + i < a.d) ? a.cent32[static_cast<int64_t>(cc) * a.d + d0 + i] : 0.f;
-      }
-      __syncthreads();
-#pragma unroll 4
-      for (int i = 0; i < kSD; ++i) {
-        float xv[4], cv[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) xv[r] = xs[tr * 4 + r][i];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) cv[c] = cs[tc * 4 + c][i];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float df = xv[r] - cv[c];
-            acc[r][c] = fmaf(df, df, acc[r][c]);
-          }
-      }
-      __syncthreads();
+    for (int e = threadIdx.x; e < kSK * a.d; e += blockDim.x) {
+      const int r = e / a.d, i = e % a.d;
+      const int kk = kb + r;
+      xs[r][i] = kk < n ? kf32(a, a.scan_list[kk], i) : 0.f;
     }
+    float best[4], second[4];
+    int bid[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int cc = c0 + tc * 4 + c;
-      if (cc >= a.K) continue;
+    for (int r = 0; r < 4; ++r) {
+      best[r] = INFINITY;
+      second[r] = INFINITY;
+      bid[r] = 0x7fffffff;
+    }
+    for (int c0 = 0; c0 < a.K; c0 += kSC) {
+      float acc[4][4] = {};
+      for (int d0 = 0; d0 < a.d; d0 += kSD) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < kSC * kSD; e += blockDim.x) {
+          const int r = e / kSD, i = e % kSD;
+          const int cc = c0 + r;
+          cs[r][i] = (cc < a.K && d0 + i < a.d) ? a.cent32[static_cast<int64_t>(cc) * a.d + d0 + i] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int i = 0; i < kSD; ++i) {
+          const bool in = d0 + i < a.d;
+          float xv[4], cv[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float v = acc[r][c];
-        if (v < best[r] || (v == best[r] && cc < bid[r])) {
-          second[r] = best[r];
-          best[r] = v;
-          bid[r] = cc;
-        } else if (v < second[r]) {
-          second[r] = v;
+          for (int r = 0; r < 4; ++r) xv[r] = in ? xs[tr * 4 + r][d0 + i] : 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) cv[c] = cs[tc * 4 + c][i];
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float df = xv[r] - cv[c];
+              acc[r][c] = fmaf(df, df, acc[r][c]);
+            }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int cc = c0 + tc * 4 + c;
+        if (cc >= a.K) continue;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float v = acc[r][c];
+          if (v < best[r] || (v == best[r] && cc < bid[r])) {
+            second[r] = best[r];
+            best[r] = v;
+            bid[r] = cc;
+          } else if (v < second[r]) {
+            second[r] = v;
+          }
         }
       }
     }
-  }
-  // merge across the 16 threads of a row (consecutive lanes)
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    for (int o = 8; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best[r], o);
-      const float os = __shfl_xor_sync(0xffffffffu, second[r], o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bid[r], o);
-      if (ob < best[r] || (ob == best[r] && oi < bid[r])) {
-        second[r] = fminf(best[r], os);
-        best[r] = ob;
-        bid[r] = oi;
-      } else {
-        second[r] = fminf(second[r], ob);
-      }
-    }
-  }
-  if (tc == 0) {
+    // merge across the 16 threads of a row (consecutive lanes)
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int kk = kb + tr * 4 + r;
-      if (kk >= n) continue;
-      const int32_t x = a.scan_list[kk];
-      a.assign[x] = bid[r];
-      if (second[r] - best[r] <= kRel * second[r] + 1e-30f) {
-        const int p = atomicAdd(n_recheck, 1);
-        recheck[p] = x;
+      for (int o = 8; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best[r], o);
+        const float os = __shfl_xor_sync(0xffffffffu, second[r], o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bid[r], o);
+        if (ob < best[r] || (ob == best[r] && oi < bid[r])) {
+          second[r] = fminf(best[r], os);
+          best[r] = ob;
+          bid[r] = oi;
+        } else {
+          second[r] = fminf(second[r], ob);
+        }
       }
-      a.ub[x] = __fmul_ru(sqrtf(best[r]), 1.f + kRel);
-      a.lb[x] = __fmul_rd(sqrtf(second[r]), 1.f - kRel);
     }
-  }
-  __syncthreads();
+    if (tc == 0) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int kk = kb + tr * 4 + r;
+        if (kk >= n) continue;
+        const int32_t x = a.scan_list[kk];
+        a.assign[x] = bid[r];
+        if (second[r] - best[r] <= kRel * second[r] + 1e-30f) {
+          const int p = atomicAdd(n_recheck, 1);
+          recheck[p] = x;
+        }
+        a.ub[x] = __fmul_ru(sqrtf(best[r]), 1.f + kRel);
+        a.lb[x] = __fmul_rd(sqrtf(second[r]), 1.f - kRel);
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -382,24 +384,78 @@ __global__ void k_scatter(RefitArgs a) {
   }
 }
 
-// one warp per cluster: float64 mean in member order, drift, bf16 rep
+// Four consecutive key elements [e, e + 4) as float64 (d % 4 == 0).
+__device__ __forceinline__ void load4_f64(const RefitArgs& a, int64_t row, int e, double* x) {
+  if (a.key_dtype == KD_BF16) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.keys) + row * a.d + e));
+    x[0] = __uint_as_float(v.x << 16);
+    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(v.y << 16);
+    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  } else if (a.key_dtype == KD_FP8) {
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(a.keys) + row * a.d + e));
+    const double sc = static_cast<double>(__ldg(a.key_scale + row));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = static_cast<double>(fp8_to_f32(static_cast<uint8_t>(v >> (8 * u)))) * sc;
+  } else {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.keys) + row * a.d + e));
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
+  }
+}
+
+// One warp per cluster: float64 member sums in member (CSR) order, lanes
+// over 4-element column blocks, member ids fetched 32 at a time and four
+// member rows in flight; then mean, drift and the bf16 representative.
 __global__ void k_update(RefitArgs a, unsigned long long* max_drift_bits) {
   const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (j >= a.K) return;
   const int o0 = a.offsets[j], o1 = a.offsets[j + 1];
   double dr = 0.0;
-  for (int i = lane; i < a.d; i += 32) {
-    const int64_t e = static_cast<int64_t>(j) * a.d + i;
-    double v = a.cent[e];
-    if (o1 > o0) {
-      double sum = 0.0;
-      for (int p = o0; p < o1; ++p) sum += kf64(a, a.members[p], i);
-      v = sum / static_cast<double>(o1 - o0);
+  for (int e0 = 0; e0 < a.d; e0 += 128) {
+    const int e = e0 + lane * 4;
+    const bool act = e < a.d;
+    double sum[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int p0 = o0; p0 < o1; p0 += 32) {
+      const int nb = min(32, o1 - p0);
+      const int myid = lane < nb ? a.members[p0 + lane] : 0;
+      int u = 0;
+      for (; u + 4 <= nb; u += 4) {
+        double x[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int id = __shfl_sync(0xffffffffu, myid, u + r);
+          if (act) load4_f64(a, id, e, x[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sum[c] += x[r][c];
+      }
+      for (; u < nb; ++u) {
+        const int id = __shfl_sync(0xffffffffu, myid, u);
+        double x[4];
+        if (act) {
+          load4_f64(a, id, e, x);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sum[c] += x[c];
+        }
+      }
     }
-    const double df = v - a.cent_old[e];
-    dr = fma(df, df, dr);
-    a.cent[e] = v;
-    a.reps[e] = f64_to_bf16_rne(v);
+    if (act) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int64_t idx = static_cast<int64_t>(j) * a.d + e + c;
+        double v = a.cent[idx];
+        if (o1 > o0) v = sum[c] / static_cast<double>(o1 - o0);
+        const double df = v - a.cent_old[idx];
+        dr = fma(df, df, dr);
+        a.cent[idx] = v;
+        a.reps[idx] = f64_to_bf16_rne(v);
+      }
+    }
   }
   for (int o = 16; o > 0; o >>= 1) dr += __shfl_xor_sync(0xffffffffu, dr, o);
   if (lane == 0) {
@@ -428,7 +484,7 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   if (n <= 0 || a.K <= 0) return cudaSuccess;
   const int64_t ntiles = (n + kTileKeys - 1) / kTileKeys;
   if (ntiles > max_tiles) return cudaErrorInvalidValue;
-  if (static_cast<size_t>(a.K) * 4 > 200 * 1024) return cudaErrorInvalidValue;
+  if (static_cast<size_t>(a.K) * 4 > 200 * 1024 || a.d > 128 || a.d % 4 != 0) return cudaErrorInvalidValue;
   // scratch words after n_scan: [1] n_recheck, [2..3] max drift bits
   int32_t* n_recheck = a.n_scan + 1;
   unsigned long long* mdb = reinterpret_cast<unsigned long long*>(a.n_scan + 2);
