@@ -172,7 +172,7 @@ int ai_debug_scores(ai_handle h, const void* q_dev, const float* w_dev, int64_t 
                     float* out_dev);
 
 /* Checkpoint / rollback of the index state (host counters, version table,
- * active cluster buffer and per-key refit bounds).  Rollback forgets keys
+ * active cluster buffer, per-key refit bounds and the last centre drifts).  Rollback forgets keys
  * appended after the checkpoint (they must be appended again).  Fails with
  * AI_ERR_STATE while a refit is pending at checkpoint time.               */
 int ai_checkpoint(ai_handle h);

@@ -213,6 +213,7 @@ struct ai_index {
   int32_t* ck_assign = nullptr;
   float* ck_ub = nullptr;
   float* ck_lb = nullptr;
+  double* ck_drift = nullptr;  // the next refit's bounds read the last drifts
 };
 
 namespace {
@@ -692,6 +693,7 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->ck_assign);
   cudaFree(h->ck_ub);
   cudaFree(h->ck_lb);
+  cudaFree(h->ck_drift);
   for (auto& r : h->recs) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -944,7 +946,9 @@ int ai_checkpoint(ai_handle h) {
     CK(dalloc(&h->ck_assign, N));
     CK(dalloc(&h->ck_ub, N));
     CK(dalloc(&h->ck_lb, N));
+    CK(dalloc(&h->ck_drift, h->maxC));
   }
+  CK(cudaMemcpyAsync(h->ck_drift, h->drift, h->maxC * sizeof(double), cudaMemcpyDeviceToDevice, h->main));
   Checkpoint& c = h->ck;
   c.valid = true;
   c.n_keys = h->n_keys;
@@ -986,6 +990,7 @@ int ai_rollback(ai_handle h) {
     b.first_window = m.first_window;
     b.versions = m.versions;
   }
+  CK(cudaMemcpyAsync(h->drift, h->ck_drift, h->maxC * sizeof(double), cudaMemcpyDeviceToDevice, h->main));
   if (h->n_keys > 0) {
     CK(cudaMemcpyAsync(h->assign, h->ck_assign, h->n_keys * 4, cudaMemcpyDeviceToDevice, h->main));
     CK(cudaMemcpyAsync(h->ub, h->ck_ub, h->n_keys * 4, cudaMemcpyDeviceToDevice, h->main));

@@ -16,17 +16,27 @@
 // (rounded outward, with a relative margin), distances are screened in fp32
 // and every near tie is decided again in float64.
 //
+// Bounds.  For a key with centre a: u >= d(x, c_a) at the current centre
+// positions, and l is a lower bound on d(x, c_j) for every other centre j
+// at the positions before the last update (no drift subtracted).  At the
+// next refit the 256 centres that moved most (and the new seeds) form a set
+// N handled through the centres: d(x, c_j) >= d(c_a, c_j) - u; every other
+// centre moved at most delta_rest, so d(x, c_j) >= l - delta_rest.  A seed
+// starts at a single key and moves far in its first update, so it must not
+// enter the global drift bound.
+//
 // Steps (all on the stream given):
-//   init     centres = previous refit centres ++ seed keys (float64)
-//   seed_lb  for each previous centre a: min over seeds of ||c_a - s||
-//   test     Hamerly test for keys with bounds; failures and new keys are
-//            queued for a full scan
-//   scan     fp32 distances to all centres (tiled SIMT), best and second
-//   recheck  float64 argmin for keys whose best two are within the margin
+//   init      centres = previous refit centres ++ seed keys (float64)
+//   far set   the 256 largest previous drifts -> N, delta_rest
+//   near far  for each previous centre a: min over N \ {a} of ||c_a - c_j||
+//   test      bound test for keys with bounds (tightening u once); failures
+//             and new keys are queued for a full scan
+//   scan      fp32 distances to all centres (tiled SIMT), best and second
+//   recheck   float64 argmin for keys whose best two are within the margin
 //   count / tile counts / scan / scatter: CSR by cluster, members in
-//            ascending key id (deterministic, no float atomics)
-//   update   float64 member means in CSR order, drift, bf16 representatives
-//   bounds   u += drift(own), l -= max drift
+//             ascending key id (deterministic, no float atomics)
+//   update    float64 member means in CSR order, drift, bf16 representatives
+//   bounds    u += drift(own centre)
 #include "common.cuh"
 #include "kernels.h"
 
@@ -47,6 +57,28 @@ __device__ __forceinline__ float kf32(const RefitArgs& a, int64_t s, int i) {
   return v;
 }
 
+// Four consecutive key elements [e, e + 4) as float64 (d % 4 == 0).
+__device__ __forceinline__ void load4_f64(const RefitArgs& a, int64_t row, int e, double* x) {
+  if (a.key_dtype == KD_BF16) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.keys) + row * a.d + e));
+    x[0] = __uint_as_float(v.x << 16);
+    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(v.y << 16);
+    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  } else if (a.key_dtype == KD_FP8) {
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(a.keys) + row * a.d + e));
+    const double sc = static_cast<double>(__ldg(a.key_scale + row));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = static_cast<double>(fp8_to_f32(static_cast<uint8_t>(v >> (8 * u)))) * sc;
+  } else {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.keys) + row * a.d + e));
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
+  }
+}
+
 __global__ void k_init(RefitArgs a) {
   const int64_t n = static_cast<int64_t>(a.K) * a.d;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
@@ -59,45 +91,119 @@ __global__ void k_init(RefitArgs a) {
   }
 }
 
-// one warp per previous centre
-__global__ void k_seed_lb(RefitArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= a.K_prev) return;
-  const int ns = a.K - a.K_prev;
-  double best = 1e300;
-  for (int sidx = 0; sidx < ns; ++sidx) {
-    double acc = 0.0;
-    for (int i = lane; i < a.d; i += 32) {
-      const double df = a.cent[static_cast<int64_t>(warp) * a.d + i] -
-                        a.cent[static_cast<int64_t>(a.K_prev + sidx) * a.d + i];
-      acc = fma(df, df, acc);
+constexpr int kFar = 256;  // previous centres treated through the centres
+
+// Single block: the kFar largest previous drifts (radix select on the bits
+// of the non-negative doubles) -> far flags and the list N = far centres ++
+// new seeds in nlist; delta_rest (largest drift outside N) -> *rest_bits.
+__global__ void __launch_bounds__(1024) k_far_set(RefitArgs a, int32_t* flags, int32_t* nlist,
+                                                  int32_t* n_list, unsigned long long* rest_bits) {
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_need, s_cnt;
+  const int K = a.K_prev;
+  unsigned long long prefix = 0, mask = 0;
+  int need = kFar;
+  if (threadIdx.x == 0) s_cnt = 0;
+  if (K > kFar) {
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      for (int j = threadIdx.x; j < K; j += blockDim.x) {
+        const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(a.drift[j]));
+        if ((b & mask) == prefix) atomicAdd(&hist[(b >> shift) & 255ull], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int cum = 0, dg = 0;
+        for (int d = 255; d >= 0; --d) {
+          const int h = static_cast<int>(hist[d]);
+          if (cum < need && need <= cum + h) {
+            dg = d;
+            break;
+          }
+          cum += h;
+        }
+        s_need = need - cum;
+        s_prefix = prefix | (static_cast<unsigned long long>(dg) << shift);
+      }
+      __syncthreads();
+      need = s_need;
+      prefix = s_prefix;
+      mask |= 255ull << shift;
+      __syncthreads();
     }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    best = fmin(best, acc);
   }
-  if (lane == 0) a.seed_lb[warp] = __double2float_rd(sqrt(best) * (1.0 - 1e-6));
+  // theta = the kFar-th largest drift; far = drift > theta (fewer than kFar)
+  const unsigned long long theta = K > kFar ? prefix : 0ull;
+  for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(a.drift[j]));
+    const bool far = K <= kFar || b > theta;
+    flags[j] = far ? 1 : 0;
+    if (far) nlist[atomicAdd(&s_cnt, 1)] = j;
+  }
+  __syncthreads();
+  for (int j = a.K_prev + threadIdx.x; j < a.K; j += blockDim.x) nlist[atomicAdd(&s_cnt, 1)] = j;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *n_list = s_cnt;
+    *rest_bits = theta;  // largest drift of a centre outside N (0 if none)
+  }
 }
 
-// Hamerly test.  One thread per key in [S, n_r).
-__global__ void k_test(RefitArgs a) {
+// One warp per previous centre a: nb(a) = min over N \ {a} of ||c_a - c_j||
+// (fp32 with a relative margin, rounded down: a lower bound).
+__global__ void k_near_far(RefitArgs a, const int32_t* nlist, const int32_t* n_list) {
+  const int ca = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (ca >= a.K_prev) return;
+  const int nn = *n_list;
+  float best = INFINITY;
+  for (int q = 0; q < nn; ++q) {
+    const int j = nlist[q];
+    if (j == ca) continue;
+    float acc = 0.f;
+    for (int i = lane; i < a.d; i += 32) {
+      const float df = a.cent32[static_cast<int64_t>(ca) * a.d + i] - a.cent32[static_cast<int64_t>(j) * a.d + i];
+      acc = fmaf(df, df, acc);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    best = fminf(best, acc);
+  }
+  if (lane == 0) a.seed_lb[ca] = isinf(best) ? INFINITY : fmaxf(0.f, __fsub_rd(__fmul_rd(sqrtf(best), 1.f - 1e-4f), 1e-6f));
+}
+
+// Exact-ish d(x, c) in fp32 (8-element vector loads), rounded up with a margin.
+__device__ __forceinline__ float dist_up(const RefitArgs& a, int64_t x, int c) {
+  float acc = 0.f;
+  for (int e = 0; e < a.d; e += 4) {
+    double v[4];
+    load4_f64(a, x, e, v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float df = static_cast<float>(v[u]) - a.cent32[static_cast<int64_t>(c) * a.d + e + u];
+      acc = fmaf(df, df, acc);
+    }
+  }
+  return __fadd_ru(__fmul_ru(sqrtf(acc), 1.f + 1e-4f), 1e-6f);
+}
+
+// Bound test.  One thread per key in [S, n_r).
+__global__ void k_test(RefitArgs a, const unsigned long long* rest_bits) {
   const int64_t x = a.S + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (x >= a.n_r) return;
   bool scan = true;
   if (x < a.n_old && a.K_prev > 0) {
     const int ca = a.assign[x];
+    const float rest = __double2float_ru(__longlong_as_double(static_cast<long long>(*rest_bits)));
     float u = a.ub[x];
-    float l = a.lb[x];
-    if (a.K > a.K_prev) l = fminf(l, __fsub_rd(a.seed_lb[ca], u));
+    const float lfar = a.seed_lb[ca];
+    float l = fminf(__fsub_rd(a.lb[x], rest), __fsub_rd(lfar, u));
     if (u < l) {
       scan = false;
+      a.lb[x] = l;
     } else {
-      // tighten u to the exact distance and retest
-      double acc = 0.0;
-      for (int i = 0; i < a.d; ++i) {
-        const double df = kf64(a, x, i) - a.cent[static_cast<int64_t>(ca) * a.d + i];
-        acc = fma(df, df, acc);
-      }
-      u = __double2float_ru(sqrt(acc) * (1.0 + 1e-6));
+      u = dist_up(a, x, ca);  // tighten u once and retest
+      l = fminf(__fsub_rd(a.lb[x], rest), __fsub_rd(lfar, u));
       if (u < l) {
         scan = false;
         a.ub[x] = u;
@@ -384,28 +490,6 @@ __global__ void k_scatter(RefitArgs a) {
   }
 }
 
-// Four consecutive key elements [e, e + 4) as float64 (d % 4 == 0).
-__device__ __forceinline__ void load4_f64(const RefitArgs& a, int64_t row, int e, double* x) {
-  if (a.key_dtype == KD_BF16) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.keys) + row * a.d + e));
-    x[0] = __uint_as_float(v.x << 16);
-    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    x[2] = __uint_as_float(v.y << 16);
-    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-  } else if (a.key_dtype == KD_FP8) {
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(a.keys) + row * a.d + e));
-    const double sc = static_cast<double>(__ldg(a.key_scale + row));
-#pragma unroll
-    for (int u = 0; u < 4; ++u) x[u] = static_cast<double>(fp8_to_f32(static_cast<uint8_t>(v >> (8 * u)))) * sc;
-  } else {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.keys) + row * a.d + e));
-    x[0] = v.x;
-    x[1] = v.y;
-    x[2] = v.z;
-    x[3] = v.w;
-  }
-}
-
 // One warp per cluster: float64 member sums in member (CSR) order, lanes
 // over 4-element column blocks, member ids fetched 32 at a time and four
 // member rows in flight; then mean, drift and the bf16 representative.
@@ -465,13 +549,10 @@ __global__ void k_update(RefitArgs a, unsigned long long* max_drift_bits) {
   }
 }
 
-__global__ void k_bounds(RefitArgs a, const unsigned long long* max_drift_bits) {
+__global__ void k_bounds(RefitArgs a) {
   const int64_t x = a.S + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (x >= a.n_r) return;
-  const double md = __longlong_as_double(static_cast<long long>(*max_drift_bits));
-  const int c = a.assign[x];
-  a.ub[x] = __fadd_ru(a.ub[x], __double2float_ru(a.drift[c]));
-  a.lb[x] = __fsub_rd(a.lb[x], __double2float_ru(md));
+  a.ub[x] = __fadd_ru(a.ub[x], __double2float_ru(a.drift[a.assign[x]]));
 }
 
 }  // namespace
@@ -485,20 +566,27 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   const int64_t ntiles = (n + kTileKeys - 1) / kTileKeys;
   if (ntiles > max_tiles) return cudaErrorInvalidValue;
   if (static_cast<size_t>(a.K) * 4 > 200 * 1024 || a.d > 128 || a.d % 4 != 0) return cudaErrorInvalidValue;
-  // scratch words after n_scan: [1] n_recheck, [2..3] max drift bits
+  // scratch words after n_scan: [1] n_recheck, [2..3] max drift bits,
+  // [4..5] drift bound of the centres outside N, [6] size of N
   int32_t* n_recheck = a.n_scan + 1;
   unsigned long long* mdb = reinterpret_cast<unsigned long long*>(a.n_scan + 2);
-  cudaMemsetAsync(a.n_scan, 0, 16, st);
+  unsigned long long* rest_bits = reinterpret_cast<unsigned long long*>(a.n_scan + 4);
+  int32_t* n_list = a.n_scan + 6;
+  cudaMemsetAsync(a.n_scan, 0, 32, st);
   const int64_t ce = static_cast<int64_t>(a.K) * a.d;
   count_launch();
   k_init<<<static_cast<unsigned>((ce + 255) / 256 < 4096 ? (ce + 255) / 256 : 4096), 256, 0, st>>>(a);
-  if (a.K_prev > 0 && a.K > a.K_prev) {
+  if (a.K_prev > 0) {
+    // far set and centre-to-far-centre bounds (counts and tile_counts are
+    // free until the CSR build below)
     count_launch();
-    k_seed_lb<<<(a.K_prev * 32 + 255) / 256, 256, 0, st>>>(a);
+    k_far_set<<<1, 1024, 0, st>>>(a, a.counts, a.tile_counts, n_list, rest_bits);
+    count_launch();
+    k_near_far<<<(a.K_prev * 32 + 255) / 256, 256, 0, st>>>(a, a.tile_counts, n_list);
   }
   const unsigned gk = static_cast<unsigned>((n + 255) / 256);
   count_launch();
-  k_test<<<gk, 256, 0, st>>>(a);
+  k_test<<<gk, 256, 0, st>>>(a, rest_bits);
   // the scan list length is only known on the device: fixed grids that stride
   const int64_t sblocks = (n + kSK - 1) / kSK;
   count_launch();
@@ -524,7 +612,7 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   count_launch();
   k_update<<<static_cast<unsigned>((static_cast<int64_t>(a.K) * 32 + 255) / 256), 256, 0, st>>>(a, mdb);
   count_launch();
-  k_bounds<<<gk, 256, 0, st>>>(a, mdb);
+  k_bounds<<<gk, 256, 0, st>>>(a);
   if (host_nscan) cudaMemcpyAsync(host_nscan, a.n_scan, 8, cudaMemcpyDeviceToHost, st);
   return cudaGetLastError();
 }

@@ -103,6 +103,49 @@ def test_synchronous_refit_matches_oracle():
     _run_prefill(wl, sample=16, async_refit=False, check_exhaustive=False)
 
 
+def test_many_refits_bounds_stay_exact():
+    """Sixteen refits over a growing prefix: every refit's CSR must equal the
+    oracle's brute-force Lloyd step, so a bound that prunes a key wrongly
+    shows up as a differing assignment."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=8192, T=512, window=128, clusters_per_window=4,
+                  refit_period=512, budget=1024, k=64, M=256)
+    _run_prefill(wl, sample=4, check_exhaustive=False)
+
+
+def test_rollback_replay_matches_a_fresh_index():
+    """Replaying chunks after rollback (bounds and drifts restored) gives the
+    same index as processing them once on a fresh handle."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=12288, T=2048, refit_period=4096,
+                  budget=2048, k=128, M=128)
+    a, _ = P.make_pair(wl)
+    b, _ = P.make_pair(wl)
+    data = [P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)[:2] for c in range(wl.n_chunks)]
+    for c in range(3):
+        for g in (a, b):
+            g.append_keys(*data[c])
+            g.seal()
+    a.publish()
+    a.checkpoint()
+    for rep in range(2):          # two replays with a refit inside
+        for c in range(3, wl.n_chunks):
+            a.append_keys(*data[c])
+            a.seal()
+        a.publish()
+        a.sync()
+        if rep == 0:
+            a.rollback()
+    for c in range(3, wl.n_chunks):
+        b.append_keys(*data[c])
+        b.seal()
+    b.publish()
+    b.sync()
+    ea, eb = a.export_index(), b.export_index()
+    for key in ("offsets", "members", "reps_bf16", "version_nc", "version_nv"):
+        assert np.array_equal(ea[key], eb[key]), key
+    a.close()
+    b.close()
+
+
 def test_encoder_correction_random_and_zero():
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k_encoder"], L=8192, T=2048, refit_period=4096,
                   budget=2048, k=128, M=128)
