@@ -72,6 +72,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   *abort = 1;
   return false;
 }
+// Bounded wait used on the way out after an abort, for asynchronous work
+// this thread issued (TMA copies, UMMAs) that may still be in flight.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return;
+}
 
 // ------------------------------------------------------------------ proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -191,6 +191,9 @@ struct ai_index {
   int64_t max_tiles = 0;
   int32_t* scan_list = nullptr;
   int32_t* scan_words = nullptr;
+  uint16_t* cent_hi = nullptr;  // tensor-core refit scan (bf16 keys, d = 128)
+  uint16_t* cent_lo = nullptr;
+  float* cent_cc = nullptr;
   int64_t* seeds_dev = nullptr;
   int64_t* seeds_host = nullptr;   // pinned
   int32_t* nscan_host = nullptr;   // pinned [2]
@@ -415,9 +418,21 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
   ra.tile_counts = h->tile_counts;
   ra.scan_list = h->scan_list;
   ra.n_scan = h->scan_words;
+  ra.cent_hi = h->cent_hi;
+  ra.cent_lo = h->cent_lo;
+  ra.cent_cc = h->cent_cc;
   ra.err = h->err_dev;
+  RefitTcMaps tcm{};
+  const bool tc = h->cent_hi != nullptr;
+  if (tc) {
+    const int64_t K_pad = round_up(K, 128);
+    if (!make_map(&tcm.keys, h->keys, n_r, 1) || !make_map(&tcm.hi, h->cent_hi, K_pad, 128) ||
+        !make_map(&tcm.lo, h->cent_lo, K_pad, 128))
+      return fail(AI_ERR_CUDA, "tensor map encoding failed (refit)");
+    tcm.num_sms = h->num_sms;
+  }
   const int pr = prof_begin(h, AI_PHASE_REFIT, st);
-  CK(launch_refit(ra, h->max_tiles, st, h->nscan_host));
+  CK(launch_refit(ra, h->max_tiles, st, h->nscan_host, tc ? &tcm : nullptr));
   if (h->enc_wts) {
     EncoderArgs ea{};
     ea.keys = h->keys;
@@ -636,7 +651,12 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   h->max_tiles = (N + refit_tile_size() - 1) / refit_tile_size();
   CKC(dalloc(&h->tile_counts, static_cast<size_t>(h->max_tiles) * h->maxC));
   CKC(dalloc(&h->scan_list, 2 * static_cast<size_t>(N)));
-  CKC(dalloc(&h->scan_words, 8));
+  CKC(dalloc(&h->scan_words, 16));
+  if (c.key_dtype == AI_BF16 && d == 128) {
+    CKC(dalloc(&h->cent_hi, static_cast<size_t>(h->maxC_pad) * 128));
+    CKC(dalloc(&h->cent_lo, static_cast<size_t>(h->maxC_pad) * 128));
+    CKC(dalloc(&h->cent_cc, h->maxC_pad));
+  }
   CKC(dalloc(&h->seeds_dev, h->max_seeds));
   CKC(cudaMallocHost(&h->seeds_host, h->max_seeds * sizeof(int64_t)));
   CKC(cudaMallocHost(&h->nscan_host, 2 * sizeof(int32_t)));
@@ -676,6 +696,9 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->lb);
   cudaFree(h->cent_old);
   cudaFree(h->cent32);
+  cudaFree(h->cent_hi);
+  cudaFree(h->cent_lo);
+  cudaFree(h->cent_cc);
   cudaFree(h->drift);
   cudaFree(h->seed_lb);
   cudaFree(h->counts);

@@ -132,11 +132,21 @@ struct RefitArgs {
   float* seed_lb;        // [K_prev] min distance from old centre to any seed
   int32_t* tile_counts;  // scratch [ntiles * K]
   int32_t* scan_list;    // scratch [n_r - S] keys needing a full scan
-  int32_t* n_scan;       // scratch [1]
+  int32_t* n_scan;       // scratch [16]
+  uint16_t* cent_hi;     // [K_pad, 128] bf16 high parts (tensor-core scan only)
+  uint16_t* cent_lo;     // [K_pad, 128] bf16 residuals
+  float* cent_cc;        // [K_pad] ||c||^2 (+inf for padding rows)
   int* err;
 };
+// Tensor maps for the tensor-core full scan (bf16 keys, d = 128): keys with a
+// one-row box (gather4), centre hi / lo parts with 128-row boxes.
+struct RefitTcMaps {
+  CUtensorMap keys, hi, lo;
+  int num_sms;
+};
 cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
-                         int32_t* host_nscan /*nullable: read back count*/);
+                         int32_t* host_nscan /*nullable: read back count*/,
+                         const RefitTcMaps* tc /*nullable: fp32 SIMT scan*/);
 int64_t refit_tile_size();
 
 // --------------------------------------------------------------- encoder

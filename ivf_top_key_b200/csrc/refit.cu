@@ -555,24 +555,282 @@ __global__ void k_bounds(RefitArgs a) {
   a.ub[x] = __fadd_ru(a.ub[x], __double2float_ru(a.drift[a.assign[x]]));
 }
 
+// ------------------------------------------------- tensor-core full scan
+// bf16 keys, d = 128.  Each fp64 centre c is split into bf16 hi + lo
+// (hi = rne(c), lo = rne(c - hi); per element |c - hi - lo| <= 2^-16 |c|),
+// and one UMMA pair per 128-centre tile accumulates x.hi + x.lo in fp32
+// TMEM.  d^2 = ||x||^2 - 2 x.c + ||c||^2 then carries, per key, at most
+//   1.5e-5 (split residual) + 3.1e-5 (256-term fp32 accumulation, counted
+//   with whole-ulp steps) + 0.8e-5 (||x||^2 in fp32) + rounding of the sum
+// times (||x||^2 + max ||c||^2); the kernel takes 1e-4 times that as its
+// bound err.  Keys whose best two lie within 2 err of each other are
+// re-decided in float64, so the assignment equals the exact one.
+constexpr int kTcKeys = 128, kTcCent = 128;
+constexpr int kTcBStages = 2;
+constexpr int kTcA = kTcKeys * 256;            // 32 KiB per key tile
+constexpr int kTcB = 2 * kTcCent * 256;        // hi + lo, 64 KiB per centre tile
+constexpr int kTcThreads = 256;
+constexpr size_t kTcSmem = 1024 + 2 * kTcA + kTcBStages * kTcB;
+constexpr double kTcErr = 1e-4;
+
+__global__ void k_cent_split(RefitArgs a, unsigned long long* ccmax_bits) {
+  const int j = blockIdx.x, i = threadIdx.x;  // 128 threads per centre
+  const bool live = j < a.K;
+  const double c = live ? a.cent[static_cast<int64_t>(j) * 128 + i] : 0.0;
+  const uint16_t hb = f64_to_bf16_rne(c);
+  const uint16_t lb = f64_to_bf16_rne(c - static_cast<double>(bf16_bits_to_f32(hb)));
+  a.cent_hi[static_cast<int64_t>(j) * 128 + i] = hb;
+  a.cent_lo[static_cast<int64_t>(j) * 128 + i] = lb;
+  __shared__ double red[4];
+  double sq = c * c;
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if ((i & 31) == 0) red[i >> 5] = sq;
+  __syncthreads();
+  if (i == 0) {
+    const double t = (red[0] + red[1]) + (red[2] + red[3]);
+    a.cent_cc[j] = live ? static_cast<float>(t) : INFINITY;
+    if (live) atomicMax(ccmax_bits, static_cast<unsigned long long>(__double_as_longlong(t)));
+  }
+}
+
+// Warp roles: 0 = centre-tile producer (TMA, lane 0), 1 = UMMA issuer
+// (lane 0), 2-3 = key-tile producers (TMA gather4 of the listed keys, 64
+// rows each), 4-7 = epilogue (one key row per thread).  Key tiles are
+// double-buffered; centre tiles stream through kTcBStages stages; two TMEM
+// accumulators of 128 columns alternate between UMMA and epilogue.
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_scan_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap hmap,
+              const __grid_constant__ CUtensorMap lmap, RefitArgs a, int K_pad,
+              const unsigned long long* ccmax_bits, int32_t* recheck, int32_t* n_recheck) {
+  extern __shared__ uint8_t raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = base;             // [2][kTcA]
+  uint8_t* sb = base + 2 * kTcA;  // [kTcBStages][kTcB]
+  __shared__ uint64_t afull[2], aempty[2], bfull[kTcBStages], bempty[kTcBStages], tfull[2], tempty[2], done;
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_flag;
+  volatile int* aborted = &abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = *a.n_scan;
+  const int ntiles = (n + kTcKeys - 1) / kTcKeys;
+  const int nct = K_pad / kTcCent;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&afull[b], 2);
+      mbar_init(&aempty[b], 1 + 128);
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    for (int s2 = 0; s2 < kTcBStages; ++s2) {
+      mbar_init(&bfull[s2], 1);
+      mbar_init(&bempty[s2], 1);
+    }
+    mbar_init(&done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_holder, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------- centre-tile producer
+    if (lane == 0) {
+      uint32_t gj = 0;
+      for (int kt = blockIdx.x; kt < ntiles && !*aborted; kt += gridDim.x) {
+        for (int ct = 0; ct < nct; ++ct, ++gj) {
+          const int s2 = gj % kTcBStages;
+          if (gj >= kTcBStages && !mbar_wait(&bempty[s2], ((gj / kTcBStages) & 1) ^ 1, a.err, &abort_flag))
+            break;
+          uint8_t* dst = sb + s2 * kTcB;
+          mbar_arrive_expect_tx(&bfull[s2], kTcB);
+          tma_load_2d(dst, &hmap, 0, ct * kTcCent, &bfull[s2]);
+          tma_load_2d(dst + kTcCent * 128, &hmap, 64, ct * kTcCent, &bfull[s2]);
+          tma_load_2d(dst + 2 * kTcCent * 128, &lmap, 0, ct * kTcCent, &bfull[s2]);
+          tma_load_2d(dst + 3 * kTcCent * 128, &lmap, 64, ct * kTcCent, &bfull[s2]);
+        }
+      }
+      if (*aborted)  // let the last copies land before the CTA exits
+        for (uint32_t g = gj > kTcBStages ? gj - kTcBStages : 0; g < gj; ++g)
+          mbar_drain(&bfull[g % kTcBStages], (g / kTcBStages) & 1);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------- key-tile producers
+    uint32_t it = 0;
+    for (int kt = blockIdx.x; kt < ntiles; kt += gridDim.x, ++it) {
+      const int b = it & 1;
+      if (it >= 2 && !mbar_wait(&aempty[b], ((it >> 1) & 1) ^ 1, a.err, &abort_flag)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&afull[b], kTcA / 2);
+      __syncwarp();
+      const int rl = (warp - 2) * 64 + (lane & 15) * 4;  // first of this lane's 4 rows
+      const int half = lane >> 4;
+      int r[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = kt * kTcKeys + rl + q;
+        r[q] = kk < n ? a.scan_list[kk] : static_cast<int>(a.S);
+      }
+      tma_gather4(sa + b * kTcA + half * (kTcKeys * 128) + rl * 128, &kmap, half * 64, r[0], r[1], r[2], r[3],
+                  &afull[b]);
+    }
+    if (*aborted)
+      for (uint32_t g = it > 2 ? it - 2 : 0; g < it; ++g) mbar_drain(&afull[g & 1], (g >> 1) & 1);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTcKeys, kTcCent);
+      uint32_t it = 0, gj = 0;
+      bool ok = true;
+      for (int kt = blockIdx.x; ok && kt < ntiles; kt += gridDim.x, ++it) {
+        const int b = it & 1;
+        if (!mbar_wait(&afull[b], (it >> 1) & 1, a.err, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sA = smem_u32(sa + b * kTcA);
+        for (int ct = 0; ct < nct; ++ct, ++gj) {
+          const int s2 = gj % kTcBStages;
+          const int acc = gj & 1;
+          if (!mbar_wait(&bfull[s2], (gj / kTcBStages) & 1, a.err, &abort_flag) ||
+              (gj >= 2 && !mbar_wait(&tempty[acc], ((gj >> 1) & 1) ^ 1, a.err, &abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sB = smem_u32(sb + s2 * kTcB);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {  // x.hi, then x.lo into the same accumulator
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
+              umma_bf16(tmem_base + acc * kTcCent, sdesc_sw128(sA + kb * (kTcKeys * 128) + ko),
+                        sdesc_sw128(sB + part * (2 * kTcCent * 128) + kb * (kTcCent * 128) + ko), idesc,
+                        (part > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&bempty[s2]);
+          umma_commit(&tfull[acc]);
+        }
+        if (ok) umma_commit(&aempty[b]);  // the key tile is free once these UMMAs finish
+      }
+      umma_commit(&done);  // every UMMA issued above has finished before TMEM is freed
+      mbar_drain(&done, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int row = (warp - 4) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const double ccmax = __longlong_as_double(static_cast<long long>(*ccmax_bits));
+    uint32_t it = 0, gj = 0;
+    bool ok = true;
+    for (int kt = blockIdx.x; ok && kt < ntiles; kt += gridDim.x, ++it) {
+      const int b = it & 1;
+      float xx = 0.f;
+      if (!mbar_wait(&afull[b], (it >> 1) & 1, a.err, &abort_flag)) break;
+      {
+        // ||x||^2 from the staged row (128-byte swizzle: 16-byte chunk c of
+        // row r sits at chunk c ^ (r & 7))
+        const uint8_t* rowp = sa + b * kTcA + row * 128;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + (c >> 3) * (kTcKeys * 128) +
+                                                          (((c & 7) ^ (row & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xFFFF0000u);
+            xx = fmaf(lo, lo, xx);
+            xx = fmaf(hi, hi, xx);
+          }
+        }
+      }
+      mbar_arrive(&aempty[b]);
+      const float err = static_cast<float>(kTcErr * (static_cast<double>(xx) + ccmax));
+      float best = INFINITY, second = INFINITY;
+      int bid = 0x7fffffff;
+      for (int ct = 0; ct < nct; ++ct, ++gj) {
+        const int acc = gj & 1;
+        if (!mbar_wait(&tfull[acc], (gj >> 1) & 1, a.err, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c32 = 0; c32 < kTcCent / 32; ++c32) {
+          float v[32];
+          tmem_ld32(tmem_base + acc * kTcCent + c32 * 32 + lane_off, v);
+          const float4* ccp = reinterpret_cast<const float4*>(a.cent_cc + ct * kTcCent + c32 * 32);
+          float cc[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 t = __ldg(ccp + q);
+            cc[4 * q] = t.x;
+            cc[4 * q + 1] = t.y;
+            cc[4 * q + 2] = t.z;
+            cc[4 * q + 3] = t.w;
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
+            if (d2 < best) {
+              second = best;
+              best = d2;
+              bid = ct * kTcCent + c32 * 32 + q;
+            } else if (d2 < second) {
+              second = d2;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+      }
+      if (!ok) break;
+      const int kk = kt * kTcKeys + row;
+      if (kk < n && bid < a.K) {
+        const int32_t x = a.scan_list[kk];
+        a.assign[x] = bid;
+        if (!(second - best > 2.f * err)) {
+          const int p = atomicAdd(n_recheck, 1);
+          recheck[p] = x;
+        }
+        a.ub[x] = __fmul_ru(sqrtf(__fadd_ru(fmaxf(best, 0.f), err)), 1.f + 1e-6f);
+        a.lb[x] = __fmul_rd(sqrtf(fmaxf(__fsub_rd(second, err), 0.f)), 1.f - 1e-6f);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
 }  // namespace
 
 int64_t refit_tile_size() { return kTileKeys; }
 
 cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
-                         int32_t* host_nscan) {
+                         int32_t* host_nscan, const RefitTcMaps* tc) {
   const int64_t n = a.n_r - a.S;
   if (n <= 0 || a.K <= 0) return cudaSuccess;
   const int64_t ntiles = (n + kTileKeys - 1) / kTileKeys;
   if (ntiles > max_tiles) return cudaErrorInvalidValue;
   if (static_cast<size_t>(a.K) * 4 > 200 * 1024 || a.d > 128 || a.d % 4 != 0) return cudaErrorInvalidValue;
   // scratch words after n_scan: [1] n_recheck, [2..3] max drift bits,
-  // [4..5] drift bound of the centres outside N, [6] size of N
+  // [4..5] drift bound of the centres outside N, [6] size of N, [8..9]
+  // largest ||c||^2 (tensor-core scan)
   int32_t* n_recheck = a.n_scan + 1;
   unsigned long long* mdb = reinterpret_cast<unsigned long long*>(a.n_scan + 2);
   unsigned long long* rest_bits = reinterpret_cast<unsigned long long*>(a.n_scan + 4);
   int32_t* n_list = a.n_scan + 6;
-  cudaMemsetAsync(a.n_scan, 0, 32, st);
+  unsigned long long* ccmax_bits = reinterpret_cast<unsigned long long*>(a.n_scan + 8);
+  if (tc && (a.key_dtype != KD_BF16 || a.d != 128)) return cudaErrorInvalidValue;
+  cudaMemsetAsync(a.n_scan, 0, 40, st);
   const int64_t ce = static_cast<int64_t>(a.K) * a.d;
   count_launch();
   k_init<<<static_cast<unsigned>((ce + 255) / 256 < 4096 ? (ce + 255) / 256 : 4096), 256, 0, st>>>(a);
@@ -588,9 +846,22 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   count_launch();
   k_test<<<gk, 256, 0, st>>>(a, rest_bits);
   // the scan list length is only known on the device: fixed grids that stride
-  const int64_t sblocks = (n + kSK - 1) / kSK;
-  count_launch();
-  k_scan<<<static_cast<unsigned>(sblocks < 1184 ? sblocks : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
+  if (tc) {
+    const int K_pad = (a.K + kTcCent - 1) / kTcCent * kTcCent;
+    count_launch();
+    k_cent_split<<<K_pad, 128, 0, st>>>(a, ccmax_bits);
+    cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTcSmem));
+    const int64_t ktiles = (n + kTcKeys - 1) / kTcKeys;
+    const int grid = static_cast<int>(ktiles < tc->num_sms ? ktiles : tc->num_sms);
+    count_launch();
+    k_scan_tc<<<grid, kTcThreads, kTcSmem, st>>>(tc->keys, tc->hi, tc->lo, a, K_pad, ccmax_bits,
+                                                  a.scan_list + n, n_recheck);
+  } else {
+    const int64_t sblocks = (n + kSK - 1) / kSK;
+    count_launch();
+    k_scan<<<static_cast<unsigned>(sblocks < 1184 ? sblocks : 1184), 256, 0, st>>>(a, a.scan_list + n,
+                                                                                    n_recheck);
+  }
   // recheck list lives after the scan list (capacity n)
   count_launch();
   k_recheck<<<static_cast<unsigned>(n < 1184 ? n : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);

@@ -21,7 +21,8 @@ if not torch.cuda.is_available():  # pragma: no cover
 def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_refit=True,
                  seed_q=0):
     """Chunked prefill on both sides; compare index state after every chunk
-    and route+refine / exhaustive results on (sampled) queries."""
+    and route+refine / exhaustive results on (sampled) queries.
+    check_exhaustive: True, False, or the set of chunk indices to check."""
     gpu, orc = P.make_pair(wl, encoder=encoder, async_refit=async_refit)
     rng = np.random.default_rng(1234 + seed_q)
     stats = collections.Counter()
@@ -47,7 +48,7 @@ def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_
         cnd = cand.cpu().numpy()[idx]
         P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], ids, scs, cnd, wl.k,
                         wl.budget, stats)
-        if check_exhaustive:
+        if check_exhaustive is True or (check_exhaustive and c in check_exhaustive):
             eo = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
             es = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
             gpu.select_exhaustive(qd, wd, p0, wl.k, out=eo, out_scores=es)
