@@ -476,7 +476,8 @@ def measure_refit_overlap(idx, chunks, wl, out, stream, reps=3):
     return {"t_refit_ms": t_refit, "t_route_ms": t_route, "t_both_ms": t_both,
             "hidden_fraction": (t_refit + t_route - t_both) / t_refit if t_refit > 0 else None,
             "keys": st["n_keys"], "clusters_after": st["n_clusters"],
-            "keys_fully_scanned": st["last_refit_scanned"]}
+            "keys_fully_scanned": st["last_refit_scanned"],
+            "keys_rechecked_f64": st["last_refit_rechecked"]}
 
 
 # --------------------------------------------------------- oracle arm --

@@ -149,6 +149,7 @@ typedef struct ai_stats {
   int64_t refit_pending; /* 1 if a refit awaits publication                 */
   int64_t base_watermark;/* n_r of the published base (0 = none)            */
   int64_t last_refit_scanned; /* keys fully scanned by the last finished refit */
+  int64_t last_refit_rechecked; /* of those, keys re-decided in float64 (near ties) */
 } ai_stats;
 int ai_get_stats(ai_handle h, ai_stats* out);
 

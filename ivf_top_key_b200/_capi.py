@@ -51,7 +51,7 @@ class AiConfig(ctypes.Structure):
 class AiStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "n_keys", "n_sealed", "n_clusters", "n_versions", "n_refits", "refit_pending",
-        "base_watermark", "last_refit_scanned")]
+        "base_watermark", "last_refit_scanned", "last_refit_rechecked")]
 
 
 class AiError(RuntimeError):

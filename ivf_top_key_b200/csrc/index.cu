@@ -194,6 +194,12 @@ struct ai_index {
   uint16_t* cent_hi = nullptr;  // tensor-core refit scan (bf16 keys, d = 128)
   uint16_t* cent_lo = nullptr;
   float* cent_cc = nullptr;
+  int32_t* upd_chunk_off = nullptr;  // refit update chunks
+  double* upd_part = nullptr;
+  float* band_best = nullptr;  // near-tie bands of the tensor-core refit scan
+  int32_t* band_ids = nullptr;
+  int32_t* band_cnt = nullptr;
+  int band_cap = 0;
   int64_t* seeds_dev = nullptr;
   int64_t* seeds_host = nullptr;   // pinned
   int32_t* nscan_host = nullptr;   // pinned [2]
@@ -421,6 +427,12 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
   ra.cent_hi = h->cent_hi;
   ra.cent_lo = h->cent_lo;
   ra.cent_cc = h->cent_cc;
+  ra.upd_chunk_off = h->upd_chunk_off;
+  ra.upd_part = h->upd_part;
+  ra.band_best = h->band_best;
+  ra.band_ids = h->band_ids;
+  ra.band_cnt = h->band_cnt;
+  ra.band_cap = h->band_cap;
   ra.err = h->err_dev;
   RefitTcMaps tcm{};
   const bool tc = h->cent_hi != nullptr;
@@ -652,10 +664,16 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   CKC(dalloc(&h->tile_counts, static_cast<size_t>(h->max_tiles) * h->maxC));
   CKC(dalloc(&h->scan_list, 2 * static_cast<size_t>(N)));
   CKC(dalloc(&h->scan_words, 16));
+  CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
+  CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
   if (c.key_dtype == AI_BF16 && d == 128) {
     CKC(dalloc(&h->cent_hi, static_cast<size_t>(h->maxC_pad) * 128));
     CKC(dalloc(&h->cent_lo, static_cast<size_t>(h->maxC_pad) * 128));
     CKC(dalloc(&h->cent_cc, h->maxC_pad));
+    h->band_cap = static_cast<int>(std::max<int64_t>(4096, N / 16));
+    CKC(dalloc(&h->band_best, h->band_cap));
+    CKC(dalloc(&h->band_ids, static_cast<size_t>(h->band_cap) * 16));
+    CKC(dalloc(&h->band_cnt, h->band_cap));
   }
   CKC(dalloc(&h->seeds_dev, h->max_seeds));
   CKC(cudaMallocHost(&h->seeds_host, h->max_seeds * sizeof(int64_t)));
@@ -699,6 +717,11 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->cent_hi);
   cudaFree(h->cent_lo);
   cudaFree(h->cent_cc);
+  cudaFree(h->upd_chunk_off);
+  cudaFree(h->upd_part);
+  cudaFree(h->band_best);
+  cudaFree(h->band_ids);
+  cudaFree(h->band_cnt);
   cudaFree(h->drift);
   cudaFree(h->seed_lb);
   cudaFree(h->counts);
@@ -941,6 +964,7 @@ int ai_get_stats(ai_handle h, ai_stats* out) {
   out->refit_pending = h->pending ? 1 : 0;
   out->base_watermark = b.base_n_r;
   out->last_refit_scanned = h->nscan_host ? h->nscan_host[0] : 0;
+  out->last_refit_rechecked = h->nscan_host ? h->nscan_host[1] : 0;
   return AI_OK;
 }
 

@@ -136,6 +136,12 @@ struct RefitArgs {
   uint16_t* cent_hi;     // [K_pad, 128] bf16 high parts (tensor-core scan only)
   uint16_t* cent_lo;     // [K_pad, 128] bf16 residuals
   float* cent_cc;        // [K_pad] ||c||^2 (+inf for padding rows)
+  int32_t* upd_chunk_off;  // scratch [K + 1] offsets of the update chunks
+  double* upd_part;        // scratch [n / 128 + K, d] chunk sums
+  float* band_best;        // scratch [band_cap] tensor-core scan: flagged keys' best d^2
+  int32_t* band_ids;       // scratch [band_cap, 16] centres within the error band
+  int32_t* band_cnt;       // scratch [band_cap]
+  int band_cap;
   int* err;
 };
 // Tensor maps for the tensor-core full scan (bf16 keys, d = 128): keys with a
@@ -148,6 +154,7 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
                          int32_t* host_nscan /*nullable: read back count*/,
                          const RefitTcMaps* tc /*nullable: fp32 SIMT scan*/);
 int64_t refit_tile_size();
+int64_t refit_update_chunk();  // members per update chunk
 
 // --------------------------------------------------------------- encoder
 struct EncoderArgs {

@@ -320,68 +320,122 @@ __global__ void __launch_bounds__(256) k_scan(RefitArgs a, int32_t* recheck, int
   }
 }
 
-// float64 decision for near ties: one block per key.
+// float64 decision for near ties.  A block takes kRkKeys listed keys (one
+// warp each); centre rows stream through shared memory in tiles of
+// kRkCent, one centre per lane, so each centre is read from L2 once per
+// block with coalesced loads.  Per (key, centre) the sum runs over the
+// dimensions in order with fma, as in the fp32 screen.
+constexpr int kRkKeys = 8, kRkCent = 32;
+constexpr int kBand = 16;  // centres listed per flagged key by the band pass
+// Entries p < cap whose band has at most kBand centres were decided by
+// k_recheck_band; this kernel takes the rest (all of them when cap = 0).
 __global__ void __launch_bounds__(256) k_recheck(RefitArgs a, const int32_t* recheck,
-                                                 const int32_t* n_recheck) {
-  __shared__ double xs[256];
-  __shared__ double rb[8], rs[8];
-  __shared__ int ri[8];
+                                                 const int32_t* n_recheck, const int32_t* band_cnt,
+                                                 int cap) {
+  __shared__ double xs[kRkKeys][kMaxD];
+  __shared__ double cs[kRkCent][kMaxD + 1];
   const int nr = *n_recheck;
-  for (int idx = blockIdx.x; idx < nr; idx += gridDim.x) {
-  const int32_t x = recheck[idx];
-  __syncthreads();
-  for (int i = threadIdx.x; i < a.d; i += blockDim.x) xs[i] = kf64(a, x, i);
-  __syncthreads();
-  double best = INFINITY, second = INFINITY;
-  int bi = 0x7fffffff;
-  for (int c = threadIdx.x; c < a.K; c += blockDim.x) {
-    double acc = 0.0;
-    for (int i = 0; i < a.d; ++i) {
-      const double df = xs[i] - a.cent[static_cast<int64_t>(c) * a.d + i];
-      acc = fma(df, df, acc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto todo = [&](int p) { return p < nr && (p >= cap || band_cnt[p] > kBand); };
+  for (int g0 = blockIdx.x * kRkKeys; g0 < nr; g0 += gridDim.x * kRkKeys) {
+    __syncthreads();
+    if (!__syncthreads_or(threadIdx.x < kRkKeys && todo(g0 + threadIdx.x))) continue;
+    for (int e = threadIdx.x; e < kRkKeys * a.d; e += blockDim.x) {
+      const int r = e / a.d, i = e % a.d;
+      xs[r][i] = g0 + r < nr ? kf64(a, recheck[g0 + r], i) : 0.0;
     }
-    if (acc < best || (acc == best && c < bi)) {
-      second = best;
-      best = acc;
-      bi = c;
-    } else if (acc < second) {
-      second = acc;
-    }
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-    const double os = __shfl_xor_sync(0xffffffffu, second, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ob < best || (ob == best && oi < bi)) {
-      second = fmin(best, os);
-      best = ob;
-      bi = oi;
-    } else {
-      second = fmin(second, ob);
-    }
-  }
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) {
-    rb[w] = best;
-    rs[w] = second;
-    ri[w] = bi;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int j = 1; j < (blockDim.x >> 5); ++j) {
-      if (rb[j] < best || (rb[j] == best && ri[j] < bi)) {
-        second = fmin(best, rs[j]);
-        best = rb[j];
-        bi = ri[j];
-      } else {
-        second = fmin(second, rb[j]);
+    double best = INFINITY, second = INFINITY;
+    int bi = 0x7fffffff;
+    for (int c0 = 0; c0 < a.K; c0 += kRkCent) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < kRkCent * a.d; e += blockDim.x) {
+        const int r = e / a.d, i = e % a.d;
+        cs[r][i] = c0 + r < a.K ? a.cent[static_cast<int64_t>(c0 + r) * a.d + i] : 0.0;
+      }
+      __syncthreads();
+      double acc = 0.0;
+      for (int i = 0; i < a.d; ++i) {
+        const double df = xs[warp][i] - cs[lane][i];
+        acc = fma(df, df, acc);
+      }
+      const int c = c0 + lane;
+      if (c < a.K) {
+        if (acc < best || (acc == best && c < bi)) {
+          second = best;
+          best = acc;
+          bi = c;
+        } else if (acc < second) {
+          second = acc;
+        }
       }
     }
-    a.assign[x] = bi;
-    a.ub[x] = __double2float_ru(sqrt(best) * (1.0 + 1e-6));
-    a.lb[x] = __double2float_rd(sqrt(second) * (1.0 - 1e-6));
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const double os = __shfl_xor_sync(0xffffffffu, second, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob < best || (ob == best && oi < bi)) {
+        second = fmin(best, os);
+        best = ob;
+        bi = oi;
+      } else {
+        second = fmin(second, ob);
+      }
+    }
+    if (lane == 0 && todo(g0 + warp)) {
+      const int32_t x = recheck[g0 + warp];
+      a.assign[x] = bi;
+      a.ub[x] = __double2float_ru(sqrt(best) * (1.0 + 1e-6));
+      a.lb[x] = __double2float_rd(sqrt(second) * (1.0 - 1e-6));
+    }
   }
-  __syncthreads();
+}
+
+// float64 decision among the band of a flagged key: one warp per key, lanes
+// over dimensions.  Centres outside the band are farther than the band's
+// best in exact arithmetic; their lower bound (stored by the band pass)
+// enters the key's lower bound.
+__global__ void k_recheck_band(RefitArgs a, const int32_t* recheck, const int32_t* n_recheck,
+                               const float* outside_lb2, const int32_t* band_ids, const int32_t* band_cnt,
+                               int cap) {
+  const int warp = static_cast<int>((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int nwarps = static_cast<int>((gridDim.x * static_cast<int64_t>(blockDim.x)) >> 5);
+  const int nr = min(*n_recheck, cap);
+  for (int p = warp; p < nr; p += nwarps) {
+    const int nb = band_cnt[p];
+    if (nb > kBand) continue;  // overflow: full decision in k_recheck
+    const int32_t x = recheck[p];
+    double xv[4];
+    const int e = lane * 4;
+    if (e < a.d) load4_f64(a, x, e, xv);
+    double best = INFINITY, second = INFINITY;
+    int bi = 0x7fffffff;
+    for (int u = 0; u < nb; ++u) {
+      const int c = band_ids[static_cast<int64_t>(p) * kBand + u];
+      double acc = 0.0;
+      if (e < a.d) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const double df = xv[q] - a.cent[static_cast<int64_t>(c) * a.d + e + q];
+          acc = fma(df, df, acc);
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (acc < best || (acc == best && c < bi)) {
+        second = best;
+        best = acc;
+        bi = c;
+      } else if (acc < second) {
+        second = acc;
+      }
+    }
+    if (lane == 0 && nb > 0) {
+      const double out2 = static_cast<double>(outside_lb2[p]);
+      const double sec = fmin(second, out2 > 0.0 ? out2 : 0.0);
+      a.assign[x] = bi;
+      a.ub[x] = __double2float_ru(sqrt(best) * (1.0 + 1e-6));
+      a.lb[x] = __double2float_rd(sqrt(sec) * (1.0 - 1e-6));
+    }
   }
 }
 
@@ -402,15 +456,17 @@ __global__ void k_count(RefitArgs a) {
 }
 
 // exclusive scan of counts -> offsets (single block)
-__global__ void __launch_bounds__(1024) k_offsets(RefitArgs a) {
-  __shared__ int warp_sums[32];
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
+// Exclusive prefix sum over j < K of f(counts[j]) into out[0..K] by one
+// 1024-thread block; f = identity (chunk = 0) or ceil(v / chunk).
+__device__ void block_scan_counts(const int32_t* counts, int K, int chunk, int32_t* out, int* warp_sums,
+                                  int* carry) {
+  if (threadIdx.x == 0) *carry = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int base = 0; base < a.K; base += blockDim.x) {
+  for (int base = 0; base < K; base += blockDim.x) {
     const int j = base + threadIdx.x;
-    const int v = j < a.K ? a.counts[j] : 0;
+    int v = j < K ? counts[j] : 0;
+    if (chunk > 0) v = (v + chunk - 1) / chunk;
     int incl = v;
     for (int o = 1; o < 32; o <<= 1) {
       const int n = __shfl_up_sync(0xffffffffu, incl, o);
@@ -428,12 +484,22 @@ __global__ void __launch_bounds__(1024) k_offsets(RefitArgs a) {
       warp_sums[lane] = si - s;
     }
     __syncthreads();
-    if (j < a.K) a.offsets[j] = carry + warp_sums[w] + incl - v;
+    if (j < K) out[j] = *carry + warp_sums[w] + incl - v;
     __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry += warp_sums[w] + incl;
+    if (threadIdx.x == blockDim.x - 1) *carry += warp_sums[w] + incl;
     __syncthreads();
   }
-  if (threadIdx.x == 0) a.offsets[a.K] = carry;
+  if (threadIdx.x == 0) out[K] = *carry;
+  __syncthreads();
+}
+
+// CSR offsets, and the offsets of the update chunks (kUpdChunk members)
+constexpr int kUpdChunk = 128;
+__global__ void __launch_bounds__(1024) k_offsets(RefitArgs a) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  block_scan_counts(a.counts, a.K, 0, a.offsets, warp_sums, &carry);
+  block_scan_counts(a.counts, a.K, kUpdChunk, a.upd_chunk_off, warp_sums, &carry);
 }
 
 // per-tile cluster counts: one warp per tile, keys walked in order
@@ -493,52 +559,85 @@ __global__ void k_scatter(RefitArgs a) {
 // One warp per cluster: float64 member sums in member (CSR) order, lanes
 // over 4-element column blocks, member ids fetched 32 at a time and four
 // member rows in flight; then mean, drift and the bf16 representative.
-__global__ void k_update(RefitArgs a, unsigned long long* max_drift_bits) {
-  const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (j >= a.K) return;
-  const int o0 = a.offsets[j], o1 = a.offsets[j + 1];
-  double dr = 0.0;
-  for (int e0 = 0; e0 < a.d; e0 += 128) {
-    const int e = e0 + lane * 4;
-    const bool act = e < a.d;
-    double sum[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int p0 = o0; p0 < o1; p0 += 32) {
-      const int nb = min(32, o1 - p0);
-      const int myid = lane < nb ? a.members[p0 + lane] : 0;
-      int u = 0;
-      for (; u + 4 <= nb; u += 4) {
-        double x[4][4];
+// Centre update in two deterministic steps.  k_update_part: one warp per
+// chunk of up to kUpdChunk consecutive members of a cluster sums them in
+// member order (lane = 4 dimensions); k_update_fin: one warp per cluster
+// adds its chunk sums in chunk order, divides by the size (an empty cluster
+// keeps its centre) and writes centre, bf16 representative and drift.
+__global__ void k_update_part(RefitArgs a) {
+  const int q = static_cast<int>((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int32_t* co = a.upd_chunk_off;
+  if (q >= co[a.K]) return;
+  int lo = 0, hi = a.K;  // co[lo] <= q < co[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (co[mid] <= q) lo = mid;
+    else hi = mid;
+  }
+  const int p0 = a.offsets[lo] + (q - co[lo]) * kUpdChunk;
+  const int p1 = min(p0 + kUpdChunk, a.offsets[lo + 1]);
+  const int e = lane * 4;
+  const bool act = e < a.d;
+  double sum[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int b0 = p0; b0 < p1; b0 += 32) {
+    const int nb = min(32, p1 - b0);
+    const int myid = lane < nb ? a.members[b0 + lane] : 0;
+    int u = 0;
+    for (; u + 8 <= nb; u += 8) {
+      double x[8][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int id = __shfl_sync(0xffffffffu, myid, u + r);
-          if (act) load4_f64(a, id, e, x[r]);
-        }
+      for (int r = 0; r < 8; ++r) {
+        const int id = __shfl_sync(0xffffffffu, myid, u + r);
+        if (act) load4_f64(a, id, e, x[r]);
+      }
+      if (act) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 8; ++r)
 #pragma unroll
           for (int c = 0; c < 4; ++c) sum[c] += x[r][c];
       }
-      for (; u < nb; ++u) {
-        const int id = __shfl_sync(0xffffffffu, myid, u);
+    }
+    for (; u < nb; ++u) {
+      const int id = __shfl_sync(0xffffffffu, myid, u);
+      if (act) {
         double x[4];
-        if (act) {
-          load4_f64(a, id, e, x);
+        load4_f64(a, id, e, x);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) sum[c] += x[c];
-        }
+        for (int c = 0; c < 4; ++c) sum[c] += x[c];
       }
     }
-    if (act) {
+  }
+  if (act) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int64_t idx = static_cast<int64_t>(j) * a.d + e + c;
-        double v = a.cent[idx];
-        if (o1 > o0) v = sum[c] / static_cast<double>(o1 - o0);
-        const double df = v - a.cent_old[idx];
-        dr = fma(df, df, dr);
-        a.cent[idx] = v;
-        a.reps[idx] = f64_to_bf16_rne(v);
-      }
+    for (int c = 0; c < 4; ++c) a.upd_part[static_cast<int64_t>(q) * a.d + e + c] = sum[c];
+  }
+}
+
+__global__ void k_update_fin(RefitArgs a, unsigned long long* max_drift_bits) {
+  const int j = static_cast<int>((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= a.K) return;
+  const int n = a.offsets[j + 1] - a.offsets[j];
+  const int q0 = a.upd_chunk_off[j], q1 = a.upd_chunk_off[j + 1];
+  const int e = lane * 4;
+  double dr = 0.0;
+  if (e < a.d) {
+    double sum[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int q = q0; q < q1; ++q) {
+      const double* pp = a.upd_part + static_cast<int64_t>(q) * a.d + e;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sum[c] += pp[c];
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t idx = static_cast<int64_t>(j) * a.d + e + c;
+      double v = a.cent[idx];
+      if (n > 0) v = sum[c] / static_cast<double>(n);
+      const double df = v - a.cent_old[idx];
+      dr = fma(df, df, dr);
+      a.cent[idx] = v;
+      a.reps[idx] = f64_to_bf16_rne(v);
     }
   }
   for (int o = 16; o > 0; o >>= 1) dr += __shfl_xor_sync(0xffffffffu, dr, o);
@@ -598,10 +697,26 @@ __global__ void k_cent_split(RefitArgs a, unsigned long long* ccmax_bits) {
 // rows each), 4-7 = epilogue (one key row per thread).  Key tiles are
 // double-buffered; centre tiles stream through kTcBStages stages; two TMEM
 // accumulators of 128 columns alternate between UMMA and epilogue.
+// Band pass (kBandPass = true): the same kernel over the keys flagged by
+// the scan, with their first-pass best value known, lists every centre
+// whose screened d^2 is within 2 err of it (at most kBand; more is marked
+// as an overflow).  The screened values are bit-identical in both passes.
+struct BandArgs {
+  const int32_t* list;  // keys of this pass (scan list, or recheck list)
+  const int32_t* n;     // its length (device)
+  int32_t* recheck;     // scan: flagged keys out
+  int32_t* n_recheck;   // scan: their count
+  float* best;          // [cap] screened best d^2 of flagged key p
+  int32_t* ids;         // [cap, kBand] band: centre ids
+  int32_t* cnt;         // [cap] band: size (> kBand: overflow)
+  int cap;              // flagged keys that get a band
+};
+
+template <bool kBandPass>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_scan_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap hmap,
               const __grid_constant__ CUtensorMap lmap, RefitArgs a, int K_pad,
-              const unsigned long long* ccmax_bits, int32_t* recheck, int32_t* n_recheck) {
+              const unsigned long long* ccmax_bits, BandArgs bd) {
   extern __shared__ uint8_t raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sa = base;             // [2][kTcA]
@@ -611,7 +726,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ int abort_flag;
   volatile int* aborted = &abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = *a.n_scan;
+  const int n = kBandPass ? min(*bd.n, bd.cap) : *bd.n;
   const int ntiles = (n + kTcKeys - 1) / kTcKeys;
   const int nct = K_pad / kTcCent;
   if (threadIdx.x == 0) {
@@ -673,7 +788,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int kk = kt * kTcKeys + rl + q;
-        r[q] = kk < n ? a.scan_list[kk] : static_cast<int>(a.S);
+        r[q] = kk < n ? bd.list[kk] : static_cast<int>(a.S);
       }
       tma_gather4(sa + b * kTcA + half * (kTcKeys * 128) + rl * 128, &kmap, half * 64, r[0], r[1], r[2], r[3],
                   &afull[b]);
@@ -749,8 +864,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       mbar_arrive(&aempty[b]);
       const float err = static_cast<float>(kTcErr * (static_cast<double>(xx) + ccmax));
+      const int kk = kt * kTcKeys + row;
       float best = INFINITY, second = INFINITY;
       int bid = 0x7fffffff;
+      float thr = 0.f;
+      int nb = 0;
+      // rounded up: every centre whose exact d^2 can be the minimum is listed
+      if (kBandPass) thr = kk < n ? __fadd_ru(bd.best[kk], 2.f * err) : -INFINITY;
       for (int ct = 0; ct < nct; ++ct, ++gj) {
         const int acc = gj & 1;
         if (!mbar_wait(&tfull[acc], (gj >> 1) & 1, a.err, &abort_flag)) {
@@ -773,15 +893,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             cc[4 * q + 3] = t.w;
           }
           tmem_ld_wait();
+          if (kBandPass) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
-            if (d2 < best) {
-              second = best;
-              best = d2;
-              bid = ct * kTcCent + c32 * 32 + q;
-            } else if (d2 < second) {
-              second = d2;
+            for (int q = 0; q < 32; ++q) {
+              const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
+              if (d2 <= thr) {
+                if (nb < kBand) bd.ids[static_cast<int64_t>(kk) * kBand + nb] = ct * kTcCent + c32 * 32 + q;
+                ++nb;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
+              if (d2 < best) {
+                second = best;
+                best = d2;
+                bid = ct * kTcCent + c32 * 32 + q;
+              } else if (d2 < second) {
+                second = d2;
+              }
             }
           }
         }
@@ -789,13 +920,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_arrive(&tempty[acc]);
       }
       if (!ok) break;
-      const int kk = kt * kTcKeys + row;
-      if (kk < n && bid < a.K) {
-        const int32_t x = a.scan_list[kk];
+      if (kBandPass) {
+        if (kk < n) {
+          bd.cnt[kk] = nb;
+          bd.best[kk] = __fsub_rd(thr, err);  // exact d^2 of every centre outside the band is above this
+        }
+      } else if (kk < n && bid < a.K) {
+        const int32_t x = bd.list[kk];
         a.assign[x] = bid;
         if (!(second - best > 2.f * err)) {
-          const int p = atomicAdd(n_recheck, 1);
-          recheck[p] = x;
+          const int p = atomicAdd(bd.n_recheck, 1);
+          bd.recheck[p] = x;
+          if (p < bd.cap) bd.best[p] = best;
         }
         a.ub[x] = __fmul_ru(sqrtf(__fadd_ru(fmaxf(best, 0.f), err)), 1.f + 1e-6f);
         a.lb[x] = __fmul_rd(sqrtf(fmaxf(__fsub_rd(second, err), 0.f)), 1.f - 1e-6f);
@@ -813,6 +949,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }  // namespace
 
 int64_t refit_tile_size() { return kTileKeys; }
+int64_t refit_update_chunk() { return kUpdChunk; }
 
 cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
                          int32_t* host_nscan, const RefitTcMaps* tc) {
@@ -850,12 +987,32 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
     const int K_pad = (a.K + kTcCent - 1) / kTcCent * kTcCent;
     count_launch();
     k_cent_split<<<K_pad, 128, 0, st>>>(a, ccmax_bits);
-    cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTcSmem));
+    cudaFuncSetAttribute(k_scan_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTcSmem));
     const int64_t ktiles = (n + kTcKeys - 1) / kTcKeys;
     const int grid = static_cast<int>(ktiles < tc->num_sms ? ktiles : tc->num_sms);
+    BandArgs bd{};
+    bd.list = a.scan_list;
+    bd.n = a.n_scan;
+    bd.recheck = a.scan_list + n;
+    bd.n_recheck = n_recheck;
+    bd.best = a.band_best;
+    bd.ids = a.band_ids;
+    bd.cnt = a.band_cnt;
+    bd.cap = a.band_cap;
     count_launch();
-    k_scan_tc<<<grid, kTcThreads, kTcSmem, st>>>(tc->keys, tc->hi, tc->lo, a, K_pad, ccmax_bits,
-                                                  a.scan_list + n, n_recheck);
+    k_scan_tc<false><<<grid, kTcThreads, kTcSmem, st>>>(tc->keys, tc->hi, tc->lo, a, K_pad, ccmax_bits, bd);
+    // the flagged keys again, listing the centres within their error band
+    bd.list = a.scan_list + n;
+    bd.n = n_recheck;
+    cudaFuncSetAttribute(k_scan_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTcSmem));
+    const int bgrid = static_cast<int>((a.band_cap + kTcKeys - 1) / kTcKeys < tc->num_sms
+                                           ? (a.band_cap + kTcKeys - 1) / kTcKeys
+                                           : tc->num_sms);
+    count_launch();
+    k_scan_tc<true><<<bgrid, kTcThreads, kTcSmem, st>>>(tc->keys, tc->hi, tc->lo, a, K_pad, ccmax_bits, bd);
+    count_launch();
+    k_recheck_band<<<static_cast<unsigned>((a.band_cap + 7) / 8 < 1184 ? (a.band_cap + 7) / 8 : 1184), 256, 0,
+                     st>>>(a, a.scan_list + n, n_recheck, a.band_best, a.band_ids, a.band_cnt, a.band_cap);
   } else {
     const int64_t sblocks = (n + kSK - 1) / kSK;
     count_launch();
@@ -863,8 +1020,10 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
                                                                                     n_recheck);
   }
   // recheck list lives after the scan list (capacity n)
+  const int64_t rblocks = (n + kRkKeys - 1) / kRkKeys;
   count_launch();
-  k_recheck<<<static_cast<unsigned>(n < 1184 ? n : 1184), 256, 0, st>>>(a, a.scan_list + n, n_recheck);
+  k_recheck<<<static_cast<unsigned>(rblocks < 1184 ? rblocks : 1184), 256, 0, st>>>(
+      a, a.scan_list + n, n_recheck, a.band_cnt, tc ? a.band_cap : 0);
   count_launch();
   k_zero_counts<<<(a.K + 255) / 256, 256, 0, st>>>(a);
   count_launch();
@@ -880,8 +1039,12 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   k_tile_base<<<(a.K + 255) / 256, 256, 0, st>>>(a, static_cast<int>(ntiles));
   count_launch();
   k_scatter<<<static_cast<unsigned>(ntiles), 32, sm, st>>>(a);
+  // chunks: at most n / kUpdChunk + K
+  const int64_t max_chunks = n / kUpdChunk + a.K;
   count_launch();
-  k_update<<<static_cast<unsigned>((static_cast<int64_t>(a.K) * 32 + 255) / 256), 256, 0, st>>>(a, mdb);
+  k_update_part<<<static_cast<unsigned>((max_chunks * 32 + 255) / 256), 256, 0, st>>>(a);
+  count_launch();
+  k_update_fin<<<static_cast<unsigned>((static_cast<int64_t>(a.K) * 32 + 255) / 256), 256, 0, st>>>(a, mdb);
   count_launch();
   k_bounds<<<gk, 256, 0, st>>>(a);
   if (host_nscan) cudaMemcpyAsync(host_nscan, a.n_scan, 8, cudaMemcpyDeviceToHost, st);

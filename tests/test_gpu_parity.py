@@ -113,6 +113,31 @@ def test_many_refits_bounds_stay_exact():
     _run_prefill(wl, sample=4, check_exhaustive=False)
 
 
+def test_duplicate_keys_exact_ties():
+    """Keys drawn from 24 distinct vectors: centres coincide exactly, so the
+    refit meets exact distance ties (lowest centre id wins, including ties
+    among more centres than the near-tie band holds) and the seal meets
+    equal pair distances.  Index state must equal the oracle's after every
+    chunk."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=6144, T=512, window=128, clusters_per_window=4,
+                  refit_period=512, refit_new_seeds=24, budget=1024, k=64, M=64)
+    base = S.to_bf16_bits(S.keys_f64(wl, 0, 24))
+    pick = np.random.default_rng(5).integers(0, 24, size=wl.L)
+    bits = base[pick]
+    gpu, orc = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        p0, p1 = c * wl.T, (c + 1) * wl.T
+        kd = torch.from_numpy(bits[p0:p1].view(np.int16)).cuda().view(torch.bfloat16)
+        gpu.append_keys(kd)
+        orc.append(S.bf16_bits_to_f64(bits[p0:p1]))
+        gpu.seal()
+        orc.seal()
+        gpu.sync()
+        P.check_index_equal(gpu, orc)
+    assert gpu.stats()["n_refits"] >= 10
+    gpu.close()
+
+
 def test_rollback_replay_matches_a_fresh_index():
     """Replaying chunks after rollback (bounds and drifts restored) gives the
     same index as processing them once on a fresh handle."""
