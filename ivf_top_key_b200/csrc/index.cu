@@ -161,6 +161,10 @@ struct ai_index {
   int num_sms = 148;
   cudaStream_t main = nullptr, side = nullptr;
   cudaEvent_t ev_main = nullptr, ev_refit = nullptr;
+  // ev_main was recorded before this ai_seal call's seal kernels: a refit it
+  // triggers needs only the appended keys and the published buffers, so it
+  // may run beside the seal
+  bool refit_ev_early = false;
   // key store
   void* keys = nullptr;
   float* scales = nullptr;
@@ -373,6 +377,8 @@ int publish(ai_index* h) {
 }
 
 int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
+  const bool early = h->refit_ev_early && !h->pending;
+  h->refit_ev_early = false;
   int rc = publish(h);
   if (rc) return rc;
   const int64_t S = h->cfg.n_sinks, W = h->cfg.window;
@@ -389,7 +395,9 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
   if (K > h->maxC) return fail(AI_ERR_OOM, "cluster capacity exceeded at refit");
   if (ns > h->max_seeds) return fail(AI_ERR_ARG, "too many refit seeds");
   cudaStream_t st = h->cfg.async_refit ? h->side : h->main;
-  CK(cudaEventRecord(h->ev_main, h->main));
+  // the target buffer was last read by work on the main stream before the
+  // event (route/refine of earlier chunks, the publish copy)
+  if (!early) CK(cudaEventRecord(h->ev_main, h->main));
   CK(cudaStreamWaitEvent(st, h->ev_main, 0));
   if (ns > 0) {
     // the pinned staging buffer may still be read by an earlier refit's copy
@@ -772,6 +780,12 @@ int ai_seal(ai_handle h, int64_t* version_out) {
   if (!h) return fail(AI_ERR_ARG, "null handle");
   const int64_t S = h->cfg.n_sinks, W = h->cfg.window, R = h->cfg.refit_period;
   const int64_t complete = h->n_keys >= S ? (h->n_keys - S) / W : 0;
+  h->refit_ev_early = false;
+  if (R > 0 && h->cfg.async_refit && h->n_windows < complete &&
+      R / W - (h->n_windows % (R / W)) <= complete - h->n_windows) {
+    CK(cudaEventRecord(h->ev_main, h->main));
+    h->refit_ev_early = true;
+  }
   while (h->n_windows < complete) {
     int64_t nw = complete - h->n_windows;
     if (R > 0) {
@@ -781,18 +795,21 @@ int ai_seal(ai_handle h, int64_t* version_out) {
       nw = std::min(nw, to_refit);
     }
     int rc = seal_group(h, h->n_windows, nw);
-    if (rc) return rc;
-    if (R > 0 && (h->n_windows * W) % R == 0) {
+    if (rc == AI_OK && R > 0 && (h->n_windows * W) % R == 0)
       rc = start_refit(h, h->n_seed_default, h->seed_window_default);
-      if (rc) return rc;
+    if (rc) {
+      h->refit_ev_early = false;
+      return rc;
     }
   }
+  h->refit_ev_early = false;
   if (version_out) *version_out = static_cast<int64_t>(h->buf[h->active].versions.size());
   return AI_OK;
 }
 
 int ai_refit(ai_handle h, int32_t n_new_seeds, int32_t seed_window, int64_t* version_out) {
   if (!h || n_new_seeds < 0 || seed_window < 0) return fail(AI_ERR_ARG, "bad refit arguments");
+  h->refit_ev_early = false;
   int rc = start_refit(h, n_new_seeds > 0 ? n_new_seeds : h->n_seed_default,
                        seed_window > 0 ? seed_window : h->seed_window_default);
   if (rc) return rc;
