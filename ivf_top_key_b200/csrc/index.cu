@@ -610,7 +610,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   if (static_cast<int64_t>(cap) * c.clusters_per_window < c.window)
     return fail(AI_ERR_ARG, "cluster_cap * m < W: a window cannot be sealed");
   if (seal_smem_bytes(c.window, c.clusters_per_window, c.d) > 227 * 1024 ||
-      static_cast<int64_t>(c.window) * c.clusters_per_window > 65535)
+      static_cast<int64_t>(c.window) * c.clusters_per_window > 65535 || c.window > 32767 ||
+      c.clusters_per_window > 64)
     return fail(AI_ERR_ARG, "window too large to seal in one CTA");
   const bool tcr = c.q_dtype == AI_BF16 && c.d == 128 && (c.H == 32 || c.H == 64);
   const bool tck = tcr && c.key_dtype != AI_FP32;

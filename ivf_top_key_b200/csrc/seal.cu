@@ -15,44 +15,101 @@
 // Members are stored per cluster in ascending key id; the representative is
 // the mean rounded once to bf16 (round to nearest even).
 //
-// One CTA (1024 threads) per window.  The sequential greedy walk over the
+// One CTA (512 threads) per window.  The sequential greedy walk over the
 // W*m sorted pairs is reproduced exactly in at most m + 1 data-parallel
 // rounds: in a round every free key proposes its best pair among the
-// clusters that are not full; the proposals are sorted by (cluster, pair
-// order); the first cluster to fill is the one whose (cap - count)-th
-// proposal comes first in pair order; every proposal up to that pair is
-// final (nothing before it can be refused), that cluster is closed, and the
-// remaining keys propose again.  Pair order is (distance, key, cluster).
+// clusters that are not full; the first cluster to fill is the one whose
+// (cap - count)-th smallest proposal comes first in pair order; every
+// proposal up to that pair is final (nothing before it can be refused),
+// that cluster is closed, and the remaining keys propose again.  Pair order
+// is (distance, key, cluster).
+//
+// The (cap - count)-th smallest proposal of each cluster is selected with a
+// histogram over the cluster's distance range (bins are a monotone function
+// of the distance, so the element lies in the bin where the running count
+// reaches it) and an exact rank among the few proposals of that one bin.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace aiidx {
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
+constexpr int kBins = 1024;  // histogram bins per cluster
 
 struct SealSmem {
-  double* D;         // [W, m] squared distances
+  double* D;         // [m, W] squared distances (cluster-major)
   double* cent;      // [m, d]
   double* cc;        // [m] squared centre norms
-  uint64_t* bk1;     // [m, NPW] proposal buckets: distance bits
-  uint16_t* bk2;     // [m, NPW] proposal buckets: key
-  int* wcnt;         // [m, 32] per-(cluster, warp) counts / offsets
-  int* bfill;        // [m] bucket sizes
-  int* bpass;        // [m]
+  double* dlo;       // [m] smallest distance to the cluster (bin origin)
+  double* dsc;       // [m] bins per unit distance
+  uint64_t* fk1;     // [m] fill pair of each cluster: distance bits
+  int* hist;         // [m, kBins]
+  uint32_t* fk2;     // [m] fill pair: (key << 16) | cluster
+  int* cnt;          // [m] members so far
+  int* tb;           // [m] bin holding the filling proposal (-1: no fill)
+  int* cb;           // [m] proposals in the bins before it
+  int* cstart;       // [m + 1] member list starts
+  int* misc;         // [0] best cluster, [1] collected, [2] free keys, [3] changed
+  unsigned long long* fullmask;
+  int8_t* prop;      // [W] proposal of each free key (-1: none)
   int16_t* assign;   // [W]
   int16_t* prev;     // [W]
-  int* cnt;          // [m] members so far
-  int* tcnt;         // [m] (spare)
-  int* tstart;       // [m + 1] (spare)
-  int* cstart;       // [m + 1] member list starts
   int16_t* mlist;    // [W] members, grouped by cluster, ascending
-  uint64_t* fk1;     // [m] fill pair of each cluster: distance bits
-  uint32_t* fk2;     // [m] fill pair: (key << 16) | cluster
-  int* flag;         // [4]
-  int* red;          // [32] per-warp partial sums
-  unsigned long long* fullmask;
+  int16_t* coll;     // [W] proposals in the target bins
 };
+
+// Lays the arrays out from p; returns the bytes used.  Shared by the kernel
+// and the host-side size computation.
+__host__ __device__ inline size_t seal_layout(uint8_t* p, int W, int m, int d, SealSmem* s) {
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* q = p + o;
+    o += (bytes + 15) & ~size_t(15);
+    return q;
+  };
+  uint8_t* D = take(static_cast<size_t>(W) * m * 8);
+  uint8_t* cent = take(static_cast<size_t>(m) * d * 8);
+  uint8_t* cc = take(static_cast<size_t>(m) * 8);
+  uint8_t* dlo = take(static_cast<size_t>(m) * 8);
+  uint8_t* dsc = take(static_cast<size_t>(m) * 8);
+  uint8_t* fk1 = take(static_cast<size_t>(m) * 8);
+  uint8_t* full = take(8);
+  uint8_t* hist = take(static_cast<size_t>(m) * kBins * 4);
+  uint8_t* fk2 = take(static_cast<size_t>(m) * 4);
+  uint8_t* cnt = take(static_cast<size_t>(m) * 4);
+  uint8_t* tb = take(static_cast<size_t>(m) * 4);
+  uint8_t* cb = take(static_cast<size_t>(m) * 4);
+  uint8_t* cstart = take(static_cast<size_t>(m + 1) * 4);
+  uint8_t* misc = take(16);
+  uint8_t* prop = take(static_cast<size_t>(W));
+  uint8_t* assign = take(static_cast<size_t>(W) * 2);
+  uint8_t* prev = take(static_cast<size_t>(W) * 2);
+  uint8_t* mlist = take(static_cast<size_t>(W) * 2);
+  uint8_t* coll = take(static_cast<size_t>(W) * 2);
+  if (s) {
+    s->D = reinterpret_cast<double*>(D);
+    s->cent = reinterpret_cast<double*>(cent);
+    s->cc = reinterpret_cast<double*>(cc);
+    s->dlo = reinterpret_cast<double*>(dlo);
+    s->dsc = reinterpret_cast<double*>(dsc);
+    s->fk1 = reinterpret_cast<uint64_t*>(fk1);
+    s->fullmask = reinterpret_cast<unsigned long long*>(full);
+    s->hist = reinterpret_cast<int*>(hist);
+    s->fk2 = reinterpret_cast<uint32_t*>(fk2);
+    s->cnt = reinterpret_cast<int*>(cnt);
+    s->tb = reinterpret_cast<int*>(tb);
+    s->cb = reinterpret_cast<int*>(cb);
+    s->cstart = reinterpret_cast<int*>(cstart);
+    s->misc = reinterpret_cast<int*>(misc);
+    s->prop = reinterpret_cast<int8_t*>(prop);
+    s->assign = reinterpret_cast<int16_t*>(assign);
+    s->prev = reinterpret_cast<int16_t*>(prev);
+    s->mlist = reinterpret_cast<int16_t*>(mlist);
+    s->coll = reinterpret_cast<int16_t*>(coll);
+  }
+  return o;
+}
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
@@ -97,56 +154,104 @@ __device__ __forceinline__ bool pair_le(uint64_t d1, uint32_t i1, uint32_t j1, u
   return j1 <= j2;
 }
 
-__global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
-  extern __shared__ uint8_t raw[];
-  const int W = a.W, m = a.m, d = a.d;
-  int NPW = 1;
-  while (NPW < W) NPW <<= 1;
-  SealSmem s;
-  uint8_t* p = raw;
-  s.D = reinterpret_cast<double*>(p);
-  p += static_cast<size_t>(W) * m * 8;
-  s.cent = reinterpret_cast<double*>(p);
-  p += static_cast<size_t>(m) * d * 8;
-  s.cc = reinterpret_cast<double*>(p);
-  p += static_cast<size_t>(m) * 8;
-  s.bk1 = reinterpret_cast<uint64_t*>(p);
-  p += static_cast<size_t>(m) * NPW * 8;
-  s.fk1 = reinterpret_cast<uint64_t*>(p);
-  p += static_cast<size_t>(m) * 8;
-  s.fullmask = reinterpret_cast<unsigned long long*>(p);
-  p += 8;
-  s.wcnt = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 32 * 4;
-  s.bfill = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.bpass = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.fk2 = reinterpret_cast<uint32_t*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.cnt = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.tcnt = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m) * 4;
-  s.tstart = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m + 1) * 4;
-  s.cstart = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(m + 1) * 4;
-  s.flag = reinterpret_cast<int*>(p);
-  p += 16;
-  s.red = reinterpret_cast<int*>(p);
-  p += 128;
-  s.assign = reinterpret_cast<int16_t*>(p);
-  p += static_cast<size_t>(W) * 2;
-  s.prev = reinterpret_cast<int16_t*>(p);
-  p += static_cast<size_t>(W) * 2;
-  s.mlist = reinterpret_cast<int16_t*>(p);
-  p += static_cast<size_t>(W) * 2;
-  s.bk2 = reinterpret_cast<uint16_t*>(p);
+__device__ __forceinline__ uint64_t dbits(double v) { return static_cast<uint64_t>(__double_as_longlong(v)); }
 
+// Histogram bin of a distance to cluster j: non-decreasing in the distance
+// (each rounded step is monotone), so a smaller bin means a smaller distance.
+__device__ __forceinline__ int dist_bin(const SealSmem& s, int j, double v) {
+  const int b = __double2int_rz((v - s.dlo[j]) * s.dsc[j]);
+  return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
+}
+
+// D[j, i] for all keys of the window, two key rows per thread, the centre
+// values read as pairs (the summation order per (i, j) is dimension order).
+template <int MM>
+__device__ __forceinline__ void seal_dist(const SealArgs& a, const SealSmem& s, int64_t lo) {
+  const int W = a.W, m = a.m, d = a.d;
+  for (int i0 = 2 * threadIdx.x; i0 < W; i0 += 2 * blockDim.x) {
+    const bool two = i0 + 1 < W;
+    double xx0 = 0.0, xx1 = 0.0;
+    double acc0[MM], acc1[MM];
+#pragma unroll
+    for (int j = 0; j < MM; ++j) {
+      acc0[j] = 0.0;
+      acc1[j] = 0.0;
+    }
+    for (int e0 = 0; e0 < d; e0 += 8) {
+      double x0[8], x1[8];
+      load8(a, lo + i0, e0, x0);
+      if (two) {
+        load8(a, lo + i0 + 1, e0, x1);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x1[u] = 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        xx0 = fma(x0[u], x0[u], xx0);
+        xx1 = fma(x1[u], x1[u], xx1);
+      }
+#pragma unroll
+      for (int j = 0; j < MM; ++j) {
+        if (j < m) {
+          const double2* c2 = reinterpret_cast<const double2*>(s.cent + j * d + e0);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const double2 c = c2[u];
+            acc0[j] = fma(x0[2 * u], c.x, acc0[j]);
+            acc0[j] = fma(x0[2 * u + 1], c.y, acc0[j]);
+            acc1[j] = fma(x1[2 * u], c.x, acc1[j]);
+            acc1[j] = fma(x1[2 * u + 1], c.y, acc1[j]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < MM; ++j) {
+      if (j < m) {
+        s.D[j * W + i0] = fmax(0.0, fma(-2.0, acc0[j], xx0) + s.cc[j]);
+        if (two) s.D[j * W + i0 + 1] = fmax(0.0, fma(-2.0, acc1[j], xx1) + s.cc[j]);
+      }
+    }
+  }
+}
+
+// Any m: one centre at a time (key row re-read per centre).
+__device__ __forceinline__ void seal_dist_any(const SealArgs& a, const SealSmem& s, int64_t lo) {
+  const int W = a.W, m = a.m, d = a.d;
+  for (int i = threadIdx.x; i < W; i += blockDim.x) {
+    double xx = 0.0;
+    for (int e0 = 0; e0 < d; e0 += 8) {
+      double x[8];
+      load8(a, lo + i, e0, x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) xx = fma(x[u], x[u], xx);
+    }
+    for (int j = 0; j < m; ++j) {
+      double acc = 0.0;
+      for (int e0 = 0; e0 < d; e0 += 8) {
+        double x[8];
+        load8(a, lo + i, e0, x);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc = fma(x[u], s.cent[j * d + e0 + u], acc);
+      }
+      s.D[j * W + i] = fmax(0.0, fma(-2.0, acc, xx) + s.cc[j]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
+  extern __shared__ __align__(16) uint8_t raw[];
+  const int W = a.W, m = a.m, d = a.d;
+  SealSmem s;
+  seal_layout(raw, W, m, d, &s);
   const int win = blockIdx.x;
   const int64_t lo = a.first_key + static_cast<int64_t>(win) * W;
   const int tid = threadIdx.x;
+  const int warp = warp_id(), lane = lane_id();
+  const int nwarps = blockDim.x >> 5;
+  // loop bound over keys rounded up to whole warps (ballots need every lane)
+  const int Wr = (W + 31) & ~31;
 
   // strided initialisation
   for (int e = tid; e < m * d; e += blockDim.x) {
@@ -158,265 +263,213 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
 
   for (int it = 0; it < a.iters; ++it) {
     // squared centre norms for this pass
-    for (int j = warp_id(); j < m; j += blockDim.x >> 5) {
+    for (int j = warp; j < m; j += nwarps) {
       double cc = 0.0;
-      for (int e = lane_id(); e < d; e += 32) cc = fma(s.cent[j * d + e], s.cent[j * d + e], cc);
+      for (int e = lane; e < d; e += 32) cc = fma(s.cent[j * d + e], s.cent[j * d + e], cc);
       for (int o = 16; o > 0; o >>= 1) cc += __shfl_xor_sync(0xffffffffu, cc, o);
-      if (lane_id() == 0) s.cc[j] = cc;
+      if (lane == 0) s.cc[j] = cc;
     }
     __syncthreads();
-    // distances ||x||^2 - 2 x.c + ||c||^2 (float64, clamped at 0): one key
-    // row per thread, read once, 32 elements per batch of loads
-    for (int i = tid; i < W; i += blockDim.x) {
-      const int64_t row = lo + i;
-      double xx = 0.0;
-      if (m <= 16) {
-        double acc[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = 0.0;
-        for (int e0 = 0; e0 < d; e0 += 8) {
-          double x[8];
-          load8(a, row, e0, x);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) xx = fma(x[u], x[u], xx);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j < m) {
-              const double* c = s.cent + j * d + e0;
-#pragma unroll
-              for (int u = 0; u < 8; ++u) acc[j] = fma(x[u], c[u], acc[j]);
-            }
-          }
-        }
-        for (int j = 0; j < m; ++j) s.D[i * m + j] = fmax(0.0, fma(-2.0, acc[j], xx) + s.cc[j]);
-      } else {
-        for (int e0 = 0; e0 < d; e0 += 8) {
-          double x[8];
-          load8(a, row, e0, x);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) xx = fma(x[u], x[u], xx);
-        }
-        for (int j = 0; j < m; ++j) {
-          double acc = 0.0;
-          for (int e0 = 0; e0 < d; e0 += 8) {
-            double x[8];
-            load8(a, row, e0, x);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc = fma(x[u], s.cent[j * d + e0 + u], acc);
-          }
-          s.D[i * m + j] = fmax(0.0, fma(-2.0, acc, xx) + s.cc[j]);
-        }
-      }
-      s.assign[i] = -1;
-    }
+    if (m <= 8) seal_dist<8>(a, s, lo);
+    else if (m <= 16) seal_dist<16>(a, s, lo);
+    else seal_dist_any(a, s, lo);
+    for (int i = tid; i < W; i += blockDim.x) s.assign[i] = -1;
     for (int j = tid; j < m; j += blockDim.x) s.cnt[j] = 0;
-    if (tid == 0) *s.fullmask = 0ull;
+    if (tid == 0) {
+      *s.fullmask = 0ull;
+      s.misc[2] = W;
+    }
+    __syncthreads();
+    // per-cluster distance range: the histogram's origin and scale
+    for (int j = warp; j < m; j += nwarps) {
+      double mn = INFINITY, mx = 0.0;
+      for (int i = lane; i < W; i += 32) {
+        const double v = s.D[j * W + i];
+        mn = fmin(mn, v);
+        mx = fmax(mx, v);
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        s.dlo[j] = mn;
+        s.dsc[j] = mx > mn ? static_cast<double>(kBins) / (mx - mn) : 0.0;
+      }
+    }
     __syncthreads();
 
     // greedy capacity assignment in rounds (see the file comment)
-    int n_free = W;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int nwarps = blockDim.x >> 5;
-    for (int round = 0; round <= m && n_free > 0; ++round) {
+    for (int round = 0; round <= m && s.misc[2] > 0; ++round) {
       const unsigned long long fullm = *s.fullmask;
-      // 1. proposals, bucketed by cluster without atomics: per-warp ballot
-      //    counts -> (cluster, warp) offsets -> scatter
-      for (int j = tid; j < m; j += blockDim.x) s.bfill[j] = 0;
+      // A. clear the histograms and the fill pairs
+      for (int e = tid; e < m * kBins; e += blockDim.x) s.hist[e] = 0;
+      for (int j = tid; j < m; j += blockDim.x) {
+        s.fk1[j] = ~0ull;
+        s.fk2[j] = ~0u;
+      }
+      if (tid == 0) s.misc[1] = 0;
       __syncthreads();
-      for (int i0 = 0; i0 < W; i0 += blockDim.x) {
-        const int i = i0 + tid;
+      // B. proposals: best open cluster of every free key, counted per bin
+      for (int i = tid; i < W; i += blockDim.x) {
         int bj = -1;
         double bd = 0.0;
-        if (i < W && s.assign[i] < 0) {
+        if (s.assign[i] < 0) {
           for (int j = 0; j < m; ++j) {
             if ((fullm >> j) & 1ull) continue;
-            const double v = s.D[i * m + j];
+            const double v = s.D[j * W + i];
             if (bj < 0 || v < bd) {
               bj = j;
               bd = v;
             }
           }
         }
-        for (int j = 0; j < m; ++j) {
-          const unsigned bal = __ballot_sync(0xffffffffu, bj == j);
-          if (lane == 0) s.wcnt[j * nwarps + warp] = __popc(bal);
-        }
-        __syncthreads();
-        // exclusive offsets of (cluster j, warp w) within this pass
-        if (tid < m) {
+        s.prop[i] = static_cast<int8_t>(bj);
+        if (bj >= 0) atomicAdd(&s.hist[bj * kBins + dist_bin(s, bj, bd)], 1);
+      }
+      __syncthreads();
+      // C. per open cluster, the bin where the running count reaches the
+      //    (cap - count)-th proposal (none if the cluster cannot fill now)
+      for (int j = warp; j < m; j += nwarps) {
+        int found = -1, before = 0;
+        if (!((fullm >> j) & 1ull)) {
+          const int need = a.cap - s.cnt[j];
           int run = 0;
-          for (int w = 0; w < nwarps; ++w) {
-            const int c = s.wcnt[tid * nwarps + w];
-            s.wcnt[tid * nwarps + w] = run;
-            run += c;
+          for (int b0 = 0; b0 < kBins; b0 += 32) {
+            const int v = s.hist[j * kBins + b0 + lane];
+            int incl = v;
+            for (int o = 1; o < 32; o <<= 1) {
+              const int t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (run + tot >= need) {
+              const unsigned bal = __ballot_sync(0xffffffffu, run + incl >= need);
+              const int first = __ffs(bal) - 1;
+              const int excl = __shfl_sync(0xffffffffu, incl - v, first);
+              found = b0 + first;
+              before = run + excl;
+              break;
+            }
+            run += tot;
           }
-          s.bpass[tid] = run;
         }
-        __syncthreads();
-        for (int j = 0; j < m; ++j) {
-          const unsigned bal = __ballot_sync(0xffffffffu, bj == j);
-          if (bj == j) {
-            const int slot = s.bfill[j] + s.wcnt[j * nwarps + warp] + __popc(bal & ((1u << lane) - 1u));
-            s.bk1[j * NPW + slot] = static_cast<uint64_t>(__double_as_longlong(bd));
-            s.bk2[j * NPW + slot] = static_cast<uint16_t>(i);
-          }
-        }
-        __syncthreads();
-        if (tid < m) s.bfill[tid] += s.bpass[tid];
-        __syncthreads();
-      }
-      // 2. the proposal that would fill each open cluster: the need-th
-      //    smallest (distance, key) of its bucket, found by counting ranks
-      //    (all threads; one entry each, compared against its bucket)
-      if (tid == 0) {
-        int run = 0;
-        for (int j = 0; j < m; ++j) {
-          s.tstart[j] = run;
-          run += s.bfill[j];
-        }
-        s.tstart[m] = run;
-      }
-      for (int j = tid; j < m; j += blockDim.x) {
-        s.fk1[j] = ~0ull;
-        s.fk2[j] = ~0u;
-      }
-      __syncthreads();
-      for (int e = tid; e < s.tstart[m]; e += blockDim.x) {
-        int j = 0;
-        while (j + 1 < m && s.tstart[j + 1] <= e) ++j;
-        const int need = a.cap - s.cnt[j];
-        const int nb = s.bfill[j];
-        if (((fullm >> j) & 1ull) || nb < need || need <= 0) continue;
-        const uint64_t* k1 = s.bk1 + j * NPW;
-        const uint16_t* k2 = s.bk2 + j * NPW;
-        const int me = e - s.tstart[j];
-        const uint64_t a1 = k1[me];
-        const uint16_t a2 = k2[me];
-        int rank = 0;
-        for (int x = 0; x < nb; ++x) {
-          const uint64_t b1 = k1[x];
-          rank += (b1 < a1 || (b1 == a1 && k2[x] < a2)) ? 1 : 0;
-        }
-        if (rank == need - 1) {
-          s.fk1[j] = a1;
-          s.fk2[j] = (static_cast<uint32_t>(a2) << 16) | static_cast<uint32_t>(j);
+        if (lane == 0) {
+          s.tb[j] = found;
+          s.cb[j] = before;
         }
       }
       __syncthreads();
+      // D. collect the proposals lying in their cluster's target bin
+      for (int i = tid; i < W; i += blockDim.x) {
+        const int j = s.prop[i];
+        if (j >= 0 && s.tb[j] >= 0 && dist_bin(s, j, s.D[j * W + i]) == s.tb[j])
+          s.coll[atomicAdd(&s.misc[1], 1)] = static_cast<int16_t>(i);
+      }
+      __syncthreads();
+      // E. exact rank (distance bits, key) inside the target bin
+      const int nc = s.misc[1];
+      for (int e = tid; e < nc; e += blockDim.x) {
+        const int i = s.coll[e];
+        const int j = s.prop[i];
+        const uint64_t di = dbits(s.D[j * W + i]);
+        int r = 0;
+        for (int x = 0; x < nc; ++x) {
+          const int k2 = s.coll[x];
+          if (s.prop[k2] != j) continue;
+          const uint64_t dk = dbits(s.D[j * W + k2]);
+          r += (dk < di || (dk == di && k2 < i)) ? 1 : 0;
+        }
+        if (r == a.cap - s.cnt[j] - s.cb[j] - 1) {
+          s.fk1[j] = di;
+          s.fk2[j] = (static_cast<uint32_t>(i) << 16) | static_cast<uint32_t>(j);
+        }
+      }
+      __syncthreads();
+      // F. the cluster that fills first closes this round
       if (tid == 0) {
         int best = -1;
         for (int j = 0; j < m; ++j) {
-          if (s.fk1[j] == ~0ull && s.fk2[j] == ~0u) continue;
-          if (best < 0 || pair_le(s.fk1[j], s.fk2[j] >> 16, s.fk2[j] & 0xFFFFu, s.fk1[best],
-                                  s.fk2[best] >> 16, s.fk2[best] & 0xFFFFu))
+          if (s.fk2[j] == ~0u) continue;
+          if (best < 0 || pair_le(s.fk1[j], s.fk2[j] >> 16, j, s.fk1[best], s.fk2[best] >> 16,
+                                  static_cast<uint32_t>(best)))
             best = j;
         }
-        s.flag[2] = best;
+        s.misc[0] = best;
+        if (best >= 0) *s.fullmask |= 1ull << best;
       }
       __syncthreads();
-      const int best = s.flag[2];
+      // G. commit every proposal up to the filling pair (all if none)
+      const int best = s.misc[0];
       const uint64_t bk1 = best >= 0 ? s.fk1[best] : 0;
       const uint32_t bi = best >= 0 ? (s.fk2[best] >> 16) : 0;
-      // 3. commit every proposal up to the filling pair (all if none)
-      for (int i = tid; i < W; i += blockDim.x) {
-        if (s.assign[i] >= 0) continue;
-        int bj = -1;
-        double bd = 0.0;
-        for (int j = 0; j < m; ++j) {
-          if ((fullm >> j) & 1ull) continue;
-          const double v = s.D[i * m + j];
-          if (bj < 0 || v < bd) {
-            bj = j;
-            bd = v;
-          }
-        }
-        if (bj >= 0 && (best < 0 || pair_le(static_cast<uint64_t>(__double_as_longlong(bd)), i, bj, bk1, bi,
-                                            static_cast<uint32_t>(best))))
-          s.assign[i] = static_cast<int16_t>(bj);
+      for (int i0 = warp * 32; i0 < Wr; i0 += blockDim.x) {
+        const int i = i0 + lane;
+        const int j = i < W ? s.prop[i] : -1;
+        bool take = false;
+        if (j >= 0)
+          take = best < 0 || pair_le(dbits(s.D[j * W + i]), i, j, bk1, bi, static_cast<uint32_t>(best));
+        if (take) s.assign[i] = static_cast<int16_t>(j);
+        const int tj = take ? j : -1;
+        const unsigned grp = __match_any_sync(0xffffffffu, tj);
+        if (take && lane == __ffs(grp) - 1) atomicAdd(&s.cnt[j], __popc(grp));
+        const unsigned nt = __ballot_sync(0xffffffffu, take);
+        if (lane == 0 && nt) atomicSub(&s.misc[2], __popc(nt));
       }
-      if (tid == 0 && best >= 0) *s.fullmask |= 1ull << best;
       __syncthreads();
-      // member counts and keys still free (ballots, no shared atomics)
-      {
-        int mine = 0;
-        for (int i = tid; i < W; i += blockDim.x) mine += s.assign[i] < 0 ? 1 : 0;
-        for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
-        if (lane == 0) s.red[warp] = mine;
-        for (int j = 0; j < m; ++j) {
-          int cj = 0;
-          for (int i0 = 0; i0 < W; i0 += blockDim.x) {
-            const int i = i0 + tid;
-            cj += __popc(__ballot_sync(0xffffffffu, i < W && s.assign[i] == j));
-          }
-          if (lane == 0) s.wcnt[j * nwarps + warp] = cj;
-        }
-        __syncthreads();
-        n_free = 0;
-        for (int w = 0; w < nwarps; ++w) n_free += s.red[w];
-        if (tid < m) {
-          int c = 0;
-          for (int w = 0; w < nwarps; ++w) c += s.wcnt[tid * nwarps + w];
-          s.cnt[tid] = c;
-        }
-        __syncthreads();
-      }
     }
-    if (tid == 0 && n_free != 0) atomicOr(a.err, DEV_ERR_CAPACITY);
+    if (tid == 0 && s.misc[2] != 0) atomicOr(a.err, DEV_ERR_CAPACITY);
 
     // member lists (ascending key order), one warp per cluster
-    {
-      const int warp = tid >> 5, lane = tid & 31;
-      if (tid == 0) {
-        int run = 0;
-        for (int j = 0; j < m; ++j) {
-          s.cstart[j] = run;
-          run += s.cnt[j];
-        }
-        s.cstart[m] = run;
+    if (tid == 0) {
+      int run = 0;
+      for (int j = 0; j < m; ++j) {
+        s.cstart[j] = run;
+        run += s.cnt[j];
       }
-      __syncthreads();
-      for (int j = warp; j < m; j += blockDim.x >> 5) {
-        int w = s.cstart[j];
-        for (int x0 = 0; x0 < W; x0 += 32) {
-          const int x = x0 + lane;
-          const bool in = x < W && s.assign[x] == j;
-          const unsigned bal = __ballot_sync(0xffffffffu, in);
-          if (in) s.mlist[w + __popc(bal & ((1u << lane) - 1u))] = static_cast<int16_t>(x);
-          w += __popc(bal);
-        }
-      }
-      __syncthreads();
-      // update: float64 mean of the members in ascending key order; the
-      // (cluster, 32-dim block) pairs are spread over all warps
-      const int nblk = (d + 31) / 32;
-      for (int wj = warp; wj < m * nblk; wj += blockDim.x >> 5) {
-        const int j = wj / nblk;
-        const int b0 = s.cstart[j], b1 = s.cstart[j + 1];
-        if (b1 == b0) continue;
-        for (int e = (wj % nblk) * 32 + lane; e < d && e < (wj % nblk) * 32 + 32; e += 32) {
-          double sum = 0.0;
-          int q = b0;
-          for (; q + 4 <= b1; q += 4) {
-            const double v0 = key_f64(a, lo + s.mlist[q], e);
-            const double v1 = key_f64(a, lo + s.mlist[q + 1], e);
-            const double v2 = key_f64(a, lo + s.mlist[q + 2], e);
-            const double v3 = key_f64(a, lo + s.mlist[q + 3], e);
-            sum += v0;
-            sum += v1;
-            sum += v2;
-            sum += v3;
-          }
-          for (; q < b1; ++q) sum += key_f64(a, lo + s.mlist[q], e);
-          s.cent[j * d + e] = sum / static_cast<double>(b1 - b0);
-        }
+      s.cstart[m] = run;
+    }
+    __syncthreads();
+    for (int j = warp; j < m; j += nwarps) {
+      int w = s.cstart[j];
+      for (int x0 = 0; x0 < W; x0 += 32) {
+        const int x = x0 + lane;
+        const bool in = x < W && s.assign[x] == j;
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        if (in) s.mlist[w + __popc(bal & ((1u << lane) - 1u))] = static_cast<int16_t>(x);
+        w += __popc(bal);
       }
     }
-    if (tid == 0) s.flag[0] = 0;
+    __syncthreads();
+    // update: float64 mean of the members in ascending key order; the
+    // (cluster, 32-dim block) pairs are spread over all warps, 16 member
+    // rows in flight per lane (added in member order)
+    {
+      const int nblk = (d + 31) / 32;
+      for (int wj = warp; wj < m * nblk; wj += nwarps) {
+        const int j = wj / nblk;
+        const int e = (wj % nblk) * 32 + lane;
+        const int b0 = s.cstart[j], b1 = s.cstart[j + 1];
+        if (b1 == b0 || e >= d) continue;
+        double sum = 0.0;
+        int q = b0;
+        for (; q + 16 <= b1; q += 16) {
+          double v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = key_f64(a, lo + s.mlist[q + u], e);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) sum += v[u];
+        }
+        for (; q < b1; ++q) sum += key_f64(a, lo + s.mlist[q], e);
+        s.cent[j * d + e] = sum / static_cast<double>(b1 - b0);
+      }
+    }
+    if (tid == 0) s.misc[3] = 0;
     __syncthreads();
     for (int i = tid; i < W; i += blockDim.x)
-      if (s.assign[i] != s.prev[i]) s.flag[0] = 1;
+      if (s.assign[i] != s.prev[i]) s.misc[3] = 1;
     __syncthreads();
-    const bool changed = s.flag[0] != 0;
+    const bool changed = s.misc[3] != 0;
     for (int i = tid; i < W; i += blockDim.x) s.prev[i] = s.assign[i];
     __syncthreads();
     if (!changed) break;
@@ -425,7 +478,7 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
   // outputs: CSR (members ascending within each cluster), centroids, reps
   const int64_t mem0 = a.mem_base + static_cast<int64_t>(win) * W;
   const int64_t cl0 = a.cl_base + static_cast<int64_t>(win) * m;
-  if (tid < m) a.offsets[cl0 + tid] = static_cast<int32_t>(mem0 + s.cstart[tid]);
+  for (int j = tid; j < m; j += blockDim.x) a.offsets[cl0 + j] = static_cast<int32_t>(mem0 + s.cstart[j]);
   for (int x = tid; x < W; x += blockDim.x) a.members[mem0 + x] = static_cast<int32_t>(lo + s.mlist[x]);
   if (win == gridDim.x - 1 && tid == 0)
     a.offsets[a.cl_base + static_cast<int64_t>(gridDim.x) * m] =
@@ -438,20 +491,11 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
 
 }  // namespace
 
-size_t seal_smem_bytes(int W, int m, int d) {
-  int NPW = 1;
-  while (NPW < W) NPW <<= 1;
-  // D, centres, proposal buckets (m x NPW of u64 + u16), counters, key lists
-  return static_cast<size_t>(W) * m * 8 + static_cast<size_t>(m) * d * 8 +
-         static_cast<size_t>(m) * NPW * 10 + static_cast<size_t>(m) * 12 + 8 +
-         static_cast<size_t>(m) * 32 * 4 + static_cast<size_t>(m) * 8 +
-         static_cast<size_t>(m + 1) * 8 + 16 + 128 + static_cast<size_t>(W) * 6 +
-         static_cast<size_t>(m) * 32 + 256 + static_cast<size_t>(m) * 8;
-}
+size_t seal_smem_bytes(int W, int m, int d) { return seal_layout(nullptr, W, m, d, nullptr) + 16; }
 
 cudaError_t launch_seal(const SealArgs& a, cudaStream_t st) {
   if (a.n_windows <= 0) return cudaSuccess;
-  if (a.m > 64 || a.W > 65535 || a.d % 8 != 0) return cudaErrorInvalidValue;
+  if (a.m < 1 || a.m > 64 || a.W < 1 || a.W > 32767 || a.d % 8 != 0) return cudaErrorInvalidValue;
   const size_t smem = seal_smem_bytes(a.W, a.m, a.d);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaFuncSetAttribute(k_seal, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
