@@ -35,7 +35,7 @@ namespace aiidx {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kBins = 1024;  // histogram bins per cluster
+constexpr int kBins = 1024;  // histogram bins per cluster (32 chunks of 32)
 
 struct SealSmem {
   double* D;         // [m, W] squared distances (cluster-major)
@@ -50,13 +50,14 @@ struct SealSmem {
   int* tb;           // [m] bin holding the filling proposal (-1: no fill)
   int* cb;           // [m] proposals in the bins before it
   int* cstart;       // [m + 1] member list starts
-  int* misc;         // [0] best cluster, [1] collected, [2] free keys, [3] changed
+  int* ncoll;        // [m] proposals collected from the target bin
+  int* misc;         // [0] best cluster, [2] free keys, [3] changed
   unsigned long long* fullmask;
   int8_t* prop;      // [W] proposal of each free key (-1: none)
   int16_t* assign;   // [W]
   int16_t* prev;     // [W]
   int16_t* mlist;    // [W] members, grouped by cluster, ascending
-  int16_t* coll;     // [W] proposals in the target bins
+  int16_t* coll;     // [m, W] proposals in each cluster's target bin
 };
 
 // Lays the arrays out from p; returns the bytes used.  Shared by the kernel
@@ -81,12 +82,13 @@ __host__ __device__ inline size_t seal_layout(uint8_t* p, int W, int m, int d, S
   uint8_t* tb = take(static_cast<size_t>(m) * 4);
   uint8_t* cb = take(static_cast<size_t>(m) * 4);
   uint8_t* cstart = take(static_cast<size_t>(m + 1) * 4);
+  uint8_t* ncoll = take(static_cast<size_t>(m) * 4);
   uint8_t* misc = take(16);
   uint8_t* prop = take(static_cast<size_t>(W));
   uint8_t* assign = take(static_cast<size_t>(W) * 2);
   uint8_t* prev = take(static_cast<size_t>(W) * 2);
   uint8_t* mlist = take(static_cast<size_t>(W) * 2);
-  uint8_t* coll = take(static_cast<size_t>(W) * 2);
+  uint8_t* coll = take(static_cast<size_t>(W) * m * 2);
   if (s) {
     s->D = reinterpret_cast<double*>(D);
     s->cent = reinterpret_cast<double*>(cent);
@@ -101,6 +103,7 @@ __host__ __device__ inline size_t seal_layout(uint8_t* p, int W, int m, int d, S
     s->tb = reinterpret_cast<int*>(tb);
     s->cb = reinterpret_cast<int*>(cb);
     s->cstart = reinterpret_cast<int*>(cstart);
+    s->ncoll = reinterpret_cast<int*>(ncoll);
     s->misc = reinterpret_cast<int*>(misc);
     s->prop = reinterpret_cast<int8_t*>(prop);
     s->assign = reinterpret_cast<int16_t*>(assign);
@@ -146,6 +149,26 @@ __device__ __forceinline__ void load8(const SealArgs& a, int64_t row, int e0, do
   }
 }
 
+// Two consecutive key elements [e, e + 2) as float64 (e even).
+__device__ __forceinline__ void load2(const SealArgs& a, int64_t row, int e, double* x) {
+  if (a.key_dtype == KD_BF16) {
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(
+        reinterpret_cast<const uint16_t*>(a.keys) + row * a.d + e));
+    x[0] = __uint_as_float(v << 16);
+    x[1] = __uint_as_float(v & 0xFFFF0000u);
+  } else if (a.key_dtype == KD_FP8) {
+    const uint16_t v = __ldg(reinterpret_cast<const uint16_t*>(
+        reinterpret_cast<const uint8_t*>(a.keys) + row * a.d + e));
+    const double sc = static_cast<double>(a.key_scale[row]);
+    x[0] = static_cast<double>(fp8_to_f32(static_cast<uint8_t>(v & 0xFF))) * sc;
+    x[1] = static_cast<double>(fp8_to_f32(static_cast<uint8_t>(v >> 8))) * sc;
+  } else {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(reinterpret_cast<const float*>(a.keys) + row * a.d + e));
+    x[0] = v.x;
+    x[1] = v.y;
+  }
+}
+
 // Pair order (distance, key, cluster): is (d1, i1, j1) <= (d2, i2, j2)?
 __device__ __forceinline__ bool pair_le(uint64_t d1, uint32_t i1, uint32_t j1, uint64_t d2,
                                         uint32_t i2, uint32_t j2) {
@@ -165,7 +188,7 @@ __device__ __forceinline__ int dist_bin(const SealSmem& s, int j, double v) {
 
 // D[j, i] for all keys of the window, two key rows per thread, the centre
 // values read as pairs (the summation order per (i, j) is dimension order).
-template <int MM>
+template <int MM, bool kBf16>
 __device__ __forceinline__ void seal_dist(const SealArgs& a, const SealSmem& s, int64_t lo) {
   const int W = a.W, m = a.m, d = a.d;
   for (int i0 = 2 * threadIdx.x; i0 < W; i0 += 2 * blockDim.x) {
@@ -179,12 +202,28 @@ __device__ __forceinline__ void seal_dist(const SealArgs& a, const SealSmem& s, 
     }
     for (int e0 = 0; e0 < d; e0 += 8) {
       double x0[8], x1[8];
-      load8(a, lo + i0, e0, x0);
-      if (two) {
-        load8(a, lo + i0 + 1, e0, x1);
-      } else {
+      if (kBf16) {
+        // both rows' 16-byte loads issued before any use
+        const uint4* kp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.keys) +
+                                                         (lo + i0) * d + e0);
+        const uint4 v0 = __ldg(kp);
+        const uint4 v1 = two ? __ldg(kp + d / 8) : make_uint4(0, 0, 0, 0);
+        const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x1[u] = 0.0;
+        for (int u = 0; u < 4; ++u) {
+          x0[2 * u] = __uint_as_float(w0[u] << 16);
+          x0[2 * u + 1] = __uint_as_float(w0[u] & 0xFFFF0000u);
+          x1[2 * u] = __uint_as_float(w1[u] << 16);
+          x1[2 * u + 1] = __uint_as_float(w1[u] & 0xFFFF0000u);
+        }
+      } else {
+        load8(a, lo + i0, e0, x0);
+        if (two) {
+          load8(a, lo + i0 + 1, e0, x1);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x1[u] = 0.0;
+        }
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -259,6 +298,8 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
     s.cent[e] = key_f64(a, lo + ((2 * j + 1) * W) / (2 * m), i);
   }
   for (int i = tid; i < W; i += blockDim.x) s.prev[i] = -1;
+  // the histograms start at zero; the scan that reads a row clears it
+  for (int e = tid; e < m * kBins; e += blockDim.x) s.hist[e] = 0;
   __syncthreads();
 
   for (int it = 0; it < a.iters; ++it) {
@@ -270,8 +311,8 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       if (lane == 0) s.cc[j] = cc;
     }
     __syncthreads();
-    if (m <= 8) seal_dist<8>(a, s, lo);
-    else if (m <= 16) seal_dist<16>(a, s, lo);
+    if (m <= 8 && a.key_dtype == KD_BF16) seal_dist<8, true>(a, s, lo);
+    else if (m <= 8) seal_dist<8, false>(a, s, lo);
     else seal_dist_any(a, s, lo);
     for (int i = tid; i < W; i += blockDim.x) s.assign[i] = -1;
     for (int j = tid; j < m; j += blockDim.x) s.cnt[j] = 0;
@@ -302,14 +343,6 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
     // greedy capacity assignment in rounds (see the file comment)
     for (int round = 0; round <= m && s.misc[2] > 0; ++round) {
       const unsigned long long fullm = *s.fullmask;
-      // A. clear the histograms and the fill pairs
-      for (int e = tid; e < m * kBins; e += blockDim.x) s.hist[e] = 0;
-      for (int j = tid; j < m; j += blockDim.x) {
-        s.fk1[j] = ~0ull;
-        s.fk2[j] = ~0u;
-      }
-      if (tid == 0) s.misc[1] = 0;
-      __syncthreads();
       // B. proposals: best open cluster of every free key, counted per bin
       for (int i = tid; i < W; i += blockDim.x) {
         int bj = -1;
@@ -329,74 +362,118 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       }
       __syncthreads();
       // C. per open cluster, the bin where the running count reaches the
-      //    (cap - count)-th proposal (none if the cluster cannot fill now)
+      //    (cap - count)-th proposal (none if the cluster cannot fill now):
+      //    32-bin chunk sums, a scan over the chunks, a scan inside the one
+      //    chunk.  The row is cleared for the next round as it is read.
       for (int j = warp; j < m; j += nwarps) {
         int found = -1, before = 0;
         if (!((fullm >> j) & 1ull)) {
           const int need = a.cap - s.cnt[j];
-          int run = 0;
-          for (int b0 = 0; b0 < kBins; b0 += 32) {
-            const int v = s.hist[j * kBins + b0 + lane];
+          int* hj = s.hist + j * kBins;
+          int csum = 0;
+#pragma unroll 8
+          for (int c = 0; c < 32; ++c) {
+            const int t = __reduce_add_sync(0xffffffffu, hj[c * 32 + lane]);
+            if (lane == c) csum = t;
+          }
+          int cin = csum;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, cin, o);
+            if (lane >= o) cin += t;
+          }
+          const unsigned cb = __ballot_sync(0xffffffffu, cin >= need);
+          if (cb) {
+            const int c = __ffs(cb) - 1;
+            const int base = __shfl_sync(0xffffffffu, cin - csum, c);
+            const int v = hj[c * 32 + lane];
             int incl = v;
             for (int o = 1; o < 32; o <<= 1) {
               const int t = __shfl_up_sync(0xffffffffu, incl, o);
               if (lane >= o) incl += t;
             }
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (run + tot >= need) {
-              const unsigned bal = __ballot_sync(0xffffffffu, run + incl >= need);
-              const int first = __ffs(bal) - 1;
-              const int excl = __shfl_sync(0xffffffffu, incl - v, first);
-              found = b0 + first;
-              before = run + excl;
-              break;
-            }
-            run += tot;
+            const unsigned bb = __ballot_sync(0xffffffffu, base + incl >= need);
+            const int first = __ffs(bb) - 1;
+            found = c * 32 + first;
+            before = base + __shfl_sync(0xffffffffu, incl - v, first);
           }
+          __syncwarp();
+          for (int c = 0; c < 32; ++c) hj[c * 32 + lane] = 0;
         }
         if (lane == 0) {
           s.tb[j] = found;
           s.cb[j] = before;
+          s.ncoll[j] = 0;
+          s.fk1[j] = ~0ull;
+          s.fk2[j] = ~0u;
         }
       }
       __syncthreads();
-      // D. collect the proposals lying in their cluster's target bin
+      // D. collect, per cluster, the proposals lying in its target bin
       for (int i = tid; i < W; i += blockDim.x) {
         const int j = s.prop[i];
         if (j >= 0 && s.tb[j] >= 0 && dist_bin(s, j, s.D[j * W + i]) == s.tb[j])
-          s.coll[atomicAdd(&s.misc[1], 1)] = static_cast<int16_t>(i);
+          s.coll[j * W + atomicAdd(&s.ncoll[j], 1)] = static_cast<int16_t>(i);
       }
       __syncthreads();
-      // E. exact rank (distance bits, key) inside the target bin
-      const int nc = s.misc[1];
-      for (int e = tid; e < nc; e += blockDim.x) {
-        const int i = s.coll[e];
-        const int j = s.prop[i];
-        const uint64_t di = dbits(s.D[j * W + i]);
-        int r = 0;
-        for (int x = 0; x < nc; ++x) {
-          const int k2 = s.coll[x];
-          if (s.prop[k2] != j) continue;
-          const uint64_t dk = dbits(s.D[j * W + k2]);
-          r += (dk < di || (dk == di && k2 < i)) ? 1 : 0;
-        }
-        if (r == a.cap - s.cnt[j] - s.cb[j] - 1) {
-          s.fk1[j] = di;
-          s.fk2[j] = (static_cast<uint32_t>(i) << 16) | static_cast<uint32_t>(j);
+      // E. exact rank (distance bits, key) inside the target bin, one warp
+      //    per cluster: lanes hold entries, the others stream by shuffles
+      for (int j = warp; j < m; j += nwarps) {
+        const int nc = s.ncoll[j];
+        if (s.tb[j] < 0 || nc == 0) continue;
+        const int want = a.cap - s.cnt[j] - s.cb[j] - 1;
+        const int16_t* cj = s.coll + j * W;
+        for (int e0 = 0; e0 < nc; e0 += 32) {
+          const int e = e0 + lane;
+          const int i = e < nc ? cj[e] : 0;
+          const uint64_t di = e < nc ? dbits(s.D[j * W + i]) : ~0ull;
+          int r = 0;
+          for (int x0 = 0; x0 < nc; x0 += 32) {
+            const int xi = x0 + lane < nc ? cj[x0 + lane] : 0;
+            const uint64_t xd = x0 + lane < nc ? dbits(s.D[j * W + xi]) : ~0ull;
+            const int nx = min(32, nc - x0);
+            for (int t = 0; t < nx; ++t) {
+              const uint64_t dk = __shfl_sync(0xffffffffu, xd, t);
+              const int k2 = __shfl_sync(0xffffffffu, xi, t);
+              r += (dk < di || (dk == di && k2 < i)) ? 1 : 0;
+            }
+          }
+          if (e < nc && r == want) {
+            s.fk1[j] = di;
+            s.fk2[j] = (static_cast<uint32_t>(i) << 16) | static_cast<uint32_t>(j);
+          }
         }
       }
       __syncthreads();
-      // F. the cluster that fills first closes this round
-      if (tid == 0) {
-        int best = -1;
-        for (int j = 0; j < m; ++j) {
+      // F. the cluster that fills first closes this round (warp 0: lanes
+      //    hold the fill pairs, an argmin in pair order)
+      if (warp == 0) {
+        uint64_t bd = ~0ull;
+        uint32_t bk = ~0u;
+        int bj = -1;
+        for (int j = lane; j < m; j += 32) {
           if (s.fk2[j] == ~0u) continue;
-          if (best < 0 || pair_le(s.fk1[j], s.fk2[j] >> 16, j, s.fk1[best], s.fk2[best] >> 16,
-                                  static_cast<uint32_t>(best)))
-            best = j;
+          const uint64_t d1 = s.fk1[j];
+          const uint32_t k1 = s.fk2[j] >> 16;
+          if (bj < 0 || pair_le(d1, k1, j, bd, bk, bj)) {
+            bd = d1;
+            bk = k1;
+            bj = j;
+          }
         }
-        s.misc[0] = best;
-        if (best >= 0) *s.fullmask |= 1ull << best;
+        for (int o = 16; o > 0; o >>= 1) {
+          const uint64_t od = __shfl_xor_sync(0xffffffffu, bd, o);
+          const uint32_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+          if (oj >= 0 && (bj < 0 || pair_le(od, ok, oj, bd, bk, bj))) {
+            bd = od;
+            bk = ok;
+            bj = oj;
+          }
+        }
+        if (lane == 0) {
+          s.misc[0] = bj;
+          if (bj >= 0) *s.fullmask |= 1ull << bj;
+        }
       }
       __syncthreads();
       // G. commit every proposal up to the filling pair (all if none)
@@ -441,27 +518,50 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       }
     }
     __syncthreads();
-    // update: float64 mean of the members in ascending key order; the
-    // (cluster, 32-dim block) pairs are spread over all warps, 16 member
-    // rows in flight per lane (added in member order)
+    // update: float64 mean of the members in ascending key order.  A warp
+    // takes (cluster, 64-dim block): each lane sums two dimensions over the
+    // members in order, 16 member rows in flight.
     {
-      const int nblk = (d + 31) / 32;
+      const int nblk = (d + 63) / 64;
       for (int wj = warp; wj < m * nblk; wj += nwarps) {
         const int j = wj / nblk;
-        const int e = (wj % nblk) * 32 + lane;
+        const int e = (wj % nblk) * 64 + 2 * lane;
         const int b0 = s.cstart[j], b1 = s.cstart[j + 1];
         if (b1 == b0 || e >= d) continue;
-        double sum = 0.0;
+        double s0 = 0.0, s1 = 0.0;
         int q = b0;
-        for (; q + 16 <= b1; q += 16) {
-          double v[16];
+        if (a.key_dtype == KD_BF16) {
+          // raw bf16 pairs: the loads of a batch are issued back to back
+          const uint32_t* kp = reinterpret_cast<const uint32_t*>(a.keys) + (lo * d + e) / 2;
+          for (; q + 16 <= b1; q += 16) {
+            uint32_t r[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = key_f64(a, lo + s.mlist[q + u], e);
+            for (int u = 0; u < 16; ++u) r[u] = __ldg(kp + static_cast<int64_t>(s.mlist[q + u]) * (d / 2));
 #pragma unroll
-          for (int u = 0; u < 16; ++u) sum += v[u];
+            for (int u = 0; u < 16; ++u) {
+              s0 += static_cast<double>(__uint_as_float(r[u] << 16));
+              s1 += static_cast<double>(__uint_as_float(r[u] & 0xFFFF0000u));
+            }
+          }
         }
-        for (; q < b1; ++q) sum += key_f64(a, lo + s.mlist[q], e);
-        s.cent[j * d + e] = sum / static_cast<double>(b1 - b0);
+        for (; q + 16 <= b1; q += 16) {
+          double v[16][2];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) load2(a, lo + s.mlist[q + u], e, v[u]);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            s0 += v[u][0];
+            s1 += v[u][1];
+          }
+        }
+        for (; q < b1; ++q) {
+          double v[2];
+          load2(a, lo + s.mlist[q], e, v);
+          s0 += v[0];
+          s1 += v[1];
+        }
+        s.cent[j * d + e] = s0 / static_cast<double>(b1 - b0);
+        s.cent[j * d + e + 1] = s1 / static_cast<double>(b1 - b0);
       }
     }
     if (tid == 0) s.misc[3] = 0;
