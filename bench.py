@@ -360,22 +360,52 @@ def run_ours(args):
             host.append((a, kd_.cpu().pin_memory(), ks_.cpu().pin_memory() if ks_ is not None else None,
                          qd_.cpu().pin_memory(), wd_.cpu().pin_memory(),
                          torch.empty((T, wl.k), dtype=torch.int32).pin_memory()))
-        kd2, qd2, wd2 = torch.empty_like(kd), torch.empty_like(qd), torch.empty_like(wd)
-        sd2 = torch.empty_like(ks) if ks is not None else None
-        out2 = torch.empty_like(out)
+        # Two device input/output sets; host-to-device copies of chunk c+1
+        # and the device-to-host copy of chunk c's result run on copy streams
+        # while chunk c is processed (every copy stays inside the timed region).
+        bufs = [(torch.empty_like(kd), torch.empty_like(ks) if ks is not None else None,
+                 torch.empty_like(qd), torch.empty_like(wd), torch.empty_like(out)) for _ in range(2)]
+        h2d_s = torch.cuda.Stream(device=dev)
+        d2h_s = torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def load(c):
+            _, kh, sh, qh, wh, _ = host[c]
+            kb, sb, qb, wb, _ = bufs[c % 2]
+            with torch.cuda.stream(h2d_s):
+                if c >= 2:
+                    h2d_s.wait_event(ev_done[c % 2])  # chunk c-2 no longer reads the set
+                kb.copy_(kh, non_blocking=True)
+                if sh is not None:
+                    sb.copy_(sh, non_blocking=True)
+                qb.copy_(qh, non_blocking=True)
+                wb.copy_(wh, non_blocking=True)
+                ev_in[c % 2].record(h2d_s)
 
         def e2e_step():
-            for a, kh, sh, qh, wh, oh in host:
-                kd2.copy_(kh, non_blocking=True)
-                if sh is not None:
-                    sd2.copy_(sh, non_blocking=True)
-                qd2.copy_(qh, non_blocking=True)
-                wd2.copy_(wh, non_blocking=True)
-                idx.append_keys(kd2, sd2)
+            n = len(host)
+            h2d_s.wait_stream(stream)  # after the work already queued (and the start event)
+            load(0)
+            for c in range(n):
+                a = host[c][0]
+                kb, sb, qb, wb, ob = bufs[c % 2]
+                stream.wait_event(ev_in[c % 2])
+                if c >= 2:
+                    stream.wait_event(ev_out[c % 2])  # chunk c-2's result has left
+                idx.append_keys(kb, sb)
                 idx.seal()
-                idx.route_refine(qd2, wd2, a, wl.k, wl.budget, out=out2)
-                oh.copy_(out2, non_blocking=True)
+                idx.route_refine(qb, wb, a, wl.k, wl.budget, out=ob)
+                ev_done[c % 2].record(stream)
+                if c + 1 < n:
+                    load(c + 1)
+                with torch.cuda.stream(d2h_s):
+                    d2h_s.wait_event(ev_done[c % 2])
+                    host[c][5].copy_(ob, non_blocking=True)
+                    ev_out[c % 2].record(d2h_s)
             idx.publish()
+            stream.wait_event(ev_out[(n - 1) % 2])
 
         for _ in range(max(1, args.warmup)):
             idx.rollback()
