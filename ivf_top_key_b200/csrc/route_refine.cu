@@ -87,7 +87,7 @@ struct P1Smem {
 // Warp 0 scans the weighted histogram ps.hist from the top for the bin
 // where the weight reaches `need`: its index and the weight above it.
 // All threads call it (it ends with a barrier).
-__device__ void p1_find_bin(P1Smem& ps, int need, int* bstar, int* above) {
+__device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, int* above) {
   const int lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {
     uint32_t lsum = 0;
@@ -182,14 +182,14 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   const float scale = vmax > vmin ? static_cast<float>(kNB1) / (vmax - vmin) : 0.f;
   // bin positions use explicitly rounded operations (no FMA contraction), so
   // every pass computes the same bin for the same score
-  auto pos1 = [&](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
-  auto binof = [&](float v) -> int {
+  auto pos1 = [=](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
+  auto binof = [=](float v) -> int {
     const int b = static_cast<int>(pos1(v));
     return b < kNB1 - 1 ? b : kNB1 - 1;
   };
   int bstar = 0, bstar2 = 0;
-  auto bin2 = [&](float v) -> int {
-    const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), static_cast<float>(bstar)),
+  auto bin2 = [=](float v, int b1) -> int {
+    const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), static_cast<float>(b1)),
                                              static_cast<float>(kNB1)));
     return b < 0 ? 0 : (b < kNB1 - 1 ? b : kNB1 - 1);
   };
@@ -227,17 +227,17 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (sz[u] > 0 && binof(v[u]) == bstar) atomicAdd(&ps.hist[bin2(v[u])], static_cast<uint32_t>(sz[u]));
+        if (sz[u] > 0 && binof(v[u]) == bstar) atomicAdd(&ps.hist[bin2(v[u], bstar)], static_cast<uint32_t>(sz[u]));
     }
     __syncthreads();
     int above2 = 0;
     p1_find_bin(ps, rem - above1, &bstar2, &above2);
   }
-  auto selected = [&](float v) -> bool {
+  auto selected = [=](float v) -> bool {
     if (take_all) return true;
     const int b = binof(v);
     if (b != bstar) return b > bstar;
-    return bin2(v) >= bstar2;
+    return bin2(v, bstar) >= bstar2;
   };
   // pass C: clusters at or above the boundary bin (any order: sorted next)
   if (tid == 0) ps.scal[1] = 0;
@@ -267,16 +267,32 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     if (tid == 0) atomicOr(a.err, DEV_ERR_CAPACITY);
     nsel = kSortCap;
   }
-  int np = 1;
-  while (np < nsel) np <<= 1;
-  for (int i = nsel + tid; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
-  __syncthreads();
-  bitonic_sort_u64(sortbuf, np);
+  // rank order (score descending, then cluster id): small selections by
+  // counting (keys are distinct, so ranks are a permutation), larger ones
+  // by a bitonic sort in place
+  const uint64_t* sorted = sortbuf;
+  if (nsel <= kSortCap / 4) {
+    uint64_t* dst = sortbuf + kSortCap / 2;
+    for (int i = tid; i < nsel; i += blockDim.x) {
+      const uint64_t x = sortbuf[i];
+      int r = 0;
+      for (int j = 0; j < nsel; ++j) r += sortbuf[j] < x ? 1 : 0;
+      dst[r] = x;
+    }
+    __syncthreads();
+    sorted = dst;
+  } else {
+    int np = 1;
+    while (np < nsel) np <<= 1;
+    for (int i = nsel + tid; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
+    __syncthreads();
+    bitonic_sort_u64(sortbuf, np);
+  }
   // member offsets and sizes of the ranked clusters (parallel loads), then
   // the exclusive prefix of sizes in rank order
   int32_t* coff = ps.coff;
   for (int r = tid; r < nsel; r += blockDim.x) {
-    const int c = static_cast<int>(sortbuf[r] & 0xffffffffu);
+    const int c = static_cast<int>(sorted[r] & 0xffffffffu);
     const int o0 = off[c];
     coff[r] = o0;
     pref[r] = off[c + 1] - o0;
@@ -300,32 +316,16 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   }
   __syncthreads();
   const int len = static_cast<int>(min64(C, static_cast<int64_t>(fixed) + pref[nsel]));
-  // flat fill: slot -> rank r (binary search over pref) -> member; four
-  // independent loads in flight per thread
-  for (int s0 = fixed + tid; s0 < len; s0 += 4 * blockDim.x) {
-    int src[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int slot = s0 + u * blockDim.x;
-      src[u] = -1;
-      if (slot < len) {
-        const int x = slot - fixed;
-        int lo = 0, hi = nsel - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (pref[mid] <= x) lo = mid;
-          else hi = mid - 1;
-        }
-        src[u] = coff[lo] + (x - pref[lo]);
-      }
-    }
-    int32_t mv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) mv[u] = src[u] >= 0 ? __ldg(a.members + src[u]) : 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (src[u] >= 0) cand[s0 + u * blockDim.x] = mv[u];
+  // fill: one warp per ranked cluster copies its member run into the list
+  // with 4-byte asynchronous copies (all in flight at once), cut at C
+  for (int r = warp; r < nsel; r += nwarps) {
+    const int d0 = fixed + pref[r];
+    if (d0 >= len) continue;
+    const int sz = min(pref[r + 1] - pref[r], len - d0);
+    const int32_t* src = a.members + coff[r];
+    for (int l = lane; l < sz; l += 32) cp_async4(cand + d0 + l, src + l);
   }
+  cp_async_wait_all();
   __syncthreads();
   return len;
 }
@@ -510,6 +510,24 @@ __device__ __forceinline__ void p3_for_each(const P3Ctx& c, F f) {
   }
 }
 
+// Every item of the thread's columns (16 at a time), with its validity as
+// an int: bodies fold it into branch-free arithmetic (a data-dependent
+// branch per item costs far more than the arithmetic).
+template <class F>
+__device__ __forceinline__ void p3_for_each_all(const P3Ctx& c, F f) {
+  for (int c0 = 0; c0 < c.ntiles; c0 += 16) {
+    float v[16];
+    tmem_ld16(c.tcol + c0, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int j = c0 + u;
+      const int slot = j * 128 + c.row;
+      f(v[u], slot, static_cast<int>(j < c.ntiles) & static_cast<int>(slot < c.n));
+    }
+  }
+}
+
 // Exclusive prefix over the 128 epilogue threads (et = 0..127).
 __device__ __forceinline__ int p3_scan(int v, int et, int* total, P3Smem& ps) {
   const int lane = et & 31, w = et >> 5;
@@ -534,14 +552,14 @@ __device__ __forceinline__ int p3_scan(int v, int et, int* total, P3Smem& ps) {
 // Radix select over the items passing pred: the value of key(v, slot) of
 // the need-th largest item, and how many items lie strictly above it.
 template <class Pred, class Key>
-__device__ uint32_t p3_radix(const P3Ctx& c, int et, Pred pred, Key key, int need, int* above,
+__device__ __forceinline__ uint32_t p3_radix(const P3Ctx& c, int et, Pred pred, Key key, int need, int* above,
                              int* eq, P3Smem& ps) {
   uint32_t prefix = 0, mask = 0;
   int needr = need, ab = 0, last = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = et; i < 256; i += 128) ps.hist[i] = 0;
     named_bar(1, 128);
-    p3_for_each(c, [&](float v, int slot) {
+    p3_for_each(c, [&, pred, key](float v, int slot) {
       if (!pred(v, slot)) return;
       const uint32_t kk = key(v, slot);
       if ((kk & mask) == prefix) atomicAdd(&ps.hist[(kk >> shift) & 255u], 1u);
@@ -578,7 +596,7 @@ __device__ uint32_t p3_radix(const P3Ctx& c, int et, Pred pred, Key key, int nee
 // The bin of ps.hist (kNB bins, scanned from the top) holding the k-th
 // item: its index, the count above it, and its own count.  All 128
 // epilogue threads call it; thread et owns bins [16 et, 16 et + 16).
-__device__ void p3_find_bin(P3Smem& ps, int et, int k, int* bstar, int* above, int* nb) {
+__device__ __forceinline__ void p3_find_bin(P3Smem& ps, int et, int k, int* bstar, int* above, int* nb) {
   int tsum = 0;
   for (int b = 0; b < 16; ++b) tsum += static_cast<int>(ps.hist[16 * et + b]);
   int tot;
@@ -630,8 +648,8 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
     const float scale = vmax > vmin ? static_cast<float>(kNB) / (vmax - vmin) : 0.f;
     // explicitly rounded (never contracted): the same score always lands in
     // the same bin in every pass
-    auto pos1 = [&](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
-    auto binof = [&](float v) -> int {
+    auto pos1 = [=](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
+    auto binof = [=](float v) -> int {
       const int b = static_cast<int>(pos1(v));
       return b < kNB - 1 ? b : kNB - 1;
     };
@@ -641,30 +659,30 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
     for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
     if (et == 0) ps.cnt = 0;
     named_bar(1, 128);
-    p3_for_each(c, [&](float v, int) { atomicAdd(&ps.hist[binof(v)], 1u); });
+    p3_for_each(c, [&ps, binof](float v, int) { atomicAdd(&ps.hist[binof(v)], 1u); });
     named_bar(1, 128);
     int above_b = 0, bstar = 0, nb = 0;
     p3_find_bin(ps, et, k, &bstar, &above_b, &nb);
     const float b1f = static_cast<float>(bstar);
-    auto bin2 = [&](float v) -> int {
+    auto bin2 = [=](float v) -> int {
       const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), b1f), static_cast<float>(kNB)));
       return b < 0 ? 0 : (b < kNB - 1 ? b : kNB - 1);
     };
     for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
     named_bar(1, 128);
-    p3_for_each(c, [&](float v, int) {
+    p3_for_each(c, [&ps, binof, bin2, bstar](float v, int) {
       if (binof(v) == bstar) atomicAdd(&ps.hist[bin2(v)], 1u);
     });
     named_bar(1, 128);
     int bstar2 = 0, above2 = 0, nb2 = 0;
     p3_find_bin(ps, et, k - above_b, &bstar2, &above2, &nb2);
     above_b += above2;
-    auto in_b = [&](float v) -> bool { return binof(v) == bstar && bin2(v) == bstar2; };
+    auto in_b = [=](float v) -> bool { return binof(v) == bstar && bin2(v) == bstar2; };
     const int need = k - above_b;
     int above_in = 0, eq = 0;
     uint32_t tkey;
     if (nb2 <= kCapB) {
-      p3_for_each(c, [&](float v, int slot) {
+      p3_for_each(c, [&ps, in_b](float v, int slot) {
         if (in_b(v)) {
           const unsigned long long pos = atomicAdd(&ps.cnt, 1ull);
           ps.buf[pos] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(slot);
@@ -704,7 +722,7 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       eq = ps.scal[7];
     } else {
       tkey = p3_radix(
-          c, et, [&](float v, int) { return in_b(v); }, [&](float v, int) { return f2key(v); }, need,
+          c, et, [=](float v, int) { return in_b(v); }, [](float v, int) { return f2key(v); }, need,
           &above_in, &eq, ps);
     }
     theta = key2f(tkey);
@@ -713,32 +731,56 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       ties_all = false;
       int ab2 = 0, eq2 = 0;
       const uint32_t idk = p3_radix(
-          c, et, [&](float v, int) { return v == theta; },
-          [&](float, int slot) { return ~static_cast<uint32_t>(c.cand[slot]); }, need_eq, &ab2, &eq2,
+          c, et, [=](float v, int) { return v == theta; },
+          [cd = c.cand](float, int slot) { return ~static_cast<uint32_t>(cd[slot]); }, need_eq, &ab2, &eq2,
           ps);
       theta_id = static_cast<int>(~idk);
     }
   }
   // emission: ids staged in shared memory in thread-major order, then
-  // written out coalesced (deterministic order)
-  auto sel = [&](float v, int slot) {
-    return take_all || v > theta || (v == theta && (ties_all || c.cand[slot] <= theta_id));
-  };
+  // written out coalesced (deterministic order).  Selection is v >= theta
+  // (everything when all items are kept), except when only some of the
+  // items tied at theta are kept: then v > theta or (v == theta and id <=
+  // theta_id).  Bodies are branch-free; unselected items write to a
+  // per-thread dummy slot.
+  const bool partial_ties = !take_all && !ties_all;
+  const float th = take_all ? -INFINITY : theta;
+  const int thid = theta_id;
+  const int32_t* cd = c.cand;
+  const int nlast = c.n - 1;  // slots past the list read entry 0 instead (their result is unused)
   int mine = 0;
-  p3_for_each(c, [&](float v, int slot) { mine += sel(v, slot) ? 1 : 0; });
+  if (!partial_ties) {
+    p3_for_each_all(c, [&mine, th](float v, int, int ok) { mine += ok & static_cast<int>(v >= th); });
+  } else {
+    p3_for_each_all(c, [&mine, th, thid, cd, nlast](float v, int slot, int ok) {
+      const int sl = slot <= nlast ? slot : 0;
+      mine += ok & (static_cast<int>(v > th) | (static_cast<int>(v == th) & static_cast<int>(cd[sl] <= thid)));
+    });
+  }
   int total;
   int pos = p3_scan(mine, et, &total, ps);
   int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] ids
   float* ssc = reinterpret_cast<float*>(ps.buf) + kCapB;       // [k] scores
-  p3_for_each(c, [&](float v, int slot) {
-    if (sel(v, slot)) {
-      if (pos < k) {
-        sid[pos] = c.cand[slot];
-        ssc[pos] = v;
-      }
-      ++pos;
-    }
-  });
+  int32_t* dump_id = reinterpret_cast<int32_t*>(ps.hist) + et;
+  float* dump_sc = reinterpret_cast<float*>(ps.hist) + 128 + et;
+  auto stage = [&pos, sid, ssc, dump_id, dump_sc, k, cd, nlast](float v, int slot, int f) {
+    const bool w = (f & static_cast<int>(pos < k)) != 0;
+    int32_t* pi = w ? sid + pos : dump_id;
+    float* pv = w ? ssc + pos : dump_sc;
+    *pi = cd[slot <= nlast ? slot : 0];
+    *pv = v;
+    pos += f;
+  };
+  if (!partial_ties) {
+    p3_for_each_all(c, [stage, th](float v, int slot, int ok) mutable {
+      stage(v, slot, ok & static_cast<int>(v >= th));
+    });
+  } else {
+    p3_for_each_all(c, [stage, th, thid, cd, nlast](float v, int slot, int ok) mutable {
+      const int sl = slot <= nlast ? slot : 0;
+      stage(v, slot, ok & (static_cast<int>(v > th) | (static_cast<int>(v == th) & static_cast<int>(cd[sl] <= thid))));
+    });
+  }
   named_bar(1, 128);
   const int nw = min(total, k);
   for (int j = et; j < k; j += 128) {
