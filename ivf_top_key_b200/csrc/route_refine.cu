@@ -651,7 +651,7 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
     auto pos1 = [=](float v) -> float { return __fmul_rn(__fsub_rn(v, vmin), scale); };
     auto binof = [=](float v) -> int {
       const int b = static_cast<int>(pos1(v));
-      return b < kNB - 1 ? b : kNB - 1;
+      return b < 0 ? 0 : (b < kNB - 1 ? b : kNB - 1);
     };
     // level 1 over [vmin, vmax]; level 2 splits the level-1 bin that holds
     // the k-th score into kNB sub-bins (a long score tail leaves the bulk
@@ -659,7 +659,10 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
     for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
     if (et == 0) ps.cnt = 0;
     named_bar(1, 128);
-    p3_for_each(c, [&ps, binof](float v, int) { atomicAdd(&ps.hist[binof(v)], 1u); });
+    // (an add of 0 for slots past the list keeps the body branch-free)
+    p3_for_each_all(c, [&ps, binof](float v, int, int ok) {
+      atomicAdd(&ps.hist[binof(v)], static_cast<uint32_t>(ok));
+    });
     named_bar(1, 128);
     int above_b = 0, bstar = 0, nb = 0;
     p3_find_bin(ps, et, k, &bstar, &above_b, &nb);
@@ -668,30 +671,70 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       const int b = static_cast<int>(__fmul_rn(__fsub_rn(pos1(v), b1f), static_cast<float>(kNB)));
       return b < 0 ? 0 : (b < kNB - 1 ? b : kNB - 1);
     };
-    for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
-    named_bar(1, 128);
-    p3_for_each(c, [&ps, binof, bin2, bstar](float v, int) {
-      if (binof(v) == bstar) atomicAdd(&ps.hist[bin2(v)], 1u);
-    });
-    named_bar(1, 128);
-    int bstar2 = 0, above2 = 0, nb2 = 0;
-    p3_find_bin(ps, et, k - above_b, &bstar2, &above2, &nb2);
-    above_b += above2;
-    auto in_b = [=](float v) -> bool { return binof(v) == bstar && bin2(v) == bstar2; };
-    const int need = k - above_b;
-    int above_in = 0, eq = 0;
-    uint32_t tkey;
-    if (nb2 <= kCapB) {
-      p3_for_each(c, [&ps, in_b](float v, int slot) {
-        if (in_b(v)) {
-          const unsigned long long pos = atomicAdd(&ps.cnt, 1ull);
-          ps.buf[pos] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(slot);
+    // The items of the threshold bin (bin bstar, or its sub-bin bstar2 when
+    // the bin is too full) are gathered and sorted; the k-th score is
+    // read off the sorted list.
+    int bsel2 = -1, nsel = nb, above_in = 0, eq = 0;
+    if (nb > kCapB) {
+      // level 2: the bin split into kNB sub-bins
+      for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
+      named_bar(1, 128);
+      // few items per warp fall in the bin: a warp-uniform test skips the rest
+      p3_for_each_all(c, [&ps, binof, bin2, bstar](float v, int, int ok) {
+        const int f = ok & static_cast<int>(binof(v) == bstar);
+        if (__any_sync(0xffffffffu, f)) {
+          if (f) atomicAdd(&ps.hist[bin2(v)], 1u);
         }
       });
       named_bar(1, 128);
+      int above2 = 0;
+      p3_find_bin(ps, et, k - above_b, &bsel2, &above2, &nsel);
+      above_b += above2;
+    }
+    auto in_b = [=](float v) -> bool { return binof(v) == bstar && (bsel2 < 0 || bin2(v) == bsel2); };
+    const int need = k - above_b;
+    uint32_t tkey;
+    if (nsel <= kCapB) {
+      // append of the items of the threshold (sub-)bin: flags for 16 items
+      // at a time without branches, then a warp-uniform test; the rare hits
+      // are appended warp-aggregated
+      for (int c0 = 0; c0 < c.ntiles; c0 += 16) {
+        float v[16];
+        tmem_ld16(c.tcol + c0, v);
+        tmem_ld_wait();
+        uint32_t m = 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = c0 + u;
+          const int slot = j * 128 + c.row;
+          const int f = static_cast<int>(j < c.ntiles) & static_cast<int>(slot < c.n) &
+                        static_cast<int>(binof(v[u]) == bstar) &
+                        (static_cast<int>(bsel2 < 0) | static_cast<int>(bin2(v[u]) == bsel2));
+          m |= static_cast<uint32_t>(f) << u;
+        }
+        if (__any_sync(0xffffffffu, m != 0u)) {
+          const int lane = threadIdx.x & 31;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int f = static_cast<int>((m >> u) & 1u);
+            const unsigned bal = __ballot_sync(0xffffffffu, f);
+            if (bal) {
+              const int lead = __ffs(bal) - 1;
+              unsigned long long base = 0;
+              if (lane == lead) base = atomicAdd(&ps.cnt, static_cast<unsigned long long>(__popc(bal)));
+              base = __shfl_sync(0xffffffffu, base, lead);
+              if (f)
+                ps.buf[base + __popc(bal & ((1u << lane) - 1u))] =
+                    (static_cast<uint64_t>(~f2key(v[u])) << 32) |
+                    static_cast<uint32_t>((c0 + u) * 128 + c.row);
+            }
+          }
+        }
+      }
+      named_bar(1, 128);
       int np = 1;
-      while (np < nb2) np <<= 1;
-      for (int i = nb2 + et; i < np; i += 128) ps.buf[i] = ~0ull;
+      while (np < nsel) np <<= 1;
+      for (int i = nsel + et; i < np; i += 128) ps.buf[i] = ~0ull;
       named_bar(1, 128);
       for (int kk = 2; kk <= np; kk <<= 1) {
         for (int j = kk >> 1; j > 0; j >>= 1) {
@@ -713,7 +756,7 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
         int i0 = need - 1;
         while (i0 > 0 && ~static_cast<uint32_t>(ps.buf[i0 - 1] >> 32) == tkey) --i0;
         int i1 = need - 1;
-        while (i1 + 1 < nb2 && ~static_cast<uint32_t>(ps.buf[i1 + 1] >> 32) == tkey) ++i1;
+        while (i1 + 1 < nsel && ~static_cast<uint32_t>(ps.buf[i1 + 1] >> 32) == tkey) ++i1;
         ps.scal[6] = i0;
         ps.scal[7] = i1 - i0 + 1;
       }
