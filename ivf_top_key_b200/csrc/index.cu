@@ -376,13 +376,16 @@ int publish(ai_index* h) {
   return AI_OK;
 }
 
-int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window) {
+// Refit over the keys of the first `windows_r` sealed windows (all sealed
+// windows when negative).  Windows sealed beyond them stay in the published
+// buffer and are carried behind the new base at publication.
+int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window, int64_t windows_r = -1) {
   const bool early = h->refit_ev_early && !h->pending;
   h->refit_ev_early = false;
   int rc = publish(h);
   if (rc) return rc;
   const int64_t S = h->cfg.n_sinks, W = h->cfg.window;
-  const int64_t n_r = S + h->n_windows * W;
+  const int64_t n_r = S + (windows_r >= 0 ? windows_r : h->n_windows) * W;
   if (n_r <= S) return AI_OK;
   Buffer& A = h->buf[h->active];
   const int target = 1 - h->active;
@@ -787,17 +790,17 @@ int ai_seal(ai_handle h, int64_t* version_out) {
     CK(cudaEventRecord(h->ev_main, h->main));
     h->refit_ev_early = true;
   }
-  while (h->n_windows < complete) {
-    int64_t nw = complete - h->n_windows;
-    if (R > 0) {
-      // stop the group at the next refit point
+  // every complete window in one launch (windows are independent); a refit
+  // whose boundary falls among them reads only keys, so it starts after the
+  // launch with the boundary's watermark
+  const int64_t w0 = h->n_windows;
+  if (complete > w0) {
+    int rc = seal_group(h, w0, complete - w0);
+    if (rc == AI_OK && R > 0) {
       const int64_t per = R / W;
-      const int64_t to_refit = per - (h->n_windows % per);
-      nw = std::min(nw, to_refit);
+      for (int64_t wb = (w0 / per + 1) * per; rc == AI_OK && wb <= complete; wb += per)
+        rc = start_refit(h, h->n_seed_default, h->seed_window_default, wb);
     }
-    int rc = seal_group(h, h->n_windows, nw);
-    if (rc == AI_OK && R > 0 && (h->n_windows * W) % R == 0)
-      rc = start_refit(h, h->n_seed_default, h->seed_window_default);
     if (rc) {
       h->refit_ev_early = false;
       return rc;
