@@ -875,10 +875,13 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
   const CUtensorMap* kmp = nullptr;
   const CUtensorMap* qmp = nullptr;
   if (tc_keys(h)) {
-    // bf16 rows gathered by TMA (box 64 x 1); fp8 rows are loaded by threads
-    // (the map then points at the queries and is not read)
-    const bool ok_k = h->cfg.key_dtype == AI_BF16 ? make_map(&kmap, h->keys, h->n_keys, 1)
-                                                  : make_map(&kmap, q, static_cast<int64_t>(T) * h->cfg.H, 1);
+    // rows gathered by TMA (box 64 x 1): the bf16 key store, or for fp8
+    // keys the bf16 copy of the codes (exact; the scale is applied to the
+    // score)
+    rc = ensure_codes_bf16(h);
+    if (rc) return rc;
+    const void* rows = h->cfg.key_dtype == AI_BF16 ? h->keys : static_cast<const void*>(h->codes_bf16);
+    const bool ok_k = make_map(&kmap, rows, h->n_keys, 1);
     if (!ok_k || !make_map(&qmap, q, static_cast<int64_t>(T) * h->cfg.H, h->cfg.H))
       return fail(AI_ERR_CUDA, "tensor map encoding failed (key store / queries)");
     kmp = &kmap;

@@ -68,7 +68,7 @@ struct RefineArgs {
 size_t refine_smem_bytes(int C, int H, int d, bool tc);
 // kmap: TMA map of the bf16 key store (box 64 x 1); qmap: TMA map of the
 // queries as [T*H, 128] bf16 rows (box 64 x H).  Both nullptr selects the
-// SIMT kernel (fp32 keys).  For fp8 keys kmap is unused but must be set.
+// SIMT kernel (fp32 keys).  For fp8 keys kmap covers the bf16 copy of the codes.
 cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUtensorMap* kmap,
                           const CUtensorMap* qmap, int num_sms, cudaStream_t st);
 

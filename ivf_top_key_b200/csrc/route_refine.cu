@@ -9,19 +9,22 @@
 // paragraph of "索引怎么边算边建？" fixes which clusters and which open window
 // a query at position t may use (passed in as a small version table).
 //
-// One persistent CTA per SM walks queries.  Per query:
-//  1. size-weighted radix select of the budget threshold over the cluster
-//     scores of the visible, non-empty clusters; the clusters at or above it
-//     are sorted by (score desc, id asc) and their member lists are copied,
-//     after sinks and the open window, into a shared-memory candidate list;
-//  2. exact rescore of the candidates, 128 at a time: the key rows are
-//     gathered into the 128-byte-swizzled UMMA layout (cp.async for bf16,
-//     fp8 codes widened to bf16 in registers), one tcgen05 UMMA
-//     (M = 128 candidates, N = H heads, K = 128) per tile accumulates in
-//     TMEM, and four epilogue warps apply ReLU, the head weights and the fp8
-//     scale (SIMT FMA path for fp32 keys);
-//  3. radix select of the k-th score; ties at the threshold go to the lower
-//     key id; ids are written in candidate-slot order, padded with -1.
+// Persistent CTAs (two per SM) walk queries.  Per query:
+//  1. candidate build: the route-score range and a size-weighted histogram
+//     (two levels) find the budget threshold over the visible non-empty
+//     clusters; the clusters at or above it are ranked by (score desc, id
+//     asc) and their member runs are copied, after the sinks and the open
+//     window, into a shared-memory candidate list;
+//  2. exact rescore, 128 candidates per tile: TMA tile::gather4 brings the
+//     bf16 rows (for fp8 keys, the bf16 copy of the codes) into the
+//     128-byte-swizzled UMMA layout, one tcgen05 UMMA (M = 128 candidates,
+//     N = H heads, K = 128) per tile accumulates in TMEM, and four epilogue
+//     warps apply ReLU, the head weights and the fp8 scale, keeping the
+//     scores in TMEM (SIMT FMA path for fp32 keys);
+//  3. top-k: a histogram over the score range locates the k-th score's bin,
+//     whose items are sorted to read the exact threshold; ties at the
+//     threshold go to the lower key id; ids are written in a fixed order,
+//     padded with -1.
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
@@ -429,46 +432,6 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
 }
 
 // ---------------------------------------------------------- tcgen05 kernel
-__device__ __forceinline__ void gather_tile_fp8(const RefineArgs& a, const int32_t* cand, int n,
-                                                int slot0, int64_t t, uint8_t* stage) {
-  const int gt = threadIdx.x;
-  const int gw = gt >> 5, lane = gt & 31;
-  const int c8 = lane & 7;  // 16-code chunk of the 128-code row
-  const uint8_t* keys = reinterpret_cast<const uint8_t*>(a.keys);
-  uint4 v[8];
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int row = gw * 32 + 4 * p + (lane >> 3);
-    const int slot = slot0 + row;
-    int32_t id = slot < n ? cand[slot] : -1;
-    if (id > t) {
-      atomicOr(a.err, DEV_ERR_RANGE);
-      id = -1;
-    }
-    v[p] = id >= 0 ? __ldg(reinterpret_cast<const uint4*>(keys + static_cast<int64_t>(id) * 128) + c8)
-                   : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int row = gw * 32 + 4 * p + (lane >> 3);
-    const uint8_t* b = reinterpret_cast<const uint8_t*>(&v[p]);
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      __nv_fp8x2_e4m3 pr;
-      pr.__x = static_cast<__nv_fp8x2_storage_t>(b[2 * j] | (b[2 * j + 1] << 8));
-      __nv_bfloat162 h2 = __float22bfloat162_rn(static_cast<float2>(pr));
-      w[j] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    // codes 16*c8 .. 16*c8+15 -> bf16 chunks 2*c8 and 2*c8+1 (8 values each)
-#pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-      const int chunk = 2 * c8 + hlf;
-      uint8_t* dst = stage + (chunk >> 3) * (kTile * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * hlf], w[4 * hlf + 1], w[4 * hlf + 2], w[4 * hlf + 3]);
-    }
-  }
-}
 
 // ------------------------------------------------- top-k by the epilogue warps
 // The 128 epilogue threads hold the candidate scores in TMEM: thread
@@ -881,7 +844,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
-      mbar_init(&full[s], fp8 ? 128 : 4);
+      mbar_init(&full[s], 4);
       mbar_init(&empty[s], 1);
     }
     for (int c = 0; c < 2; ++c) {
@@ -925,7 +888,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __syncthreads();
 
     const int ntiles = (n + kTile - 1) / kTile;
-    if (!fp8 && warp < 4) {
+    if (warp < 4) {
       // ------------------------------------------- TMA gather4 producers
       // Four warps share a tile (32 rows each): a single issuing warp
       // limits gather4 throughput, so the issue is spread out.
@@ -952,16 +915,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           uint8_t* dst = region + s * (kTile * 256) + half * (kTile * 128) + rl * 128;
           tma_gather4(dst, &kmap, half * 64, r[0], r[1], r[2], r[3], &full[s]);
         }
-      }
-    } else if (fp8 && warp < 4) {
-      // --------------------------------------- fp8 rows widened to bf16
-      for (int j = 0; j < ntiles; ++j) {
-        const uint32_t gj = g + j;
-        const int s = gj % kStages2;
-        if (gj >= kStages2 && !mbar_wait(&empty[s], ((gj / kStages2) & 1) ^ 1, a.err, abort_flag)) break;
-        gather_tile_fp8(a, cand, n, j * kTile, t, region + s * (kTile * 256));
-        fence_proxy_async_smem();
-        mbar_arrive(&full[s]);
       }
     } else if (warp == 4) {
       // ------------------------------------------------------ UMMA issue
