@@ -449,7 +449,9 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window, int64_t window
   const bool tc = h->cent_hi != nullptr;
   if (tc) {
     const int64_t K_pad = round_up(K, 128);
-    if (!make_map(&tcm.keys, h->keys, n_r, 1) || !make_map(&tcm.hi, h->cent_hi, K_pad, 128) ||
+    // bf16 keys, or for fp8 keys the bf16 copy of the codes (kept current at append)
+    const void* rows = h->cfg.key_dtype == AI_FP8E4M3 ? static_cast<const void*>(h->codes_bf16) : h->keys;
+    if (!rows || !make_map(&tcm.keys, rows, n_r, 1) || !make_map(&tcm.hi, h->cent_hi, K_pad, 128) ||
         !make_map(&tcm.lo, h->cent_lo, K_pad, 128))
       return fail(AI_ERR_CUDA, "tensor map encoding failed (refit)");
     tcm.num_sms = h->num_sms;
@@ -678,7 +680,7 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   CKC(dalloc(&h->scan_words, 16));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
   CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
-  if (c.key_dtype == AI_BF16 && d == 128) {
+  if ((c.key_dtype == AI_BF16 || c.key_dtype == AI_FP8E4M3) && d == 128 && c.refit_period > 0) {
     CKC(dalloc(&h->cent_hi, static_cast<size_t>(h->maxC_pad) * 128));
     CKC(dalloc(&h->cent_lo, static_cast<size_t>(h->maxC_pad) * 128));
     CKC(dalloc(&h->cent_cc, h->maxC_pad));
@@ -777,6 +779,8 @@ int ai_append_keys(ai_handle h, const void* keys_dev, const float* scales_dev, i
   if (h->cfg.key_dtype == AI_FP8E4M3)
     CK(cudaMemcpyAsync(h->scales + h->n_keys, scales_dev, n * sizeof(float), cudaMemcpyDeviceToDevice, h->main));
   h->n_keys += n;
+  // the tensor-core refit screen reads fp8 keys through their bf16 copy
+  if (h->cfg.key_dtype == AI_FP8E4M3 && h->cent_hi) return ensure_codes_bf16(h);
   return AI_OK;
 }
 

@@ -863,8 +863,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       mbar_arrive(&aempty[b]);
-      const float err = static_cast<float>(kTcErr * (static_cast<double>(xx) + ccmax));
       const int kk = kt * kTcKeys + row;
+      // fp8 keys: the tile holds the codes (exact in bf16), the key is
+      // scale * code; ||x||^2 and x.c take the scale (2^-24-level roundings,
+      // far inside the bound below)
+      float m2 = -2.f;
+      if (a.key_dtype == KD_FP8) {
+        const float sx = kk < n ? a.key_scale[bd.list[kk]] : 1.f;
+        xx = sx * sx * xx;
+        m2 = -2.f * sx;
+      }
+      const float err = static_cast<float>(kTcErr * (static_cast<double>(xx) + ccmax));
       float best = INFINITY, second = INFINITY;
       int bid = 0x7fffffff;
       float thr = 0.f;
@@ -896,7 +905,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kBandPass) {
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
+              const float d2 = fmaf(m2, v[q], xx + cc[q]);
               if (d2 <= thr) {
                 if (nb < kBand) bd.ids[static_cast<int64_t>(kk) * kBand + nb] = ct * kTcCent + c32 * 32 + q;
                 ++nb;
@@ -905,7 +914,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else {
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              const float d2 = fmaf(-2.f, v[q], xx + cc[q]);
+              const float d2 = fmaf(m2, v[q], xx + cc[q]);
               if (d2 < best) {
                 second = best;
                 best = d2;
@@ -966,7 +975,7 @@ cudaError_t launch_refit(const RefitArgs& a, int64_t max_tiles, cudaStream_t st,
   unsigned long long* rest_bits = reinterpret_cast<unsigned long long*>(a.n_scan + 4);
   int32_t* n_list = a.n_scan + 6;
   unsigned long long* ccmax_bits = reinterpret_cast<unsigned long long*>(a.n_scan + 8);
-  if (tc && (a.key_dtype != KD_BF16 || a.d != 128)) return cudaErrorInvalidValue;
+  if (tc && ((a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8) || a.d != 128)) return cudaErrorInvalidValue;
   cudaMemsetAsync(a.n_scan, 0, 40, st);
   const int64_t ce = static_cast<int64_t>(a.K) * a.d;
   count_launch();
