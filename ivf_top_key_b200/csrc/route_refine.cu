@@ -127,8 +127,7 @@ __device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, in
 }
 
 __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, int64_t n_v,
-                                int32_t* cand, uint64_t* sortbuf, int32_t* pref,
-                                BlockScratch& bs) {
+                                int32_t* cand, uint64_t* sortbuf, int32_t* pref) {
   const int C = a.C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = (blockDim.x + 31) >> 5;
@@ -397,7 +396,7 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref, bs);
+    const int n = build_candidates(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref);
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? L.cand[i] : -1;
@@ -805,8 +804,9 @@ __host__ __device__ inline size_t tc_region_bytes() {
   size_t m = p1 > p2 ? p1 : p2;
   return align_up(m > p3 ? m : p3, 1024);
 }
+constexpr int kTcSlack = 128;  // alignment slack of the dynamic shared memory
 __host__ __device__ inline size_t tc_smem_bytes(int C, int H) {
-  return 1024 + tc_region_bytes() + static_cast<size_t>(H) * 256 + align_up(static_cast<size_t>(C) * 4, 16) +
+  return kTcSlack + tc_region_bytes() + static_cast<size_t>(H) * 256 + align_up(static_cast<size_t>(C) * 4, 16) +
          align_up(static_cast<size_t>(H) * 4, 16) + (2 * kStages2 + 5) * 8 + 16;
 }
 __host__ __device__ inline int tc_tmem_cols(int C, int H) {
@@ -820,9 +820,15 @@ template <int H>
 __global__ void __launch_bounds__(kTcThreads, 2)
     k_refine_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 RefineArgs a, VersionTable vt) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ BlockScratch bs;
+  // 1024-byte alignment (128-byte swizzle atoms) is requested from the
+  // runtime; the launch adds kTcSlack bytes, and a base that would need
+  // more than that is reported instead of overrunning the allocation
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (base - smem_raw > kTcSlack) {
+    if (threadIdx.x == 0) atomicOr(a.err, DEV_ERR_RANGE);
+    return;
+  }
   uint8_t* region = base;
   uint8_t* qtile = region + tc_region_bytes();
   int32_t* cand = reinterpret_cast<int32_t*>(qtile + H * 256);
@@ -878,7 +884,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates(a, qi, t, nC, n_v, cand, sortbuf, pref, bs);
+    const int n = build_candidates(a, qi, t, nC, n_v, cand, sortbuf, pref);
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cand[i] : -1;
@@ -1010,8 +1016,16 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
   if (tc) {
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
-    // CTAs per SM bounded by shared memory and by TMEM (512 columns)
-    int per_sm = static_cast<int>((228 * 1024) / (smem + 2048));
+    // CTAs per SM bounded by shared memory (228 KiB per SM, 1 KiB reserved
+    // per CTA; the carveout is set to the maximum) and by TMEM (512 columns)
+    if (a.H == 32) {
+      cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    } else if (a.H == 64) {
+      cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    }
+    int per_sm = static_cast<int>((228 * 1024) / (smem + 1024));
     const int tm = 512 / tc_tmem_cols(a.C, a.H);
     per_sm = per_sm < tm ? per_sm : tm;
     per_sm = per_sm < 1 ? 1 : per_sm;
