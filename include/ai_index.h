@@ -227,6 +227,17 @@ int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_
                                  int64_t pos0, int32_t T, int32_t k, int32_t* out_dev,
                                  float* out_scores_dev, void* cuda_stream);
 
+/* ------------------------------------------------- failure-path test hook */
+/* Runs the library's bounded wait against a barrier that nothing completes
+ * (the pages have no counterpart: this exists to test failure detection).
+ * One thread polls an mbarrier phase at most spin_limit times (1 .. 2^26),
+ * then records the timeout in a device status word and returns, exactly as
+ * a kernel whose producer never arrives would.  Enqueued on cuda_stream and
+ * waited for.  *status_out receives the device status flags (bit 0 =
+ * timeout).  Returns AI_OK when the wait ran out and was reported,
+ * AI_ERR_ARG for a bad limit or null output, AI_ERR_CUDA on a CUDA error.  */
+int ai_debug_wait_timeout(int32_t spin_limit, int32_t* status_out, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

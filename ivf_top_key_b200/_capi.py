@@ -29,7 +29,7 @@ EXPORTED = [
     "ai_publish", "ai_route_refine", "ai_select_exhaustive", "ai_sync", "ai_last_error",
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
-    "ai_kernel_launches", "ai_select_exhaustive_noalloc",
+    "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
 
@@ -85,6 +85,7 @@ def _load():
         "ai_profile_enable": [vp, ctypes.c_int],
         "ai_profile_read": [vp, vp, vp],
         "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp],
+        "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -237,6 +238,14 @@ def ai_select_exhaustive_noalloc(keys, key_dtype: int, q, w, pos0: int, k: int, 
                                              pos0, q.shape[0], k, _ptr(out), _ptr(out_scores),
                                              _stream(stream)))
     return out
+
+
+def ai_debug_wait_timeout(spin_limit: int, stream=None) -> int:
+    """Bounded wait on a barrier nothing completes; returns the device status
+    flags it recorded (bit 0 = timeout)."""
+    st = ctypes.c_int32(0)
+    _check(_lib.ai_debug_wait_timeout(spin_limit, ctypes.byref(st), _stream(stream)))
+    return st.value
 
 
 def ai_last_error() -> str:
