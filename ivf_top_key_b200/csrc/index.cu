@@ -198,6 +198,7 @@ struct ai_index {
   uint16_t* cent_hi = nullptr;  // tensor-core refit scan (bf16 keys, d = 128)
   uint16_t* cent_lo = nullptr;
   float* cent_cc = nullptr;
+  int32_t* cand_scratch = nullptr;  // tensor-core refine: a candidate list per CTA
   int32_t* upd_chunk_off = nullptr;  // refit update chunks
   double* upd_part = nullptr;
   float* band_best = nullptr;  // near-tie bands of the tensor-core refit scan
@@ -678,6 +679,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   CKC(dalloc(&h->tile_counts, static_cast<size_t>(h->max_tiles) * h->maxC));
   CKC(dalloc(&h->scan_list, 2 * static_cast<size_t>(N)));
   CKC(dalloc(&h->scan_words, 16));
+  // one candidate row per refine CTA (at most 4 per SM)
+  if (tck) CKC(dalloc(&h->cand_scratch, static_cast<size_t>(h->num_sms) * 4 * c.max_budget));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
   CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
   if ((c.key_dtype == AI_BF16 || c.key_dtype == AI_FP8E4M3) && d == 128 && c.refit_period > 0) {
@@ -731,6 +734,7 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->cent_hi);
   cudaFree(h->cent_lo);
   cudaFree(h->cent_cc);
+  cudaFree(h->cand_scratch);
   cudaFree(h->upd_chunk_off);
   cudaFree(h->upd_part);
   cudaFree(h->band_best);
@@ -869,6 +873,7 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
   ra.out = out;
   ra.out_scores = out_scores;
   ra.cand_out = cand_out;
+  ra.cand_scratch = h->cand_scratch;
   ra.err = h->err_dev;
   int32_t* tmp_out = nullptr;
   if (!out) {  // debug call: outputs still need a home

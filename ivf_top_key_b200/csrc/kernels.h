@@ -63,6 +63,7 @@ struct RefineArgs {
   int32_t* out;              // [T, k]
   float* out_scores;         // [T, k] or nullptr
   int32_t* cand_out;         // debug: [T, C] candidate lists or nullptr
+  int32_t* cand_scratch;     // tensor-core path: [grid, C] candidate list per CTA
   int* err;
 };
 size_t refine_smem_bytes(int C, int H, int d, bool tc);

@@ -126,6 +126,9 @@ __device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, in
   __syncthreads();
 }
 
+// The list is written to shared memory (kGlobal = false) or to the CTA's
+// global scratch row (kGlobal = true).
+template <bool kGlobal>
 __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, int64_t n_v,
                                 int32_t* cand, uint64_t* sortbuf, int32_t* pref) {
   const int C = a.C;
@@ -325,9 +328,13 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     if (d0 >= len) continue;
     const int sz = min(pref[r + 1] - pref[r], len - d0);
     const int32_t* src = a.members + coff[r];
-    for (int l = lane; l < sz; l += 32) cp_async4(cand + d0 + l, src + l);
+    if (kGlobal) {
+      for (int l = lane; l < sz; l += 32) cand[d0 + l] = __ldg(src + l);
+    } else {
+      for (int l = lane; l < sz; l += 32) cp_async4(cand + d0 + l, src + l);
+    }
   }
-  cp_async_wait_all();
+  if (!kGlobal) cp_async_wait_all();
   __syncthreads();
   return len;
 }
@@ -396,7 +403,7 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref);
+    const int n = build_candidates<false>(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref);
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? L.cand[i] : -1;
@@ -757,22 +764,23 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   if (!partial_ties) {
     p3_for_each_all(c, [&mine, th](float v, int, int ok) { mine += ok & static_cast<int>(v >= th); });
   } else {
+    // rare: the id decides among the items tied at theta
     p3_for_each_all(c, [&mine, th, thid, cd, nlast](float v, int slot, int ok) {
       const int sl = slot <= nlast ? slot : 0;
-      mine += ok & (static_cast<int>(v > th) | (static_cast<int>(v == th) & static_cast<int>(cd[sl] <= thid)));
+      mine += ok & (static_cast<int>(v > th) | (v == th ? static_cast<int>(cd[sl] <= thid) : 0));
     });
   }
   int total;
   int pos = p3_scan(mine, et, &total, ps);
-  int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] ids
+  int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] slots
   float* ssc = reinterpret_cast<float*>(ps.buf) + kCapB;       // [k] scores
   int32_t* dump_id = reinterpret_cast<int32_t*>(ps.hist) + et;
   float* dump_sc = reinterpret_cast<float*>(ps.hist) + 128 + et;
-  auto stage = [&pos, sid, ssc, dump_id, dump_sc, k, cd, nlast](float v, int slot, int f) {
+  auto stage = [&pos, sid, ssc, dump_id, dump_sc, k](float v, int slot, int f) {
     const bool w = (f & static_cast<int>(pos < k)) != 0;
     int32_t* pi = w ? sid + pos : dump_id;
     float* pv = w ? ssc + pos : dump_sc;
-    *pi = cd[slot <= nlast ? slot : 0];
+    *pi = slot;
     *pv = v;
     pos += f;
   };
@@ -783,13 +791,13 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   } else {
     p3_for_each_all(c, [stage, th, thid, cd, nlast](float v, int slot, int ok) mutable {
       const int sl = slot <= nlast ? slot : 0;
-      stage(v, slot, ok & (static_cast<int>(v > th) | (static_cast<int>(v == th) & static_cast<int>(cd[sl] <= thid))));
+      stage(v, slot, ok & (static_cast<int>(v > th) | (v == th ? static_cast<int>(cd[sl] <= thid) : 0)));
     });
   }
   named_bar(1, 128);
   const int nw = min(total, k);
   for (int j = et; j < k; j += 128) {
-    out[j] = j < nw ? sid[j] : -1;
+    out[j] = j < nw ? cd[sid[j]] : -1;
     if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
   }
   named_bar(1, 128);
@@ -805,9 +813,13 @@ __host__ __device__ inline size_t tc_region_bytes() {
   return align_up(m > p3 ? m : p3, 1024);
 }
 constexpr int kTcSlack = 128;  // alignment slack of the dynamic shared memory
-__host__ __device__ inline size_t tc_smem_bytes(int C, int H) {
-  return kTcSlack + tc_region_bytes() + static_cast<size_t>(H) * 256 + align_up(static_cast<size_t>(C) * 4, 16) +
-         align_up(static_cast<size_t>(H) * 4, 16) + (2 * kStages2 + 5) * 8 + 16;
+constexpr int kTcCtasPerSm = 2;  // launch bound: CTAs per SM the registers allow
+// global_cand: the candidate list lives in a global scratch row (for large
+// budgets whose list would leave room for one CTA per SM only)
+__host__ __device__ inline size_t tc_smem_bytes(int C, int H, bool global_cand) {
+  return kTcSlack + tc_region_bytes() + static_cast<size_t>(H) * 256 +
+         (global_cand ? 0 : align_up(static_cast<size_t>(C) * 4, 16)) + align_up(static_cast<size_t>(H) * 4, 16) +
+         (2 * kStages2 + 5) * 8 + 16;
 }
 __host__ __device__ inline int tc_tmem_cols(int C, int H) {
   const int sc = ((C + 127) / 128 + 15) / 16 * 16;
@@ -816,8 +828,8 @@ __host__ __device__ inline int tc_tmem_cols(int C, int H) {
   return cols;
 }
 
-template <int H>
-__global__ void __launch_bounds__(kTcThreads, 2)
+template <int H, bool kGC>
+__global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     k_refine_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 RefineArgs a, VersionTable vt) {
   // 1024-byte alignment (128-byte swizzle atoms) is requested from the
@@ -831,8 +843,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   }
   uint8_t* region = base;
   uint8_t* qtile = region + tc_region_bytes();
-  int32_t* cand = reinterpret_cast<int32_t*>(qtile + H * 256);
-  float* wsh = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(cand) + align_up(static_cast<size_t>(a.C) * 4, 16));
+  // the candidate list of the query in flight: in shared memory, or (kGC)
+  // this CTA's row of the global scratch
+  int32_t* cand = kGC ? a.cand_scratch + static_cast<int64_t>(blockIdx.x) * a.C
+                      : reinterpret_cast<int32_t*>(qtile + H * 256);
+  float* wsh = reinterpret_cast<float*>(qtile + H * 256 + (kGC ? 0 : align_up(static_cast<size_t>(a.C) * 4, 16)));
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(wsh) + align_up(H * 4, 16));
   uint64_t* qfull = bars + 2 * kStages2 + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages2 + 5);
@@ -884,7 +899,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates(a, qi, t, nC, n_v, cand, sortbuf, pref);
+    const int n = build_candidates<kGC>(a, qi, t, nC, n_v, cand, sortbuf, pref);
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cand[i] : -1;
@@ -1002,7 +1017,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 }  // namespace
 
 size_t refine_smem_bytes(int C, int H, int d, bool tc) {
-  if (tc) return tc_smem_bytes(C, H);
+  if (tc) return tc_smem_bytes(C, H, true);  // the smaller layout; the launch picks
   return 1024 + region_bytes(H, d, false) + 2 * align_up(static_cast<size_t>(C) * 4, 16) +
          align_up(static_cast<size_t>(H) * 4, 16) + (2 * kStages + 4) * 8 + 16;
 }
@@ -1017,30 +1032,35 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
     // CTAs per SM bounded by shared memory (228 KiB per SM, 1 KiB reserved
-    // per CTA; the carveout is set to the maximum) and by TMEM (512 columns)
-    if (a.H == 32) {
-      cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    } else if (a.H == 64) {
-      cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    }
-    int per_sm = static_cast<int>((228 * 1024) / (smem + 1024));
-    const int tm = 512 / tc_tmem_cols(a.C, a.H);
-    per_sm = per_sm < tm ? per_sm : tm;
-    per_sm = per_sm < 1 ? 1 : per_sm;
+    // per CTA; the carveout is set to the maximum), by TMEM (512 columns)
+    // and by the registers; the list stays in shared memory unless that
+    // costs the second CTA
+    auto per_sm_for = [&](size_t sm) {
+      int p = static_cast<int>((228 * 1024) / (sm + 1024));
+      const int tm = 512 / tc_tmem_cols(a.C, a.H);
+      p = p < tm ? p : tm;
+      p = p < kTcCtasPerSm ? p : kTcCtasPerSm;
+      return p < 1 ? 1 : p;
+    };
+    const size_t sm_local = tc_smem_bytes(a.C, a.H, false);
+    const bool gc = !(sm_local <= 227 * 1024 && per_sm_for(sm_local) >= kTcCtasPerSm) && a.cand_scratch != nullptr;
+    const size_t smem = gc ? tc_smem_bytes(a.C, a.H, true) : sm_local;
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    const int per_sm = per_sm_for(smem);
     const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
-    if (a.H == 32) {
-      cudaFuncSetAttribute(k_refine_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      count_launch();
-      k_refine_tc<32><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);
-    } else if (a.H == 64) {
-      cudaFuncSetAttribute(k_refine_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      count_launch();
-      k_refine_tc<64><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);
-    } else {
-      return cudaErrorInvalidValue;
-    }
+#define AI_LAUNCH_REFINE(HH, GC)                                                                         \
+  do {                                                                                                   \
+    cudaFuncSetAttribute(k_refine_tc<HH, GC>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
+    cudaFuncSetAttribute(k_refine_tc<HH, GC>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);      \
+    count_launch();                                                                                      \
+    k_refine_tc<HH, GC><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);                           \
+  } while (0)
+    if (a.H == 32 && gc) AI_LAUNCH_REFINE(32, true);
+    else if (a.H == 32) AI_LAUNCH_REFINE(32, false);
+    else if (a.H == 64 && gc) AI_LAUNCH_REFINE(64, true);
+    else if (a.H == 64) AI_LAUNCH_REFINE(64, false);
+    else return cudaErrorInvalidValue;
+#undef AI_LAUNCH_REFINE
   } else {
     cudaFuncSetAttribute(k_refine_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     int per_sm = 1;
