@@ -227,6 +227,19 @@ int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_
                                  int64_t pos0, int32_t T, int32_t k, int32_t* out_dev,
                                  float* out_scores_dev, void* cuda_stream);
 
+/* ------------------------------------------------ refine kernel variant */
+/* Selects the kernel that runs route+refine on the tensor-core path (bf16
+ * or fp8 keys) for later ai_route_refine / ai_debug_candidates calls on h.
+ * All variants compute the same result; this exists so tests can cover
+ * each one.  kernel: 0 = chosen by occupancy (the default), 1 = one query
+ * at a time per CTA with the candidate list in shared memory, 2 = the same
+ * with the list in global scratch, 3 = pipelined (the candidate build and
+ * the top-k of neighbouring queries overlap the rescore of the current
+ * one).  A variant whose shared memory or TMEM need does not fit the
+ * configuration makes those calls fail with AI_ERR_CUDA.  Returns AI_OK,
+ * or AI_ERR_ARG for a null handle or a kernel outside 0..3.              */
+int ai_debug_refine_kernel(ai_handle h, int32_t kernel);
+
 /* ------------------------------------------------- failure-path test hook */
 /* Runs the library's bounded wait against a barrier that nothing completes
  * (the pages have no counterpart: this exists to test failure detection).

@@ -106,6 +106,12 @@ class AttentionIndex:
         out = torch.empty((q.shape[0], n), dtype=torch.float32, device=q.device)
         return C.ai_debug_scores(self.h, q, w, pos0, out)
 
+    def debug_refine_kernel(self, kernel: int):
+        """Force a tensor-core refine variant (0 = by occupancy, 1 / 2 =
+        one query per CTA with the list in shared / global memory, 3 =
+        pipelined); every variant computes the same result."""
+        C.ai_debug_refine_kernel(self.h, kernel)
+
     def profile(self, enable: bool = True):
         C.ai_profile_enable(self.h, enable)
 

@@ -30,6 +30,7 @@ EXPORTED = [
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
     "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
+    "ai_debug_refine_kernel",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
 
@@ -86,6 +87,7 @@ def _load():
         "ai_profile_read": [vp, vp, vp],
         "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp],
         "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
+        "ai_debug_refine_kernel": [vp, i32],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -246,6 +248,12 @@ def ai_debug_wait_timeout(spin_limit: int, stream=None) -> int:
     st = ctypes.c_int32(0)
     _check(_lib.ai_debug_wait_timeout(spin_limit, ctypes.byref(st), _stream(stream)))
     return st.value
+
+
+def ai_debug_refine_kernel(h, kernel: int):
+    """Select the tensor-core refine variant (0 auto, 1 sequential with the
+    list in shared memory, 2 sequential with a global list, 3 pipelined)."""
+    _check(_lib.ai_debug_refine_kernel(h, kernel))
 
 
 def ai_last_error() -> str:

@@ -198,7 +198,8 @@ struct ai_index {
   uint16_t* cent_hi = nullptr;  // tensor-core refit scan (bf16 keys, d = 128)
   uint16_t* cent_lo = nullptr;
   float* cent_cc = nullptr;
-  int32_t* cand_scratch = nullptr;  // tensor-core refine: a candidate list per CTA
+  int32_t* cand_scratch = nullptr;  // tensor-core refine: candidate lists, 4 per SM
+  int refine_kernel = 0;             // tensor-core refine variant (0 = by occupancy)
   int32_t* upd_chunk_off = nullptr;  // refit update chunks
   double* upd_part = nullptr;
   float* band_best = nullptr;  // near-tie bands of the tensor-core refit scan
@@ -874,6 +875,7 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
   ra.out_scores = out_scores;
   ra.cand_out = cand_out;
   ra.cand_scratch = h->cand_scratch;
+  ra.refine_kernel = h->refine_kernel;
   ra.err = h->err_dev;
   int32_t* tmp_out = nullptr;
   if (!out) {  // debug call: outputs still need a home
@@ -1079,6 +1081,13 @@ int ai_rollback(ai_handle h) {
   // the side stream must not start the next refit before the restore lands
   CK(cudaEventRecord(h->ev_main, h->main));
   CK(cudaStreamWaitEvent(h->side, h->ev_main, 0));
+  return AI_OK;
+}
+
+int ai_debug_refine_kernel(ai_handle h, int32_t kernel) {
+  if (!h) return fail(AI_ERR_ARG, "null handle");
+  if (kernel < 0 || kernel > 3) return fail(AI_ERR_ARG, "refine kernel must be 0..3");
+  h->refine_kernel = kernel;
   return AI_OK;
 }
 

@@ -63,9 +63,11 @@ struct RefineArgs {
   int32_t* out;              // [T, k]
   float* out_scores;         // [T, k] or nullptr
   int32_t* cand_out;         // debug: [T, C] candidate lists or nullptr
-  int32_t* cand_scratch;     // tensor-core path: [grid, C] candidate list per CTA
+  int32_t* cand_scratch;     // tensor-core path: candidate lists, [4 * num_sms, C]
+  int refine_kernel;         // REFINE_* (tensor-core path; AUTO picks by occupancy)
   int* err;
 };
+enum RefineKernel { REFINE_AUTO = 0, REFINE_SEQ_SMEM = 1, REFINE_SEQ_GLOBAL = 2, REFINE_PIPE = 3 };
 size_t refine_smem_bytes(int C, int H, int d, bool tc);
 // kmap: TMA map of the bf16 key store (box 64 x 1); qmap: TMA map of the
 // queries as [T*H, 128] bf16 rows (box 64 x H).  Both nullptr selects the

@@ -41,10 +41,25 @@ constexpr int kSimtThreads = 256;
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
-__device__ __forceinline__ void bitonic_sort_u64(uint64_t* buf, int n) {
+// The threads that run the candidate build: the whole block, or a
+// warp-aligned group of 128 threads synchronised by a named barrier.
+struct BlockGrp {
+  __device__ int tid() const { return threadIdx.x; }
+  __device__ int size() const { return blockDim.x; }
+  __device__ void sync() const { __syncthreads(); }
+};
+struct SubGrp128 {
+  int first, bar;  // first thread of the group, named barrier id
+  __device__ int tid() const { return threadIdx.x - first; }
+  __device__ int size() const { return 128; }
+  __device__ void sync() const { named_bar(bar, 128); }
+};
+
+template <class G>
+__device__ __forceinline__ void bitonic_sort_u64(uint64_t* buf, int n, const G& g) {
   for (int k = 2; k <= n; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      for (int i = g.tid(); i < n; i += g.size()) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const uint64_t x = buf[i], y = buf[ixj];
@@ -55,7 +70,7 @@ __device__ __forceinline__ void bitonic_sort_u64(uint64_t* buf, int n) {
           }
         }
       }
-      __syncthreads();
+      g.sync();
     }
   }
 }
@@ -80,8 +95,10 @@ __device__ __forceinline__ void version_of(const VersionTable& vt, int64_t t, in
 // exactly and the fill stops at C.
 constexpr int kNB1 = 2048;
 struct P1Smem {
-  int32_t coff[kSortCap];  // member offset of each ranked cluster
-  uint32_t hist[kNB1];
+  union {                    // the histogram is dead before the offsets are written
+    int32_t coff[kSortCap];  // member offset of each ranked cluster
+    uint32_t hist[kNB1];
+  };
   float fred[32];
   unsigned long long wred[16];
   int scal[4];
@@ -89,10 +106,11 @@ struct P1Smem {
 
 // Warp 0 scans the weighted histogram ps.hist from the top for the bin
 // where the weight reaches `need`: its index and the weight above it.
-// All threads call it (it ends with a barrier).
-__device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, int* above) {
+// All threads of the group call it (it ends with a barrier).
+template <class G>
+__device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, int* above, const G& g) {
   const int lane = threadIdx.x & 31;
-  if (threadIdx.x < 32) {
+  if (g.tid() < 32) {
     uint32_t lsum = 0;
     for (int b = 0; b < 64; ++b) lsum += ps.hist[lane * 64 + b];
     uint32_t incl = lsum;  // sum over lanes >= this one
@@ -120,29 +138,30 @@ __device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, in
       ps.scal[2] = static_cast<int>(fa);
     }
   }
-  __syncthreads();
+  g.sync();
   *bstar = ps.scal[0];
   *above = ps.scal[2];
-  __syncthreads();
+  g.sync();
 }
 
 // The list is written to shared memory (kGlobal = false) or to the CTA's
 // global scratch row (kGlobal = true).
-template <bool kGlobal>
+template <bool kGlobal, class G>
 __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, int64_t n_v,
-                                int32_t* cand, uint64_t* sortbuf, int32_t* pref) {
+                                int32_t* cand, uint64_t* sortbuf, int32_t* pref, const G& g) {
   const int C = a.C;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = (blockDim.x + 31) >> 5;
+  const int tid = g.tid(), lane = tid & 31, warp = tid >> 5;
+  const int nthr = g.size();
+  const int nwarps = (nthr + 31) >> 5;
   const int n_s = static_cast<int>(min64(a.n_sinks, t + 1));
   const int64_t open_lo = max64(n_v, a.n_sinks);
   const int64_t n_open64 = open_lo <= t ? t + 1 - open_lo : 0;
   const int fixed = static_cast<int>(min64(C, n_s + n_open64));
-  for (int i = tid; i < fixed; i += blockDim.x)
+  for (int i = tid; i < fixed; i += nthr)
     cand[i] = i < n_s ? i : static_cast<int32_t>(open_lo + (i - n_s));
   const int rem = C - fixed;
   if (rem <= 0 || nC == 0) {
-    __syncthreads();
+    g.sync();
     return fixed;
   }
   // scratch after the sort buffer and prefix array
@@ -154,7 +173,7 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   float vmin = INFINITY, vmax = -INFINITY;
   unsigned long long wsum = 0;
 #pragma unroll 4
-  for (int c = tid; c < nC; c += blockDim.x) {
+  for (int c = tid; c < nC; c += nthr) {
     const int sz = __ldg(off + c + 1) - __ldg(off + c);
     const float v = __ldg(rs + c);
     if (sz > 0) {
@@ -173,8 +192,8 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     ps.fred[16 + warp] = vmax;
     ps.wred[warp] = wsum;
   }
-  for (int i = tid; i < kNB1; i += blockDim.x) ps.hist[i] = 0;
-  __syncthreads();
+  for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
+  g.sync();
   vmin = INFINITY;
   vmax = -INFINITY;
   wsum = 0;
@@ -201,12 +220,12 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   if (!take_all) {
     // pass B: size-weighted histogram; the bin where the weight from the top
     // reaches the remaining budget
-    for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+    for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
       float v[4];
       int sz[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * blockDim.x;
+        const int c = c0 + u * nthr;
         sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
         v[u] = c < nC ? __ldg(rs + c) : 0.f;
       }
@@ -214,19 +233,19 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
       for (int u = 0; u < 4; ++u)
         if (sz[u] > 0) atomicAdd(&ps.hist[binof(v[u])], static_cast<uint32_t>(sz[u]));
     }
-    __syncthreads();
+    g.sync();
     int above1 = 0;
-    p1_find_bin(ps, rem, &bstar, &above1);
+    p1_find_bin(ps, rem, &bstar, &above1, g);
     // pass B2: the boundary bin split into kNB1 sub-bins (a long score tail
     // leaves most clusters in few level-1 bins)
-    for (int i = tid; i < kNB1; i += blockDim.x) ps.hist[i] = 0;
-    __syncthreads();
-    for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+    for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
+    g.sync();
+    for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
       float v[4];
       int sz[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * blockDim.x;
+        const int c = c0 + u * nthr;
         sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
         v[u] = c < nC ? __ldg(rs + c) : 0.f;
       }
@@ -234,9 +253,9 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
       for (int u = 0; u < 4; ++u)
         if (sz[u] > 0 && binof(v[u]) == bstar) atomicAdd(&ps.hist[bin2(v[u], bstar)], static_cast<uint32_t>(sz[u]));
     }
-    __syncthreads();
+    g.sync();
     int above2 = 0;
-    p1_find_bin(ps, rem - above1, &bstar2, &above2);
+    p1_find_bin(ps, rem - above1, &bstar2, &above2, g);
   }
   auto selected = [=](float v) -> bool {
     if (take_all) return true;
@@ -246,19 +265,19 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   };
   // pass C: clusters at or above the boundary bin (any order: sorted next)
   if (tid == 0) ps.scal[1] = 0;
-  __syncthreads();
-  for (int c0 = tid; c0 < nC; c0 += 4 * blockDim.x) {
+  g.sync();
+  for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
     float v[4];
     int sz[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * blockDim.x;
+      const int c = c0 + u * nthr;
       sz[u] = c < nC ? off[c + 1] - off[c] : 0;
       v[u] = c < nC ? rs[c] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * blockDim.x;
+      const int c = c0 + u * nthr;
       if (sz[u] > 0 && selected(v[u])) {
         const int pos = atomicAdd(&ps.scal[1], 1);
         if (pos < kSortCap)
@@ -266,7 +285,7 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
       }
     }
   }
-  __syncthreads();
+  g.sync();
   int nsel = ps.scal[1];
   if (nsel > kSortCap) {
     if (tid == 0) atomicOr(a.err, DEV_ERR_CAPACITY);
@@ -278,31 +297,31 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   const uint64_t* sorted = sortbuf;
   if (nsel <= kSortCap / 4) {
     uint64_t* dst = sortbuf + kSortCap / 2;
-    for (int i = tid; i < nsel; i += blockDim.x) {
+    for (int i = tid; i < nsel; i += nthr) {
       const uint64_t x = sortbuf[i];
       int r = 0;
       for (int j = 0; j < nsel; ++j) r += sortbuf[j] < x ? 1 : 0;
       dst[r] = x;
     }
-    __syncthreads();
+    g.sync();
     sorted = dst;
   } else {
     int np = 1;
     while (np < nsel) np <<= 1;
-    for (int i = nsel + tid; i < np; i += blockDim.x) sortbuf[i] = ~0ull;
-    __syncthreads();
-    bitonic_sort_u64(sortbuf, np);
+    for (int i = nsel + tid; i < np; i += nthr) sortbuf[i] = ~0ull;
+    g.sync();
+    bitonic_sort_u64(sortbuf, np, g);
   }
   // member offsets and sizes of the ranked clusters (parallel loads), then
   // the exclusive prefix of sizes in rank order
   int32_t* coff = ps.coff;
-  for (int r = tid; r < nsel; r += blockDim.x) {
+  for (int r = tid; r < nsel; r += nthr) {
     const int c = static_cast<int>(sorted[r] & 0xffffffffu);
     const int o0 = off[c];
     coff[r] = o0;
     pref[r] = off[c + 1] - o0;
   }
-  __syncthreads();
+  g.sync();
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < nsel; base += 32) {
@@ -319,23 +338,44 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     }
     if (lane == 0) pref[nsel] = carry;
   }
-  __syncthreads();
+  g.sync();
   const int len = static_cast<int>(min64(C, static_cast<int64_t>(fixed) + pref[nsel]));
-  // fill: one warp per ranked cluster copies its member run into the list
-  // with 4-byte asynchronous copies (all in flight at once), cut at C
-  for (int r = warp; r < nsel; r += nwarps) {
-    const int d0 = fixed + pref[r];
-    if (d0 >= len) continue;
-    const int sz = min(pref[r + 1] - pref[r], len - d0);
-    const int32_t* src = a.members + coff[r];
-    if (kGlobal) {
-      for (int l = lane; l < sz; l += 32) cand[d0 + l] = __ldg(src + l);
-    } else {
+  if (kGlobal) {
+    // fill of a list in global memory: each thread walks its slots (stride
+    // = group size) through the ranked runs, several loads in flight
+    int r = 0;
+    for (int i0 = fixed + tid; i0 < len; i0 += 4 * nthr) {
+      int32_t v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * nthr;
+        v[u] = 0;
+        if (i < len) {
+          const int rel = i - fixed;
+          while (pref[r + 1] <= rel) ++r;
+          v[u] = __ldg(a.members + coff[r] + (rel - pref[r]));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * nthr;
+        if (i < len) cand[i] = v[u];
+      }
+    }
+  } else {
+    // fill of a list in shared memory: one warp per ranked cluster copies
+    // its member run with 4-byte asynchronous copies (all in flight at
+    // once), cut at C
+    for (int r = warp; r < nsel; r += nwarps) {
+      const int d0 = fixed + pref[r];
+      if (d0 >= len) continue;
+      const int sz = min(pref[r + 1] - pref[r], len - d0);
+      const int32_t* src = a.members + coff[r];
       for (int l = lane; l < sz; l += 32) cp_async4(cand + d0 + l, src + l);
     }
+    cp_async_wait_all();
   }
-  if (!kGlobal) cp_async_wait_all();
-  __syncthreads();
+  g.sync();
   return len;
 }
 
@@ -403,7 +443,7 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates<false>(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref);
+    const int n = build_candidates<false>(a, qi, t, nC, n_v, L.cand, L.sortbuf, L.pref, BlockGrp{});
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? L.cand[i] : -1;
@@ -899,7 +939,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     int nC;
     int64_t n_v;
     version_of(vt, t, &nC, &n_v);
-    const int n = build_candidates<kGC>(a, qi, t, nC, n_v, cand, sortbuf, pref);
+    const int n = build_candidates<kGC>(a, qi, t, nC, n_v, cand, sortbuf, pref, BlockGrp{});
     if (a.cand_out) {
       for (int i = threadIdx.x; i < a.C; i += blockDim.x)
         a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cand[i] : -1;
@@ -1014,6 +1054,288 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
   }
 }
 
+// ------------------------------------------------- pipelined tcgen05 kernel
+// The three phases of consecutive queries overlap inside one CTA:
+//   warps 0-3  gather the candidate rows of query i (TMA gather4) and run
+//              the epilogue (ReLU, head weights) into TMEM score columns
+//   warp 4     loads query i's head tile and issues the UMMAs
+//   warps 5-8  build the candidate list of query i+1, then select the
+//              top-k of query i-1 from its score columns
+// Candidate lists live in two global scratch rows per CTA and score
+// columns in two TMEM buffers, so the build and the top-k of neighbouring
+// queries run while the gather of query i keeps the copy engine busy.
+// Synchronisation (all mbarriers, every wait bounded):
+//   full[s]    tile rows landed in stage s (TMA transaction count)
+//   tfull[a]   UMMAs of a tile done: accumulator a written, its stage free
+//   tempty[a]  epilogue has read accumulator a
+//   qfull      head tile landed;  qempty  UMMAs of the previous query done
+//   cready[b]  list b built;  sready[b]  score columns b written;
+//   sfree[b]   score columns b read by the top-k
+__host__ __device__ inline size_t pipe_bg_bytes() {
+  const size_t p1 = align_up(static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4, 16) + sizeof(P1Smem);
+  const size_t p3 = sizeof(P3Smem);
+  return align_up(p1 > p3 ? p1 : p3, 16);
+}
+constexpr int kPipeBars = 14;
+__host__ __device__ inline size_t pipe_smem_bytes(int H) {
+  return kTcSlack + static_cast<size_t>(kStages2) * kTile * 256 + static_cast<size_t>(H) * 256 + pipe_bg_bytes() +
+         align_up(static_cast<size_t>(H) * 4, 16) + 16 + kPipeBars * 8 + 8;
+}
+__host__ __device__ inline int pipe_sc_cols(int C) { return ((C + 127) / 128 + 15) / 16 * 16; }
+__host__ __device__ inline int pipe_tmem_cols(int C, int H) {
+  const int need = 2 * H + 2 * pipe_sc_cols(C);
+  int cols = 32;
+  while (cols < need) cols <<= 1;
+  return cols;
+}
+
+template <int H>
+__global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
+    k_refine_pipe(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                  RefineArgs a, VersionTable vt) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (base - smem_raw > kTcSlack) {
+    if (threadIdx.x == 0) atomicOr(a.err, DEV_ERR_RANGE);
+    return;
+  }
+  uint8_t* stages = base;
+  uint8_t* qtile = stages + kStages2 * kTile * 256;
+  uint8_t* bg = qtile + H * 256;
+  float* wsh = reinterpret_cast<float*>(bg + pipe_bg_bytes());
+  int* meta = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(wsh) + align_up(H * 4, 16));  // list lengths [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta + 4);
+  uint64_t* full = bars;
+  uint64_t* tfull = bars + 2;
+  uint64_t* tempty = bars + 4;
+  uint64_t* qfull = bars + 6;
+  uint64_t* qempty = bars + 7;
+  uint64_t* cready = bars + 8;
+  uint64_t* sready = bars + 10;
+  uint64_t* sfree = bars + 12;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kPipeBars);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tcols = pipe_tmem_cols(a.C, H);
+  const int sc_cols = pipe_sc_cols(a.C);
+  int32_t* rows = a.cand_scratch + static_cast<int64_t>(2 * blockIdx.x) * a.C;  // this CTA's two lists
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 4);  // one arrive.expect_tx per gathering warp
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+      mbar_init(&cready[i], 128);
+      mbar_init(&sready[i], 128);
+      mbar_init(&sfree[i], 128);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_holder, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int nq = static_cast<int>(blockIdx.x) < a.T ? (a.T - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+
+  if (warp < 4) {
+    // --------------------------------------------- gather + epilogue (0-3)
+    const int row = warp * 32 + lane;  // tile row == TMEM lane of this thread
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const bool fp8 = a.key_dtype == KD_FP8;
+    uint32_t g = 0;           // tiles issued by this CTA so far
+    int64_t last_issued = -1;
+    bool dead = false;
+    for (int q = 0; q < nq; ++q) {
+      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const int64_t t = a.pos0 + qi;
+      const int b = q & 1;
+      bool ok = !dead && mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
+      if (ok && q >= 2) ok = mbar_wait(&sfree[b], ((q >> 1) & 1) ^ 1, a.err, abort_flag);
+      // every thread of the group takes the same way out; the barrier also
+      // orders the previous query's reads of wsh before its rewrite
+      if (!named_bar_and(3, 128, ok)) break;
+      tc_fence_after();
+      const int n = meta[b];
+      const int nt = (n + kTile - 1) / kTile;
+      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C;
+      for (int h = row; h < H; h += 128) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
+      named_bar(3, 128);
+      const uint32_t scol = tmem_base + 2 * H + b * sc_cols + lane_off;
+      int myid = row < n ? cl[row] : 0;  // this thread's row of tile 0
+      float sc0 = 1.f, sc1 = 1.f;          // fp8 scales of the tiles in flight (by tile parity)
+      // iteration j issues tile j and finishes the epilogue of tile j-2
+      auto step = [&](int j, float& s_slot) -> bool {
+        const uint32_t gj = g + j;
+        const int acc = gj & 1;
+        if (j >= 2) {
+          // UMMAs of tile j-2 done: its accumulator is ready and stage
+          // gj & 1 is free
+          const bool w = mbar_wait(&tfull[acc], ((gj - 2) >> 1) & 1, a.err, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) return false;
+          tc_fence_after();
+        }
+        const float s_ep = s_slot;  // scale of tile j-2
+        if (j < nt) {
+          int id = myid;
+          if (row + j * kTile < n && (id < 0 || id > t)) {
+            atomicOr(a.err, DEV_ERR_RANGE);
+            id = 0;
+          }
+          int r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, id, (lane & 7) * 4 + i);
+          if (lane == 0) mbar_arrive_expect_tx(&full[gj & 1], kTile * 256 / 4);
+          __syncwarp();
+          if (lane < 16) {
+            const int half = lane >> 3;
+            const int rl = warp * 32 + (lane & 7) * 4;
+            uint8_t* dst = stages + (gj & 1) * (kTile * 256) + half * (kTile * 128) + rl * 128;
+            tma_gather4(dst, &kmap, half * 64, r[0], r[1], r[2], r[3], &full[gj & 1]);
+          }
+          last_issued = gj;
+          // consumed two iterations later: the loads stay in flight
+          s_slot = fp8 ? a.key_scale[id] : 1.f;
+          const int nslot = (j + 1) * kTile + row;
+          myid = (j + 1 < nt && nslot < n) ? cl[nslot] : 0;
+        }
+        if (j >= 2) {
+          float sc = 0.f;
+#pragma unroll
+          for (int c = 0; c < H / 32; ++c) {
+            float v[32];
+            tmem_ld32(tmem_base + acc * H + c * 32 + lane_off, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int h = 0; h < 32; ++h) sc = fmaf(wsh[c * 32 + h], fmaxf(v[h], 0.f), sc);
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+          tmem_st1(scol + (j - 2), sc * s_ep);
+        }
+        return true;
+      };
+      bool good = true;
+      for (int j = 0; good && j < nt + 2; j += 2) {
+        good = step(j, sc0);
+        if (good && j + 1 < nt + 2) good = step(j + 1, sc1);
+      }
+      if (!good) {
+        dead = true;
+        continue;  // the next barrier takes every thread of the group out
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sready[b]);
+      g += nt;
+    }
+    if (*abort_flag && lane == 0 && last_issued >= 0) {
+      // copies this warp issued may still be landing: bounded wait
+      for (int64_t e = last_issued > 0 ? last_issued - 1 : 0; e <= last_issued; ++e)
+        mbar_drain(&full[e & 1], (e >> 1) & 1);
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------ UMMA issue (4)
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTile, H);
+      const uint32_t sb = smem_u32(qtile);
+      uint32_t g = 0;
+      int commits = 0;
+      for (int q = 0; q < nq; ++q) {
+        const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+        const int b = q & 1;
+        if (!mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag)) break;
+        const int nt = (meta[b] + kTile - 1) / kTile;
+        // the head tile is rewritten once the previous query's UMMAs are done
+        if (q > 0 && !mbar_wait(qempty, (commits - 1) & 1, a.err, abort_flag)) break;
+        mbar_arrive_expect_tx(qfull, H * 256);
+        tma_load_2d(qtile, &qmap, 0, qi * H, qfull);
+        tma_load_2d(qtile + H * 128, &qmap, 64, qi * H, qfull);
+        if (!mbar_wait(qfull, q & 1, a.err, abort_flag)) {
+          mbar_drain(qfull, q & 1);
+          break;
+        }
+        bool good = true;
+        for (int j = 0; j < nt; ++j) {
+          const uint32_t gj = g + j;
+          const int s = gj & 1;
+          if (!mbar_wait(&full[s], (gj >> 1) & 1, a.err, abort_flag) ||
+              (gj >= 2 && !mbar_wait(&tempty[s], ((gj >> 1) & 1) ^ 1, a.err, abort_flag))) {
+            good = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + s * (kTile * 256));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
+            umma_bf16(tmem_base + s * H, sdesc_sw128(sa + kb * (kTile * 128) + ko),
+                      sdesc_sw128(sb + kb * (H * 128) + ko), idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&tfull[s]);
+        }
+        umma_commit(qempty);
+        ++commits;
+        g += nt;
+        if (!good) break;
+      }
+      // every UMMA issued has completed before the TMEM is released
+      if (commits > 0) mbar_drain(qempty, (commits - 1) & 1);
+    }
+  } else {
+    // ------------------------------------------- candidate build + top-k (5-8)
+    const SubGrp128 grp{160, 2};
+    const int et = threadIdx.x - 160;
+    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(bg);
+    int32_t* pref = reinterpret_cast<int32_t*>(bg + static_cast<size_t>(kSortCap) * 8);
+    P3Smem& ps = *reinterpret_cast<P3Smem*>(bg);
+    auto build = [&](int q) {
+      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const int64_t t = a.pos0 + qi;
+      int nC;
+      int64_t n_v;
+      version_of(vt, t, &nC, &n_v);
+      int32_t* cl = rows + static_cast<int64_t>(q & 1) * a.C;
+      const int n = build_candidates<true>(a, qi, t, nC, n_v, cl, sortbuf, pref, grp);
+      if (a.cand_out) {
+        for (int i = et; i < a.C; i += 128) a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cl[i] : -1;
+      }
+      if (et == 0) meta[q & 1] = n;
+      mbar_arrive(&cready[q & 1]);  // after this thread's own list stores
+    };
+    if (nq > 0) build(0);
+    for (int q = 0; q < nq; ++q) {
+      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      if (q + 1 < nq) build(q + 1);
+      const bool ok = mbar_wait(&sready[q & 1], (q >> 1) & 1, a.err, abort_flag);
+      if (!named_bar_and(1, 128, ok)) break;
+      tc_fence_after();
+      const int quarter = warp & 3;
+      P3Ctx c;
+      c.row = quarter * 32 + lane;
+      c.tcol = tmem_base + 2 * H + (q & 1) * sc_cols + (static_cast<uint32_t>(quarter * 32) << 16);
+      c.n = meta[q & 1];
+      c.ntiles = (c.n + kTile - 1) / kTile;
+      c.cand = rows + static_cast<int64_t>(q & 1) * a.C;
+      p3_topk(a, qi, c, et, ps);
+      tc_fence_before();
+      mbar_arrive(&sfree[q & 1]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tcols);
+  }
+}
+
 }  // namespace
 
 size_t refine_smem_bytes(int C, int H, int d, bool tc) {
@@ -1031,35 +1353,56 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
   if (tc) {
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
+    if (a.H != 32 && a.H != 64) return cudaErrorInvalidValue;
     // CTAs per SM bounded by shared memory (228 KiB per SM, 1 KiB reserved
     // per CTA; the carveout is set to the maximum), by TMEM (512 columns)
-    // and by the registers; the list stays in shared memory unless that
-    // costs the second CTA
-    auto per_sm_for = [&](size_t sm) {
+    // and by the registers
+    auto per_sm_for = [&](size_t sm, int cols) {
       int p = static_cast<int>((228 * 1024) / (sm + 1024));
-      const int tm = 512 / tc_tmem_cols(a.C, a.H);
+      const int tm = 512 / cols;
       p = p < tm ? p : tm;
       p = p < kTcCtasPerSm ? p : kTcCtasPerSm;
       return p < 1 ? 1 : p;
     };
-    const size_t sm_local = tc_smem_bytes(a.C, a.H, false);
-    const bool gc = !(sm_local <= 227 * 1024 && per_sm_for(sm_local) >= kTcCtasPerSm) && a.cand_scratch != nullptr;
-    const size_t smem = gc ? tc_smem_bytes(a.C, a.H, true) : sm_local;
-    if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    const int per_sm = per_sm_for(smem);
+    const size_t sm_local = tc_smem_bytes(a.C, a.H, false), sm_glob = tc_smem_bytes(a.C, a.H, true);
+    const size_t sm_pipe = pipe_smem_bytes(a.H);
+    const int tm_seq = tc_tmem_cols(a.C, a.H), tm_pipe = pipe_tmem_cols(a.C, a.H);
+    constexpr size_t kMaxSmem = 227 * 1024;
+    // the pipelined kernel where it keeps two CTAs per SM; else the
+    // block-sequential one, its list in shared memory unless that costs
+    // the second CTA
+    int kind = a.refine_kernel;
+    if (kind == REFINE_AUTO) {
+      if (a.cand_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, tm_pipe) >= kTcCtasPerSm)
+        kind = REFINE_PIPE;
+      else if (sm_local <= kMaxSmem && per_sm_for(sm_local, tm_seq) >= kTcCtasPerSm)
+        kind = REFINE_SEQ_SMEM;
+      else
+        kind = a.cand_scratch ? REFINE_SEQ_GLOBAL : REFINE_SEQ_SMEM;
+    }
+    if ((kind == REFINE_SEQ_GLOBAL || kind == REFINE_PIPE) && !a.cand_scratch) return cudaErrorInvalidValue;
+    if (kind != REFINE_SEQ_SMEM && kind != REFINE_SEQ_GLOBAL && kind != REFINE_PIPE) return cudaErrorInvalidValue;
+    const size_t smem = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
+    if (smem > kMaxSmem || (kind == REFINE_PIPE ? tm_pipe : tm_seq) > 512) return cudaErrorInvalidValue;
+    const int per_sm = per_sm_for(smem, kind == REFINE_PIPE ? tm_pipe : tm_seq);
     const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
-#define AI_LAUNCH_REFINE(HH, GC)                                                                         \
+    if (grid <= 0) return cudaSuccess;
+#define AI_LAUNCH_REFINE(KERNEL)                                                                         \
   do {                                                                                                   \
-    cudaFuncSetAttribute(k_refine_tc<HH, GC>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
-    cudaFuncSetAttribute(k_refine_tc<HH, GC>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);      \
+    cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));   \
+    cudaFuncSetAttribute(KERNEL, cudaFuncAttributePreferredSharedMemoryCarveout, 100);                   \
     count_launch();                                                                                      \
-    k_refine_tc<HH, GC><<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);                           \
+    KERNEL<<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);                                         \
   } while (0)
-    if (a.H == 32 && gc) AI_LAUNCH_REFINE(32, true);
-    else if (a.H == 32) AI_LAUNCH_REFINE(32, false);
-    else if (a.H == 64 && gc) AI_LAUNCH_REFINE(64, true);
-    else if (a.H == 64) AI_LAUNCH_REFINE(64, false);
-    else return cudaErrorInvalidValue;
+    if (a.H == 32) {
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE(k_refine_pipe<32>);
+      else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<32, true>));
+      else AI_LAUNCH_REFINE((k_refine_tc<32, false>));
+    } else {
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE(k_refine_pipe<64>);
+      else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<64, true>));
+      else AI_LAUNCH_REFINE((k_refine_tc<64, false>));
+    }
 #undef AI_LAUNCH_REFINE
   } else {
     cudaFuncSetAttribute(k_refine_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -19,11 +19,14 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 
 def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_refit=True,
-                 seed_q=0):
+                 seed_q=0, refine_kernel=0):
     """Chunked prefill on both sides; compare index state after every chunk
     and route+refine / exhaustive results on (sampled) queries.
-    check_exhaustive: True, False, or the set of chunk indices to check."""
+    check_exhaustive: True, False, or the set of chunk indices to check.
+    refine_kernel: tensor-core refine variant to force (0 = automatic)."""
     gpu, orc = P.make_pair(wl, encoder=encoder, async_refit=async_refit)
+    if refine_kernel:
+        gpu.debug_refine_kernel(refine_kernel)
     rng = np.random.default_rng(1234 + seed_q)
     stats = collections.Counter()
     for c in range(wl.n_chunks):
@@ -84,18 +87,57 @@ def test_tiny_fp32_full_prefill_every_query():
     assert st["cand_near_tie"] <= 0.01 * wl.L, st
 
 
-def test_glm_bf16_scaled_sampled():
+# refine variants: 1 / 2 = one query per CTA (list in shared / global
+# memory), 3 = pipelined build / rescore / top-k
+@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3])
+def test_glm_bf16_scaled_sampled(refine_kernel):
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=20480, T=2048, refit_period=8192,
                   budget=3000, k=256, M=256)
-    st = _run_prefill(wl, sample=48)
+    st = _run_prefill(wl, sample=48, refine_kernel=refine_kernel,
+                      check_exhaustive=True if refine_kernel == 0 else False)
     assert st["cand_near_tie"] <= 0.02 * (st["cand_equal"] + st["cand_near_tie"]), st
 
 
-def test_v4flash_fp8_scaled_sampled():
+@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3])
+def test_v4flash_fp8_scaled_sampled(refine_kernel):
     wl = S.scaled(S.WORKLOADS["v4flash_fp8_L256k"], L=12288, T=2048, refit_period=4096,
                   budget=2500, k=200, M=256)
-    st = _run_prefill(wl, sample=32)
+    st = _run_prefill(wl, sample=32, refine_kernel=refine_kernel,
+                      check_exhaustive=True if refine_kernel == 0 else False)
     assert st["cand_equal"] > 0, st
+
+
+def test_refine_variants_agree_bitwise():
+    """The three tensor-core refine kernels return identical ids and scores
+    (same arithmetic in the same order), over ragged query counts that
+    leave CTAs with different numbers of queries, and a chunk whose first
+    queries have short lists."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=6144, T=2048, refit_period=4096,
+                  budget=1000, k=100, M=128)
+    gpu, _ = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        p0, p1 = c * wl.T, (c + 1) * wl.T
+        kd, ks, _ = P.keys_inputs(wl, p0, p1)
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+    for T in (1, 7, 300, 2048):
+        p0 = wl.L - T
+        qd, wd, _, _ = P.query_inputs(wl, p0, wl.L)
+        res = []
+        for kern in (1, 2, 3):
+            gpu.debug_refine_kernel(kern)
+            out = torch.full((T, wl.k), -7, dtype=torch.int32, device="cuda")
+            osc = torch.zeros((T, wl.k), dtype=torch.float32, device="cuda")
+            gpu.route_refine(qd, wd, p0, wl.k, wl.budget, out=out, out_scores=osc)
+            cand, _ = gpu.debug_candidates(qd, wd, p0, wl.budget, with_scores=False)
+            gpu.sync()
+            res.append((out.cpu().numpy(), osc.cpu().numpy(), cand.cpu().numpy()))
+        for kern, r in zip((2, 3), res[1:]):
+            assert np.array_equal(r[2], res[0][2]), f"candidates differ: kernel {kern}, T={T}"
+            assert np.array_equal(r[0], res[0][0]), f"ids differ: kernel {kern}, T={T}"
+            assert np.array_equal(r[1].view(np.uint32), res[0][1].view(np.uint32)), \
+                f"scores differ: kernel {kern}, T={T}"
+    gpu.close()
 
 
 def test_synchronous_refit_matches_oracle():
