@@ -336,7 +336,11 @@ def run_ours(args):
         ach = refine_bytes / avg / 1e9
         traffic = traffic_from_profile(os.path.join(ROOT, "ivf_top_key_b200", "csrc", "route_refine.cu"),
                                        os.path.join(ROOT, "profiles", f"refine_{wl.name}.md"))
-        roofline = {"kernel": "k_refine_tc (candidate fill + gathered rescore + top-k)",
+        kname = {0: "k_refine_simt", 1: "k_refine_tc (list in shared memory)",
+                 2: "k_refine_tc (list in global scratch)",
+                 3: "k_refine_pipe (warp-specialised: build / gather + rescore / top-k overlapped)"}[
+            idx.refine_kernel_choice(wl.budget)]
+        roofline = {"kernel": kname,
                     "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",

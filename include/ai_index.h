@@ -118,8 +118,10 @@ int ai_publish(ai_handle h);
  * fills C candidate slots with the sinks, the open window [n_v, t] and
  * whole member lists in rank order (score desc, cluster id asc; the last
  * list is truncated), rescores the candidates exactly and writes the top k
- * ids by (score desc, id asc) to out_dev[T, k] in candidate order, padded
- * with -1.  q_dev: [T, H, d] in q_dtype; w_dev: [T, H] float32;
+ * ids by (score desc, id asc) to out_dev[T, k], padded with -1.  Their
+ * order follows the candidate slots s: ascending s on the fp32 path, and
+ * ascending (s mod 128, s div 128) on the tensor-core path (bf16 / fp8
+ * keys), the same for every kernel variant.  q_dev: [T, H, d] in q_dtype; w_dev: [T, H] float32;
  * out_scores_dev: [T, k] float32 or NULL.  Errors: AI_ERR_ARG (T, k, C
  * beyond the create-time maxima), AI_ERR_CAUSALITY (pos0 + T - 1 >=
  * appended keys).                                                          */
@@ -239,6 +241,13 @@ int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_
  * configuration makes those calls fail with AI_ERR_CUDA.  Returns AI_OK,
  * or AI_ERR_ARG for a null handle or a kernel outside 0..3.              */
 int ai_debug_refine_kernel(ai_handle h, int32_t kernel);
+
+/* The refine kernel ai_route_refine launches on h for budget C:
+ * *kernel_out = 0 for the fp32 (SIMT) path, else the tensor-core variant
+ * as numbered for ai_debug_refine_kernel (1, 2 or 3; the forced one if
+ * set).  Host-only: launches nothing.  AI_ERR_ARG for a null argument or
+ * C outside 1 .. max_budget.                                              */
+int ai_refine_kernel_choice(ai_handle h, int32_t C, int32_t* kernel_out);
 
 /* ------------------------------------------------- failure-path test hook */
 /* Runs the library's bounded wait against a barrier that nothing completes

@@ -112,6 +112,11 @@ class AttentionIndex:
         pipelined); every variant computes the same result."""
         C.ai_debug_refine_kernel(self.h, kernel)
 
+    def refine_kernel_choice(self, C_budget: int) -> int:
+        """The refine kernel route_refine launches for this budget (0 = fp32
+        SIMT path, 1 / 2 = one query per CTA, 3 = pipelined)."""
+        return C.ai_refine_kernel_choice(self.h, C_budget)
+
     def profile(self, enable: bool = True):
         C.ai_profile_enable(self.h, enable)
 

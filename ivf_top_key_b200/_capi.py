@@ -30,7 +30,7 @@ EXPORTED = [
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
     "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
-    "ai_debug_refine_kernel",
+    "ai_debug_refine_kernel", "ai_refine_kernel_choice",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
 
@@ -88,6 +88,7 @@ def _load():
         "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp],
         "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
         "ai_debug_refine_kernel": [vp, i32],
+        "ai_refine_kernel_choice": [vp, i32, ctypes.POINTER(i32)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -254,6 +255,14 @@ def ai_debug_refine_kernel(h, kernel: int):
     """Select the tensor-core refine variant (0 auto, 1 sequential with the
     list in shared memory, 2 sequential with a global list, 3 pipelined)."""
     _check(_lib.ai_debug_refine_kernel(h, kernel))
+
+
+def ai_refine_kernel_choice(h, C: int) -> int:
+    """Refine kernel the library launches for budget C (0 = fp32 SIMT path,
+    1 / 2 = one query per CTA, 3 = pipelined)."""
+    v = ctypes.c_int32()
+    _check(_lib.ai_refine_kernel_choice(h, C, ctypes.byref(v)))
+    return v.value
 
 
 def ai_last_error() -> str:

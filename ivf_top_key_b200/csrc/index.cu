@@ -1091,6 +1091,18 @@ int ai_debug_refine_kernel(ai_handle h, int32_t kernel) {
   return AI_OK;
 }
 
+int ai_refine_kernel_choice(ai_handle h, int32_t C, int32_t* kernel_out) {
+  if (!h || !kernel_out) return fail(AI_ERR_ARG, "null handle or output");
+  if (C <= 0 || C > h->cfg.max_budget) return fail(AI_ERR_ARG, "C out of range");
+  if (!tc_keys(h)) {
+    *kernel_out = 0;
+  } else {
+    *kernel_out = h->refine_kernel != REFINE_AUTO ? h->refine_kernel
+                                                 : pick_refine_kernel(C, h->cfg.H, h->cand_scratch != nullptr);
+  }
+  return AI_OK;
+}
+
 int ai_profile_enable(ai_handle h, int enable) {
   if (!h) return fail(AI_ERR_ARG, "null handle");
   h->prof = enable != 0;

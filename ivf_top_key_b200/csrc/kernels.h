@@ -68,6 +68,8 @@ struct RefineArgs {
   int* err;
 };
 enum RefineKernel { REFINE_AUTO = 0, REFINE_SEQ_SMEM = 1, REFINE_SEQ_GLOBAL = 2, REFINE_PIPE = 3 };
+// The variant REFINE_AUTO launches for budget C and H heads (tensor-core path).
+int pick_refine_kernel(int C, int H, bool has_scratch);
 size_t refine_smem_bytes(int C, int H, int d, bool tc);
 // kmap: TMA map of the bf16 key store (box 64 x 1); qmap: TMA map of the
 // queries as [T*H, 128] bf16 rows (box 64 x H).  Both nullptr selects the

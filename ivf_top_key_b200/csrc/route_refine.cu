@@ -843,6 +843,32 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   named_bar(1, 128);
 }
 
+// Indexer score of one candidate row from its H head dot products in TMEM
+// (columns acc .. acc + H - 1 of this thread's lane): sum_h w_h ReLU(dot_h).
+// Four interleaved partial sums (head h goes to sum h mod 4, combined as
+// (s0 + s1) + (s2 + s3)) keep the dependent chain short; every tensor-core
+// kernel uses this same order, so their scores agree bit for bit.  The
+// weights are read four at a time from shared memory (16-byte aligned).
+template <int H>
+__device__ __forceinline__ float head_sum(uint32_t acc, const float* wsh) {
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < H / 32; ++c) {
+    float v[32];
+    tmem_ld32(acc + c * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int h4 = 0; h4 < 8; ++h4) {
+      const float4 w4 = reinterpret_cast<const float4*>(wsh)[c * 8 + h4];
+      s[0] = fmaf(w4.x, fmaxf(v[4 * h4 + 0], 0.f), s[0]);
+      s[1] = fmaf(w4.y, fmaxf(v[4 * h4 + 1], 0.f), s[1]);
+      s[2] = fmaf(w4.z, fmaxf(v[4 * h4 + 2], 0.f), s[2]);
+      s[3] = fmaf(w4.w, fmaxf(v[4 * h4 + 3], 0.f), s[3]);
+    }
+  }
+  return (s[0] + s[1]) + (s[2] + s[3]);
+}
+
 // Layout of the tensor-core kernel (one region reused by the three phases).
 constexpr int kStages2 = 2;
 __host__ __device__ inline size_t tc_region_bytes() {
@@ -1012,15 +1038,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         const int acc = gj & 1;
         if (!mbar_wait(&tfull[acc], (gj >> 1) & 1, a.err, abort_flag)) break;
         tc_fence_after();
-        float sc = 0.f;
-#pragma unroll
-        for (int c = 0; c < H / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem_base + acc * H + c * 32 + lane_off, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc = fmaf(wsh[c * 32 + h], fmaxf(v[h], 0.f), sc);
-        }
+        float sc = head_sum<H>(tmem_base + acc * H + lane_off, wsh);
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
         const int slot = j * kTile + row;
@@ -1042,7 +1060,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       c.ntiles = ntiles;
       c.n = n;
       c.cand = cand;
-      p3_topk(a, qi, c, threadIdx.x - 160, ps);
+      p3_topk(a, qi, c, c.row, ps);  // threads ordered by row: the emission order
     }
     __syncthreads();
   }
@@ -1056,11 +1074,20 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
 
 // ------------------------------------------------- pipelined tcgen05 kernel
 // The three phases of consecutive queries overlap inside one CTA:
-//   warps 0-3  gather the candidate rows of query i (TMA gather4) and run
-//              the epilogue (ReLU, head weights) into TMEM score columns
-//   warp 4     loads query i's head tile and issues the UMMAs
-//   warps 5-8  build the candidate list of query i+1, then select the
-//              top-k of query i-1 from its score columns
+//   warps 0-3   gather candidate rows of query i (TMA gather4) and run the
+//               epilogue (ReLU, head weights) into TMEM score columns
+//   warps 4-7   build the candidate list of query i+1, then select the
+//               top-k of query i-1 from its score columns
+//   warps 8-11  (NGW = 8 only) gather rows
+//   last warp   loads query i's head tile and issues the UMMAs
+// Gather throughput grows with the number of warps issuing gather4
+// (each warp's ops are issued one after another), so NGW = 8 splits a
+// tile's 128 rows over eight warps, 16 rows each.  The roles sit on
+// warpgroup boundaries so that, with NGW = 8, the gather-only warpgroup
+// hands registers to the build / top-k warpgroup (setmaxnreg): launched
+// at 72 per thread, 416 threads hold 29,952; afterwards 128 x 72
+// (gather + epilogue) + 128 x 96 (build / top-k) + 128 x 40 (gather only)
+// + 32 x 72 (UMMA) = 28,928 are in use.
 // Candidate lists live in two global scratch rows per CTA and score
 // columns in two TMEM buffers, so the build and the top-k of neighbouring
 // queries run while the gather of query i keeps the copy engine busy.
@@ -1077,6 +1104,13 @@ __host__ __device__ inline size_t pipe_bg_bytes() {
   return align_up(p1 > p3 ? p1 : p3, 16);
 }
 constexpr int kPipeBars = 14;
+// Gathering warps of the pipelined kernel (4 or 8).  Eight measured
+// slower on B200 (128K bf16: 2.21M vs 2.40M query tokens/s): the SM's
+// gather4 throughput, not the issuing warps, bounds the rescore there.
+#ifndef AI_PIPE_NGW
+#define AI_PIPE_NGW 4
+#endif
+constexpr int kPipeNgw = AI_PIPE_NGW;
 __host__ __device__ inline size_t pipe_smem_bytes(int H) {
   return kTcSlack + static_cast<size_t>(kStages2) * kTile * 256 + static_cast<size_t>(H) * 256 + pipe_bg_bytes() +
          align_up(static_cast<size_t>(H) * 4, 16) + 16 + kPipeBars * 8 + 8;
@@ -1089,8 +1123,17 @@ __host__ __device__ inline int pipe_tmem_cols(int C, int H) {
   return cols;
 }
 
-template <int H>
-__global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
+constexpr int pipe_threads(int ngw) { return kTcThreads + (ngw - 4) * 32; }
+constexpr int kPipeRegsLaunch = 72, kPipeRegsBuild = 96, kPipeRegsGather = 40;
+static_assert(128 * kPipeRegsLaunch + 128 * kPipeRegsBuild + 128 * kPipeRegsGather + 32 * kPipeRegsLaunch <=
+                  416 * kPipeRegsLaunch,
+              "register split above the launch allocation");
+static_assert(65536 / (2 * 416) / 8 * 8 == kPipeRegsLaunch, "launch allocation of the NGW = 8 kernel");
+__device__ __forceinline__ void regs_inc96() { asm volatile("setmaxnreg.inc.sync.aligned.u32 96;\n" ::: "memory"); }
+__device__ __forceinline__ void regs_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory"); }
+
+template <int H, int NGW>
+__global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     k_refine_pipe(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                   RefineArgs a, VersionTable vt) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1116,13 +1159,14 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kPipeBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kMmaWarp = NGW + 4;
   const int tcols = pipe_tmem_cols(a.C, H);
   const int sc_cols = pipe_sc_cols(a.C);
   int32_t* rows = a.cand_scratch + static_cast<int64_t>(2 * blockIdx.x) * a.C;  // this CTA's two lists
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&full[i], 4);  // one arrive.expect_tx per gathering warp
+      mbar_init(&full[i], NGW);  // one arrive.expect_tx per gathering warp
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 128);
       mbar_init(&cready[i], 128);
@@ -1134,7 +1178,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, tcols);
     tmem_relinquish();
   }
@@ -1143,6 +1187,35 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int nq = static_cast<int>(blockIdx.x) < a.T ? (a.T - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+
+  // Gathering warp gw (0 .. NGW-1) owns rows [gw * RPW, gw * RPW + RPW) of
+  // every tile; lane l holds the id of row gw * RPW + l % RPW and lanes
+  // below 2 * RPW / 4 issue one gather4 (4 rows, one 64-column half) each.
+  constexpr int RPW = kTile / NGW;
+  constexpr int GPH = RPW / 4;  // gather4 ops per half
+  auto next_gid = [&](int j, int gw, int n, const int32_t* cl) -> int {
+    const int slot = (j + 1) * kTile + gw * RPW + lane % RPW;
+    return slot < n ? cl[slot] : 0;
+  };
+  auto issue_rows = [&](uint32_t gj, int j, int gid, int gw, int n, int64_t t, const int32_t* cl) {
+    (void)cl;
+    int id = gid;
+    if (j * kTile + gw * RPW + lane % RPW < n && (id < 0 || id > t)) {
+      atomicOr(a.err, DEV_ERR_RANGE);
+      id = 0;
+    }
+    int r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, id, ((lane % GPH) * 4 + i) % RPW);
+    if (lane == 0) mbar_arrive_expect_tx(&full[gj & 1], kTile * 256 / NGW);
+    __syncwarp();
+    if (lane < 2 * GPH) {
+      const int half = lane / GPH;
+      const int rl = gw * RPW + (lane % GPH) * 4;
+      uint8_t* dst = stages + (gj & 1) * (kTile * 256) + half * (kTile * 128) + rl * 128;
+      tma_gather4(dst, &kmap, half * 64, r[0], r[1], r[2], r[3], &full[gj & 1]);
+    }
+  };
 
   if (warp < 4) {
     // --------------------------------------------- gather + epilogue (0-3)
@@ -1168,7 +1241,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       for (int h = row; h < H; h += 128) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
       named_bar(3, 128);
       const uint32_t scol = tmem_base + 2 * H + b * sc_cols + lane_off;
-      int myid = row < n ? cl[row] : 0;  // this thread's row of tile 0
+      int myid = fp8 && row < n ? cl[row] : 0;  // this thread's epilogue row of tile 0 (fp8 scale)
+      int gid = next_gid(-1, warp, n, cl);      // this lane's gather row of tile 0
       float sc0 = 1.f, sc1 = 1.f;          // fp8 scales of the tiles in flight (by tile parity)
       // iteration j issues tile j and finishes the epilogue of tile j-2
       auto step = [&](int j, float& s_slot) -> bool {
@@ -1183,38 +1257,20 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         }
         const float s_ep = s_slot;  // scale of tile j-2
         if (j < nt) {
-          int id = myid;
-          if (row + j * kTile < n && (id < 0 || id > t)) {
-            atomicOr(a.err, DEV_ERR_RANGE);
-            id = 0;
-          }
-          int r[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, id, (lane & 7) * 4 + i);
-          if (lane == 0) mbar_arrive_expect_tx(&full[gj & 1], kTile * 256 / 4);
-          __syncwarp();
-          if (lane < 16) {
-            const int half = lane >> 3;
-            const int rl = warp * 32 + (lane & 7) * 4;
-            uint8_t* dst = stages + (gj & 1) * (kTile * 256) + half * (kTile * 128) + rl * 128;
-            tma_gather4(dst, &kmap, half * 64, r[0], r[1], r[2], r[3], &full[gj & 1]);
-          }
+          issue_rows(gj, j, gid, warp, n, t, cl);
           last_issued = gj;
-          // consumed two iterations later: the loads stay in flight
-          s_slot = fp8 ? a.key_scale[id] : 1.f;
-          const int nslot = (j + 1) * kTile + row;
-          myid = (j + 1 < nt && nslot < n) ? cl[nslot] : 0;
+          if (fp8) {
+            // consumed two iterations later: the load stays in flight
+            int id = myid;
+            if (row + j * kTile >= n || id < 0 || id > t) id = 0;
+            s_slot = a.key_scale[id];
+            const int nslot = (j + 1) * kTile + row;
+            myid = (j + 1 < nt && nslot < n) ? cl[nslot] : 0;
+          }
+          gid = next_gid(j, warp, n, cl);
         }
         if (j >= 2) {
-          float sc = 0.f;
-#pragma unroll
-          for (int c = 0; c < H / 32; ++c) {
-            float v[32];
-            tmem_ld32(tmem_base + acc * H + c * 32 + lane_off, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int h = 0; h < 32; ++h) sc = fmaf(wsh[c * 32 + h], fmaxf(v[h], 0.f), sc);
-          }
+          float sc = head_sum<H>(tmem_base + acc * H + lane_off, wsh);
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
           tmem_st1(scol + (j - 2), sc * s_ep);
@@ -1240,8 +1296,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       for (int64_t e = last_issued > 0 ? last_issued - 1 : 0; e <= last_issued; ++e)
         mbar_drain(&full[e & 1], (e >> 1) & 1);
     }
-  } else if (warp == 4) {
-    // ------------------------------------------------------ UMMA issue (4)
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------- UMMA issue
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTile, H);
       const uint32_t sb = smem_u32(qtile);
@@ -1288,10 +1344,49 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       // every UMMA issued has completed before the TMEM is released
       if (commits > 0) mbar_drain(qempty, (commits - 1) & 1);
     }
+  } else if (warp >= 8) {
+    // ------------------------------------------------ gather only (8-11)
+    if (NGW == 8) regs_dec40();
+    const int gw = warp - 4;
+    uint32_t g = 0;
+    int64_t last_issued = -1;
+    for (int q = 0; q < nq; ++q) {
+      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const int64_t t = a.pos0 + qi;
+      const int b = q & 1;
+      const bool ok = mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int n = meta[b];
+      const int nt = (n + kTile - 1) / kTile;
+      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C;
+      int gid = next_gid(-1, gw, n, cl);
+      bool good = true;
+      for (int j = 0; j < nt; ++j) {
+        const uint32_t gj = g + j;
+        if (gj >= 2) {
+          // stage gj & 1 is free once the UMMAs of tile gj - 2 are done
+          const bool w = mbar_wait(&tfull[gj & 1], ((gj - 2) >> 1) & 1, a.err, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) {
+            good = false;
+            break;
+          }
+        }
+        issue_rows(gj, j, gid, gw, n, t, cl);
+        last_issued = gj;
+        gid = next_gid(j, gw, n, cl);
+      }
+      if (!good) break;
+      g += nt;
+    }
+    if (*abort_flag && lane == 0 && last_issued >= 0) {
+      for (int64_t e = last_issued > 0 ? last_issued - 1 : 0; e <= last_issued; ++e)
+        mbar_drain(&full[e & 1], (e >> 1) & 1);
+    }
   } else {
-    // ------------------------------------------- candidate build + top-k (5-8)
-    const SubGrp128 grp{160, 2};
-    const int et = threadIdx.x - 160;
+    // ------------------------------------------- candidate build + top-k (4-7)
+    if (NGW == 8) regs_inc96();
+    const SubGrp128 grp{128, 2};
+    const int et = threadIdx.x - 128;
     uint64_t* sortbuf = reinterpret_cast<uint64_t*>(bg);
     int32_t* pref = reinterpret_cast<int32_t*>(bg + static_cast<size_t>(kSortCap) * 8);
     P3Smem& ps = *reinterpret_cast<P3Smem*>(bg);
@@ -1323,20 +1418,43 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       c.n = meta[q & 1];
       c.ntiles = (c.n + kTile - 1) / kTile;
       c.cand = rows + static_cast<int64_t>(q & 1) * a.C;
-      p3_topk(a, qi, c, et, ps);
+      p3_topk(a, qi, c, c.row, ps);  // c.row == et: rows in thread order
       tc_fence_before();
       mbar_arrive(&sfree[q & 1]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tcols);
   }
 }
 
+// CTAs per SM of a tensor-core refine launch: bounded by shared memory
+// (228 KiB per SM, 1 KiB reserved per CTA; the carveout is set to the
+// maximum), by TMEM (512 columns) and by the registers.
+int per_sm_for(size_t smem, int tmem_cols) {
+  int p = static_cast<int>((228 * 1024) / (smem + 1024));
+  const int tm = 512 / tmem_cols;
+  p = p < tm ? p : tm;
+  p = p < kTcCtasPerSm ? p : kTcCtasPerSm;
+  return p < 1 ? 1 : p;
+}
+
 }  // namespace
+
+int pick_refine_kernel(int C, int H, bool has_scratch) {
+  // the pipelined kernel where it keeps two CTAs per SM; else the
+  // block-sequential one, its list in shared memory unless that costs the
+  // second CTA
+  constexpr size_t kMaxSmem = 227 * 1024;
+  const size_t sm_local = tc_smem_bytes(C, H, false), sm_pipe = pipe_smem_bytes(H);
+  if (has_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, pipe_tmem_cols(C, H)) >= kTcCtasPerSm)
+    return REFINE_PIPE;
+  if (sm_local <= kMaxSmem && per_sm_for(sm_local, tc_tmem_cols(C, H)) >= kTcCtasPerSm) return REFINE_SEQ_SMEM;
+  return has_scratch ? REFINE_SEQ_GLOBAL : REFINE_SEQ_SMEM;
+}
 
 size_t refine_smem_bytes(int C, int H, int d, bool tc) {
   if (tc) return tc_smem_bytes(C, H, true);  // the smaller layout; the launch picks
@@ -1354,32 +1472,12 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
     if (a.H != 32 && a.H != 64) return cudaErrorInvalidValue;
-    // CTAs per SM bounded by shared memory (228 KiB per SM, 1 KiB reserved
-    // per CTA; the carveout is set to the maximum), by TMEM (512 columns)
-    // and by the registers
-    auto per_sm_for = [&](size_t sm, int cols) {
-      int p = static_cast<int>((228 * 1024) / (sm + 1024));
-      const int tm = 512 / cols;
-      p = p < tm ? p : tm;
-      p = p < kTcCtasPerSm ? p : kTcCtasPerSm;
-      return p < 1 ? 1 : p;
-    };
     const size_t sm_local = tc_smem_bytes(a.C, a.H, false), sm_glob = tc_smem_bytes(a.C, a.H, true);
     const size_t sm_pipe = pipe_smem_bytes(a.H);
     const int tm_seq = tc_tmem_cols(a.C, a.H), tm_pipe = pipe_tmem_cols(a.C, a.H);
     constexpr size_t kMaxSmem = 227 * 1024;
-    // the pipelined kernel where it keeps two CTAs per SM; else the
-    // block-sequential one, its list in shared memory unless that costs
-    // the second CTA
-    int kind = a.refine_kernel;
-    if (kind == REFINE_AUTO) {
-      if (a.cand_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, tm_pipe) >= kTcCtasPerSm)
-        kind = REFINE_PIPE;
-      else if (sm_local <= kMaxSmem && per_sm_for(sm_local, tm_seq) >= kTcCtasPerSm)
-        kind = REFINE_SEQ_SMEM;
-      else
-        kind = a.cand_scratch ? REFINE_SEQ_GLOBAL : REFINE_SEQ_SMEM;
-    }
+    const int kind = a.refine_kernel == REFINE_AUTO ? pick_refine_kernel(a.C, a.H, a.cand_scratch != nullptr)
+                                                    : a.refine_kernel;
     if ((kind == REFINE_SEQ_GLOBAL || kind == REFINE_PIPE) && !a.cand_scratch) return cudaErrorInvalidValue;
     if (kind != REFINE_SEQ_SMEM && kind != REFINE_SEQ_GLOBAL && kind != REFINE_PIPE) return cudaErrorInvalidValue;
     const size_t smem = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
@@ -1392,14 +1490,14 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));   \
     cudaFuncSetAttribute(KERNEL, cudaFuncAttributePreferredSharedMemoryCarveout, 100);                   \
     count_launch();                                                                                      \
-    KERNEL<<<grid, kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);                                         \
+    KERNEL<<<grid, kind == REFINE_PIPE ? pipe_threads(kPipeNgw) : kTcThreads, smem, st>>>(*kmap, *qmap, a, vt); \
   } while (0)
     if (a.H == 32) {
-      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE(k_refine_pipe<32>);
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<32, kPipeNgw>));
       else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<32, true>));
       else AI_LAUNCH_REFINE((k_refine_tc<32, false>));
     } else {
-      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE(k_refine_pipe<64>);
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<64, kPipeNgw>));
       else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<64, true>));
       else AI_LAUNCH_REFINE((k_refine_tc<64, false>));
     }

@@ -105,8 +105,17 @@ def check_index_equal(gpu, orc):
 
 # ----------------------------------------------------------- query checks --
 
-def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats):
-    """Compare route+refine results of the listed queries with the oracle."""
+def output_order_key(slots, tile_order):
+    """Sort key of the documented output order: ascending candidate slot s
+    (fp32 path), or ascending (s mod 128, s div 128) (tensor-core path)."""
+    slots = np.asarray(slots, dtype=np.int64)
+    return (slots % 128) * (1 << 32) + slots // 128 if tile_order else slots
+
+
+def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats, tile_order=None):
+    """Compare route+refine results of the listed queries with the oracle.
+    tile_order: True / False checks the documented output order (tensor-core
+    / fp32 path) against the GPU's own candidate list; None skips it."""
     for i, t in enumerate(t_list):
         qi, wi = q[i], w[i]
         o_cand, rs, v = orc.candidates(t, qi, wi, C)
@@ -115,6 +124,10 @@ def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats)
         valid = g_ids[g_ids >= 0]
         assert np.all(valid <= t), f"t={t}: selected a future key"
         assert len(set(valid.tolist())) == valid.size, f"t={t}: duplicate ids"
+        if tile_order is not None and valid.size:
+            slot_of = {int(s): j for j, s in enumerate(g_cand.tolist())}
+            key = output_order_key([slot_of[int(s)] for s in valid.tolist()], tile_order)
+            assert np.all(np.diff(key) > 0), f"t={t}: output order"
         # scores of the selected ids agree with float64
         exact = O.indexer_score(qi, wi, orc.keys[valid])
         tol = score_tol(qi, wi, orc.keys[valid])

@@ -165,7 +165,8 @@ def test_glm_bf16_L1m_sampled_steps():
     idx = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, size=8, replace=False)]))
     stats = collections.Counter()
     P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], out.cpu().numpy()[idx],
-                    osc.cpu().numpy()[idx], cand.cpu().numpy()[idx], wl.k, wl.budget, stats)
+                    osc.cpu().numpy()[idx], cand.cpu().numpy()[idx], wl.k, wl.budget, stats,
+                    tile_order=wl.key_dtype != "fp32")
     eo = eo.cpu().numpy()
     for i in idx[:4]:
         t = p0 + i

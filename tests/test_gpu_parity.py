@@ -50,7 +50,7 @@ def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_
         scs = osc.cpu().numpy()[idx]
         cnd = cand.cpu().numpy()[idx]
         P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], ids, scs, cnd, wl.k,
-                        wl.budget, stats)
+                        wl.budget, stats, tile_order=wl.key_dtype != "fp32")
         if check_exhaustive is True or (check_exhaustive and c in check_exhaustive):
             eo = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
             es = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
