@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="glm_bf16_L128k", choices=sorted(S.WORKLOADS))
+    p.add_argument("--refine-kernel", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                   help="force a tensor-core refine variant (0 = the library's choice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=48, help="queries timed per oracle step")
@@ -242,6 +244,8 @@ def run_ours(args):
                          max_query_chunk=T, max_budget=wl.budget, max_k=wl.k, max_keys=L,
                          seed=wl.seed,
                          encoder_weights=S.encoder_weights(wl) if wl.encoder == "random" else None)
+    if args.refine_kernel:
+        idx.debug_refine_kernel(args.refine_kernel)
     # prefix before the timed chunks (untimed setup)
     for c in range(wl.n_chunks - ncs):
         kd, ks = chunk_keys_dev(wl, c * T, (c + 1) * T, dev)
@@ -338,7 +342,8 @@ def run_ours(args):
                                        os.path.join(ROOT, "profiles", f"refine_{wl.name}.md"))
         kname = {0: "k_refine_simt", 1: "k_refine_tc (list in shared memory)",
                  2: "k_refine_tc (list in global scratch)",
-                 3: "k_refine_pipe (warp-specialised: build / gather + rescore / top-k overlapped)"}[
+                 3: "k_refine_pipe (warp-specialised: build / gather + rescore / top-k overlapped)",
+                 4: "k_refine_pipe (warp-specialised, one TMEM score buffer)"}[
             idx.refine_kernel_choice(wl.budget)]
         roofline = {"kernel": kname,
                     "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],

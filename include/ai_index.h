@@ -237,14 +237,17 @@ int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_
  * at a time per CTA with the candidate list in shared memory, 2 = the same
  * with the list in global scratch, 3 = pipelined (the candidate build and
  * the top-k of neighbouring queries overlap the rescore of the current
- * one).  A variant whose shared memory or TMEM need does not fit the
- * configuration makes those calls fail with AI_ERR_CUDA.  Returns AI_OK,
- * or AI_ERR_ARG for a null handle or a kernel outside 0..3.              */
+ * one), 4 = pipelined with one TMEM score buffer (the epilogue's first
+ * score store waits for the previous query's top-k; the default for
+ * budgets where two buffers would cost the second CTA per SM).  A variant
+ * whose shared memory or TMEM need does not fit the configuration makes
+ * those calls fail with AI_ERR_CUDA.  Returns AI_OK, or AI_ERR_ARG for a
+ * null handle or a kernel outside 0..4.                                   */
 int ai_debug_refine_kernel(ai_handle h, int32_t kernel);
 
 /* The refine kernel ai_route_refine launches on h for budget C:
  * *kernel_out = 0 for the fp32 (SIMT) path, else the tensor-core variant
- * as numbered for ai_debug_refine_kernel (1, 2 or 3; the forced one if
+ * as numbered for ai_debug_refine_kernel (1 to 4; the forced one if
  * set).  Host-only: launches nothing.  AI_ERR_ARG for a null argument or
  * C outside 1 .. max_budget.                                              */
 int ai_refine_kernel_choice(ai_handle h, int32_t C, int32_t* kernel_out);

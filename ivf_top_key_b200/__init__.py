@@ -109,12 +109,14 @@ class AttentionIndex:
     def debug_refine_kernel(self, kernel: int):
         """Force a tensor-core refine variant (0 = by occupancy, 1 / 2 =
         one query per CTA with the list in shared / global memory, 3 =
-        pipelined); every variant computes the same result."""
+        pipelined, 4 = pipelined with one TMEM score buffer); every variant
+        computes the same result."""
         C.ai_debug_refine_kernel(self.h, kernel)
 
     def refine_kernel_choice(self, C_budget: int) -> int:
         """The refine kernel route_refine launches for this budget (0 = fp32
-        SIMT path, 1 / 2 = one query per CTA, 3 = pipelined)."""
+        SIMT path, 1 / 2 = one query per CTA, 3 / 4 = pipelined with two /
+        one score buffers)."""
         return C.ai_refine_kernel_choice(self.h, C_budget)
 
     def profile(self, enable: bool = True):

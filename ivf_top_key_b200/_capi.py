@@ -253,13 +253,15 @@ def ai_debug_wait_timeout(spin_limit: int, stream=None) -> int:
 
 def ai_debug_refine_kernel(h, kernel: int):
     """Select the tensor-core refine variant (0 auto, 1 sequential with the
-    list in shared memory, 2 sequential with a global list, 3 pipelined)."""
+    list in shared memory, 2 sequential with a global list, 3 pipelined,
+    4 pipelined with one TMEM score buffer)."""
     _check(_lib.ai_debug_refine_kernel(h, kernel))
 
 
 def ai_refine_kernel_choice(h, C: int) -> int:
     """Refine kernel the library launches for budget C (0 = fp32 SIMT path,
-    1 / 2 = one query per CTA, 3 = pipelined)."""
+    1 / 2 = one query per CTA, 3 / 4 = pipelined with two / one score
+    buffers)."""
     v = ctypes.c_int32()
     _check(_lib.ai_refine_kernel_choice(h, C, ctypes.byref(v)))
     return v.value

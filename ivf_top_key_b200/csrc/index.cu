@@ -1086,7 +1086,7 @@ int ai_rollback(ai_handle h) {
 
 int ai_debug_refine_kernel(ai_handle h, int32_t kernel) {
   if (!h) return fail(AI_ERR_ARG, "null handle");
-  if (kernel < 0 || kernel > 3) return fail(AI_ERR_ARG, "refine kernel must be 0..3");
+  if (kernel < 0 || kernel > 4) return fail(AI_ERR_ARG, "refine kernel must be 0..4");
   h->refine_kernel = kernel;
   return AI_OK;
 }

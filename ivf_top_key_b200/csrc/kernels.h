@@ -67,7 +67,13 @@ struct RefineArgs {
   int refine_kernel;         // REFINE_* (tensor-core path; AUTO picks by occupancy)
   int* err;
 };
-enum RefineKernel { REFINE_AUTO = 0, REFINE_SEQ_SMEM = 1, REFINE_SEQ_GLOBAL = 2, REFINE_PIPE = 3 };
+enum RefineKernel {
+  REFINE_AUTO = 0,        // chosen by occupancy
+  REFINE_SEQ_SMEM = 1,    // one query at a time per CTA, list in shared memory
+  REFINE_SEQ_GLOBAL = 2,  // the same, list in global scratch
+  REFINE_PIPE = 3,        // pipelined, two TMEM score buffers
+  REFINE_PIPE_1BUF = 4    // pipelined, one TMEM score buffer (large budgets)
+};
 // The variant REFINE_AUTO launches for budget C and H heads (tensor-core path).
 int pick_refine_kernel(int C, int H, bool has_scratch);
 size_t refine_smem_bytes(int C, int H, int d, bool tc);

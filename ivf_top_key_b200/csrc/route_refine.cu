@@ -1116,8 +1116,9 @@ __host__ __device__ inline size_t pipe_smem_bytes(int H) {
          align_up(static_cast<size_t>(H) * 4, 16) + 16 + kPipeBars * 8 + 8;
 }
 __host__ __device__ inline int pipe_sc_cols(int C) { return ((C + 127) / 128 + 15) / 16 * 16; }
-__host__ __device__ inline int pipe_tmem_cols(int C, int H) {
-  const int need = 2 * H + 2 * pipe_sc_cols(C);
+// TMEM columns: two H-column accumulators and nsb score buffers
+__host__ __device__ inline int pipe_tmem_cols(int C, int H, int nsb) {
+  const int need = 2 * H + nsb * pipe_sc_cols(C);
   int cols = 32;
   while (cols < need) cols <<= 1;
   return cols;
@@ -1132,7 +1133,11 @@ static_assert(65536 / (2 * 416) / 8 * 8 == kPipeRegsLaunch, "launch allocation o
 __device__ __forceinline__ void regs_inc96() { asm volatile("setmaxnreg.inc.sync.aligned.u32 96;\n" ::: "memory"); }
 __device__ __forceinline__ void regs_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory"); }
 
-template <int H, int NGW>
+// NSB score buffers: 2 lets the epilogue of query i run while the top-k of
+// query i-1 reads its columns; 1 (large budgets, where two buffers would
+// need all 512 TMEM columns) makes the epilogue's first score store wait
+// for that top-k, the gather and the build still overlapping.
+template <int H, int NGW, int NSB>
 __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     k_refine_pipe(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                   RefineArgs a, VersionTable vt) {
@@ -1160,7 +1165,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kMmaWarp = NGW + 4;
-  const int tcols = pipe_tmem_cols(a.C, H);
+  const int tcols = pipe_tmem_cols(a.C, H, NSB);
   const int sc_cols = pipe_sc_cols(a.C);
   int32_t* rows = a.cand_scratch + static_cast<int64_t>(2 * blockIdx.x) * a.C;  // this CTA's two lists
 
@@ -1229,8 +1234,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
       const int64_t t = a.pos0 + qi;
       const int b = q & 1;
-      bool ok = !dead && mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
-      if (ok && q >= 2) ok = mbar_wait(&sfree[b], ((q >> 1) & 1) ^ 1, a.err, abort_flag);
+      const bool ok = !dead && mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
       // every thread of the group takes the same way out; the barrier also
       // orders the previous query's reads of wsh before its rewrite
       if (!named_bar_and(3, 128, ok)) break;
@@ -1240,7 +1244,8 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       const int32_t* cl = rows + static_cast<int64_t>(b) * a.C;
       for (int h = row; h < H; h += 128) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
       named_bar(3, 128);
-      const uint32_t scol = tmem_base + 2 * H + b * sc_cols + lane_off;
+      const int sb = q % NSB;  // score buffer of this query
+      const uint32_t scol = tmem_base + 2 * H + sb * sc_cols + lane_off;
       int myid = fp8 && row < n ? cl[row] : 0;  // this thread's epilogue row of tile 0 (fp8 scale)
       int gid = next_gid(-1, warp, n, cl);      // this lane's gather row of tile 0
       float sc0 = 1.f, sc1 = 1.f;          // fp8 scales of the tiles in flight (by tile parity)
@@ -1268,6 +1273,13 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
             myid = (j + 1 < nt && nslot < n) ? cl[nslot] : 0;
           }
           gid = next_gid(j, warp, n, cl);
+        }
+        if (j == 2 && q >= NSB) {
+          // the first score store of this query: the top-k of query q - NSB
+          // has finished reading the buffer
+          const bool w = mbar_wait(&sfree[sb], ((q - NSB) / NSB) & 1, a.err, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) return false;
+          tc_fence_after();
         }
         if (j >= 2) {
           float sc = head_sum<H>(tmem_base + acc * H + lane_off, wsh);
@@ -1414,13 +1426,13 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       const int quarter = warp & 3;
       P3Ctx c;
       c.row = quarter * 32 + lane;
-      c.tcol = tmem_base + 2 * H + (q & 1) * sc_cols + (static_cast<uint32_t>(quarter * 32) << 16);
+      c.tcol = tmem_base + 2 * H + (q % NSB) * sc_cols + (static_cast<uint32_t>(quarter * 32) << 16);
       c.n = meta[q & 1];
       c.ntiles = (c.n + kTile - 1) / kTile;
       c.cand = rows + static_cast<int64_t>(q & 1) * a.C;
       p3_topk(a, qi, c, c.row, ps);  // c.row == et: rows in thread order
       tc_fence_before();
-      mbar_arrive(&sfree[q & 1]);
+      mbar_arrive(&sfree[q % NSB]);
     }
   }
   tc_fence_before();
@@ -1450,8 +1462,10 @@ int pick_refine_kernel(int C, int H, bool has_scratch) {
   // second CTA
   constexpr size_t kMaxSmem = 227 * 1024;
   const size_t sm_local = tc_smem_bytes(C, H, false), sm_pipe = pipe_smem_bytes(H);
-  if (has_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, pipe_tmem_cols(C, H)) >= kTcCtasPerSm)
+  if (has_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, pipe_tmem_cols(C, H, 2)) >= kTcCtasPerSm)
     return REFINE_PIPE;
+  if (has_scratch && sm_pipe <= kMaxSmem && per_sm_for(sm_pipe, pipe_tmem_cols(C, H, 1)) >= kTcCtasPerSm)
+    return REFINE_PIPE_1BUF;
   if (sm_local <= kMaxSmem && per_sm_for(sm_local, tc_tmem_cols(C, H)) >= kTcCtasPerSm) return REFINE_SEQ_SMEM;
   return has_scratch ? REFINE_SEQ_GLOBAL : REFINE_SEQ_SMEM;
 }
@@ -1474,15 +1488,16 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     if (a.H != 32 && a.H != 64) return cudaErrorInvalidValue;
     const size_t sm_local = tc_smem_bytes(a.C, a.H, false), sm_glob = tc_smem_bytes(a.C, a.H, true);
     const size_t sm_pipe = pipe_smem_bytes(a.H);
-    const int tm_seq = tc_tmem_cols(a.C, a.H), tm_pipe = pipe_tmem_cols(a.C, a.H);
     constexpr size_t kMaxSmem = 227 * 1024;
     const int kind = a.refine_kernel == REFINE_AUTO ? pick_refine_kernel(a.C, a.H, a.cand_scratch != nullptr)
                                                     : a.refine_kernel;
-    if ((kind == REFINE_SEQ_GLOBAL || kind == REFINE_PIPE) && !a.cand_scratch) return cudaErrorInvalidValue;
-    if (kind != REFINE_SEQ_SMEM && kind != REFINE_SEQ_GLOBAL && kind != REFINE_PIPE) return cudaErrorInvalidValue;
+    if (kind < REFINE_SEQ_SMEM || kind > REFINE_PIPE_1BUF) return cudaErrorInvalidValue;
+    const bool pipe = kind == REFINE_PIPE || kind == REFINE_PIPE_1BUF;
+    if ((kind == REFINE_SEQ_GLOBAL || pipe) && !a.cand_scratch) return cudaErrorInvalidValue;
+    const int tm = pipe ? pipe_tmem_cols(a.C, a.H, kind == REFINE_PIPE ? 2 : 1) : tc_tmem_cols(a.C, a.H);
     const size_t smem = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
-    if (smem > kMaxSmem || (kind == REFINE_PIPE ? tm_pipe : tm_seq) > 512) return cudaErrorInvalidValue;
-    const int per_sm = per_sm_for(smem, kind == REFINE_PIPE ? tm_pipe : tm_seq);
+    if (smem > kMaxSmem || tm > 512) return cudaErrorInvalidValue;
+    const int per_sm = per_sm_for(smem, tm);
     const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
     if (grid <= 0) return cudaSuccess;
 #define AI_LAUNCH_REFINE(KERNEL)                                                                         \
@@ -1490,14 +1505,16 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));   \
     cudaFuncSetAttribute(KERNEL, cudaFuncAttributePreferredSharedMemoryCarveout, 100);                   \
     count_launch();                                                                                      \
-    KERNEL<<<grid, kind == REFINE_PIPE ? pipe_threads(kPipeNgw) : kTcThreads, smem, st>>>(*kmap, *qmap, a, vt); \
+    KERNEL<<<grid, pipe ? pipe_threads(kPipeNgw) : kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);         \
   } while (0)
     if (a.H == 32) {
-      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<32, kPipeNgw>));
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<32, kPipeNgw, 2>));
+      else if (kind == REFINE_PIPE_1BUF) AI_LAUNCH_REFINE((k_refine_pipe<32, kPipeNgw, 1>));
       else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<32, true>));
       else AI_LAUNCH_REFINE((k_refine_tc<32, false>));
     } else {
-      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<64, kPipeNgw>));
+      if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<64, kPipeNgw, 2>));
+      else if (kind == REFINE_PIPE_1BUF) AI_LAUNCH_REFINE((k_refine_pipe<64, kPipeNgw, 1>));
       else if (kind == REFINE_SEQ_GLOBAL) AI_LAUNCH_REFINE((k_refine_tc<64, true>));
       else AI_LAUNCH_REFINE((k_refine_tc<64, false>));
     }

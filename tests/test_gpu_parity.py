@@ -88,8 +88,9 @@ def test_tiny_fp32_full_prefill_every_query():
 
 
 # refine variants: 1 / 2 = one query per CTA (list in shared / global
-# memory), 3 = pipelined build / rescore / top-k
-@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3])
+# memory), 3 / 4 = pipelined build / rescore / top-k (two / one TMEM score
+# buffers)
+@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3, 4])
 def test_glm_bf16_scaled_sampled(refine_kernel):
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=20480, T=2048, refit_period=8192,
                   budget=3000, k=256, M=256)
@@ -108,7 +109,7 @@ def test_v4flash_fp8_scaled_sampled(refine_kernel):
 
 
 def test_refine_variants_agree_bitwise():
-    """The three tensor-core refine kernels return identical ids and scores
+    """The four tensor-core refine kernels return identical ids and scores
     (same arithmetic in the same order), over ragged query counts that
     leave CTAs with different numbers of queries, and a chunk whose first
     queries have short lists."""
@@ -124,7 +125,7 @@ def test_refine_variants_agree_bitwise():
         p0 = wl.L - T
         qd, wd, _, _ = P.query_inputs(wl, p0, wl.L)
         res = []
-        for kern in (1, 2, 3):
+        for kern in (1, 2, 3, 4):
             gpu.debug_refine_kernel(kern)
             out = torch.full((T, wl.k), -7, dtype=torch.int32, device="cuda")
             osc = torch.zeros((T, wl.k), dtype=torch.float32, device="cuda")
@@ -132,7 +133,7 @@ def test_refine_variants_agree_bitwise():
             cand, _ = gpu.debug_candidates(qd, wd, p0, wl.budget, with_scores=False)
             gpu.sync()
             res.append((out.cpu().numpy(), osc.cpu().numpy(), cand.cpu().numpy()))
-        for kern, r in zip((2, 3), res[1:]):
+        for kern, r in zip((2, 3, 4), res[1:]):
             assert np.array_equal(r[2], res[0][2]), f"candidates differ: kernel {kern}, T={T}"
             assert np.array_equal(r[0], res[0][0]), f"ids differ: kernel {kern}, T={T}"
             assert np.array_equal(r[1].view(np.uint32), res[0][1].view(np.uint32)), \
