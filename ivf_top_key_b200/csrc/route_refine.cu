@@ -341,26 +341,42 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   g.sync();
   const int len = static_cast<int>(min64(C, static_cast<int64_t>(fixed) + pref[nsel]));
   if (kGlobal) {
-    // fill of a list in global memory: each thread walks its slots (stride
-    // = group size) through the ranked runs, several loads in flight
-    int r = 0;
-    for (int i0 = fixed + tid; i0 < len; i0 += 4 * nthr) {
-      int32_t v[4];
+    // fill of a list in global memory: one warp per ranked cluster, four
+    // clusters per warp at a time (their run bounds are independent shared
+    // loads, their first 64 members eight coalesced loads per lane in
+    // flight), cut at C
+    for (int r0 = warp; r0 < nsel; r0 += 4 * nwarps) {
+      int d0[4], sz[4], src[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * nthr;
-        v[u] = 0;
-        if (i < len) {
-          const int rel = i - fixed;
-          while (pref[r + 1] <= rel) ++r;
-          v[u] = __ldg(a.members + coff[r] + (rel - pref[r]));
+        const int r = r0 + u * nwarps;
+        d0[u] = 0;
+        sz[u] = 0;
+        src[u] = 0;
+        if (r < nsel) {
+          d0[u] = fixed + pref[r];
+          sz[u] = min(pref[r + 1] - pref[r], len - d0[u]);
+          src[u] = coff[r];
         }
       }
+      int32_t v[4][2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * nthr;
-        if (i < len) cand[i] = v[u];
-      }
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int l = lane + 32 * h;
+          v[u][h] = l < sz[u] ? __ldg(a.members + src[u] + l) : 0;
+        }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int l = lane + 32 * h;
+          if (l < sz[u]) cand[d0[u] + l] = v[u][h];
+        }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        for (int l = 64 + lane; l < sz[u]; l += 32) cand[d0[u] + l] = __ldg(a.members + src[u] + l);
     }
   } else {
     // fill of a list in shared memory: one warp per ranked cluster copies
@@ -836,9 +852,23 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   }
   named_bar(1, 128);
   const int nw = min(total, k);
-  for (int j = et; j < k; j += 128) {
-    out[j] = j < nw ? cd[sid[j]] : -1;
-    if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
+  // the ids of a thread's outputs are all loaded before any is stored (the
+  // stores could alias the list, so the compiler would not reorder them)
+  for (int j0 = et; j0 < k; j0 += 8 * 128) {
+    int32_t id[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 128;
+      id[u] = j < nw ? cd[sid[j]] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 128;
+      if (j < k) {
+        out[j] = id[u];
+        if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
+      }
+    }
   }
   named_bar(1, 128);
 }
