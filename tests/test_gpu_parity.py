@@ -321,3 +321,27 @@ def test_checkpoint_rollback_repeats_a_chunk_exactly():
     assert np.array_equal(outs[0][0], outs[1][0])
     assert np.array_equal(outs[0][1]["members"], outs[1][1]["members"])
     gpu.close()
+
+
+def test_refine_kernel_choice():
+    """The refine kernel the library reports for each path: the fp32 SIMT
+    kernel (0); the pipelined kernel with two TMEM score buffers up to
+    C = 8192 (3) and with one at C = 16384 (4); a forced variant as set."""
+    tiny = S.WORKLOADS["tiny_fp32_L4k"]
+    gpu, _ = P.make_pair(tiny)
+    assert gpu.refine_kernel_choice(tiny.budget) == 0
+    gpu.close()
+    glm = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=4096, T=1024, refit_period=2048, budget=8192,
+                   k=64, M=128)
+    gpu, _ = P.make_pair(glm)
+    assert gpu.refine_kernel_choice(8192) == 3
+    assert gpu.refine_kernel_choice(1000) == 3
+    gpu.debug_refine_kernel(2)
+    assert gpu.refine_kernel_choice(8192) == 2
+    gpu.close()
+    v4 = S.scaled(S.WORKLOADS["v4flash_fp8_L256k"], L=4096, T=1024, refit_period=2048, budget=16384,
+                  k=64, M=128)
+    gpu, _ = P.make_pair(v4)
+    assert gpu.refine_kernel_choice(16384) == 4
+    assert gpu.refine_kernel_choice(8192) == 3
+    gpu.close()
