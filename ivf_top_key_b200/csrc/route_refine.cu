@@ -14,7 +14,7 @@
 //     (two levels) find the budget threshold over the visible non-empty
 //     clusters; the clusters at or above it are ranked by (score desc, id
 //     asc) and their member runs are copied, after the sinks and the open
-//     window, into a shared-memory candidate list;
+//     window, into the candidate list (shared memory or global scratch);
 //  2. exact rescore, 128 candidates per tile: TMA tile::gather4 brings the
 //     bf16 rows (for fp8 keys, the bf16 copy of the codes) into the
 //     128-byte-swizzled UMMA layout, one tcgen05 UMMA (M = 128 candidates,
