@@ -33,8 +33,9 @@ an asynchronous refit becomes visible at the next append (or explicit
 publish).
 
 Parity pins: see tests/test_oracle_pins.py.  The encoder (learned
-correction) is pinned only by its zero-output case; otherwise its
-architecture is a reading of the explainer and its parity is unpinned.
+correction) is pinned by its zero-output case, its norm bound and closed
+forms of each stage under hand-chosen weights; its architecture itself is
+a reading of the explainer (the pages give no shapes).
 """
 from __future__ import annotations
 

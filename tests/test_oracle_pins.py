@@ -260,6 +260,53 @@ def test_encoder_zero_output_is_plain_ivf_and_bound_holds():
     assert np.linalg.norm(corr) > 0
 
 
+def _enc(A, a, B1, b1, B2, b2):
+    f = lambda x: np.asarray(x, dtype=np.float64)
+    return {"A": f(A), "a": f(a), "B1": f(B1), "b1": f(b1), "B2": f(B2), "b2": f(b2)}
+
+
+def _sel(i, n=7):
+    e = np.zeros(n)
+    e[i] = 1.0
+    return e
+
+
+def test_encoder_closed_forms():
+    """Weights chosen so each stage of the correction reduces to numbers a
+    reader can derive by hand (d = 2, so f has 3d + 1 = 7 entries in the
+    order [mean phi ; max phi ; mu ; ln n]).  A swapped feature block, a
+    missing ReLU or bias, or a wrong bound rule changes the result."""
+    # 1. phi = ReLU(k); h picks max phi_0 and ln n; bound inactive, corr = t
+    members = np.array([[1.0, 0.0], [3.0, 2.0]])
+    mu = members.mean(0)                                   # [2, 1]
+    w = _enc(np.eye(2), [0, 0], np.stack([_sel(2), _sel(6)]), [0, 0],
+             [[0.1, 0.0], [0.0, 1.0]], [0.0, -0.5])
+    # h = [max phi_0, ln 2] = [3, ln 2]; z = [0.3, ln 2 - 0.5]
+    want = np.array([math.tanh(0.3), math.tanh(math.log(2.0) - 0.5)])
+    assert np.linalg.norm(want) < 0.25 * math.sqrt(5.0)     # the bound does not bind
+    np.testing.assert_allclose(O.encoder_correction(members, mu, w), want, rtol=0, atol=1e-15)
+    # 2. the bound binds: corr = t * 0.25 ||mu|| / ||t|| = [0.25 * 0.2, 0]
+    members = np.array([[0.2, 0.0], [-0.2, 0.4]])
+    mu = members.mean(0)                                   # [0, 0.2]
+    w = _enc(np.eye(2), [0, 0], np.zeros((2, 7)), [0, 0], np.zeros((2, 2)), [1.0, 0.0])
+    np.testing.assert_allclose(O.encoder_correction(members, mu, w), [0.05, 0.0], rtol=0, atol=1e-15)
+    # 3. phi = ReLU(k + a) with a = [-1, 0] clips; h picks mean phi_0 and max phi_1
+    members = np.array([[0.5, -1.0], [2.0, 3.0]])
+    mu = members.mean(0)                                   # [1.25, 1]
+    w = _enc(np.eye(2), [-1.0, 0.0], np.stack([_sel(0), _sel(3)]), [0, 0], 0.2 * np.eye(2), [0, 0])
+    # phi = [[0, 0], [1, 3]]: mean phi_0 = 0.5, max phi_1 = 3; z = 0.2 * [0.5, 3]
+    t = np.array([math.tanh(0.1), math.tanh(0.6)])
+    bound = 0.25 * math.hypot(1.25, 1.0)
+    assert np.linalg.norm(t) > bound                       # the bound binds
+    np.testing.assert_allclose(O.encoder_correction(members, mu, w), t * bound / np.linalg.norm(t),
+                               rtol=1e-14, atol=0)
+    # 4. a ReLU in h: a negative pre-activation gives h = 0, so t = tanh(b2)
+    w = _enc(np.eye(2), [0, 0], np.stack([-_sel(2), -_sel(6)]), [0, 0], np.eye(2), [0.01, 0.0])
+    members = np.array([[1.0, 0.0], [3.0, 2.0]])
+    np.testing.assert_allclose(O.encoder_correction(members, members.mean(0), w),
+                               [math.tanh(0.01), 0.0], rtol=0, atol=1e-15)
+
+
 # ------------------------------------------------------------ index-level --
 
 def _tiny_index(wl, enc=None):
