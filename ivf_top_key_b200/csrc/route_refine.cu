@@ -1127,13 +1127,14 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
 //   tempty[a]  epilogue has read accumulator a
 //   qfull      head tile landed;  qempty  UMMAs of the previous query done
 //   cready[b]  list b built;  sready[b]  score columns b written;
-//   sfree[b]   score columns b read by the top-k
+//   sfree[b]   score columns b read by the top-k;
+//   mread[b]   list b's length read by the UMMA warp
 __host__ __device__ inline size_t pipe_bg_bytes() {
   const size_t p1 = align_up(static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4, 16) + sizeof(P1Smem);
   const size_t p3 = sizeof(P3Smem);
   return align_up(p1 > p3 ? p1 : p3, 16);
 }
-constexpr int kPipeBars = 14;
+constexpr int kPipeBars = 16;
 // Gathering warps of the pipelined kernel (4 or 8).  Eight measured
 // slower on B200 (128K bf16: 2.21M vs 2.40M query tokens/s): the SM's
 // gather4 throughput, not the issuing warps, bounds the rescore there.
@@ -1191,6 +1192,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
   uint64_t* cready = bars + 8;
   uint64_t* sready = bars + 10;
   uint64_t* sfree = bars + 12;
+  uint64_t* mread = bars + 14;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kPipeBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1207,6 +1209,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       mbar_init(&cready[i], 128);
       mbar_init(&sready[i], 128);
       mbar_init(&sfree[i], 128);
+      mbar_init(&mread[i], 1);
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -1350,6 +1353,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
         const int b = q & 1;
         if (!mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag)) break;
         const int nt = (meta[b] + kTile - 1) / kTile;
+        mbar_arrive(&mread[b]);  // the slot's length is read; it may be rebuilt
         // the head tile is rewritten once the previous query's UMMAs are done
         if (q > 0 && !mbar_wait(qempty, (commits - 1) & 1, a.err, abort_flag)) break;
         mbar_arrive_expect_tx(qfull, H * 256);
@@ -1432,7 +1436,16 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     uint64_t* sortbuf = reinterpret_cast<uint64_t*>(bg);
     int32_t* pref = reinterpret_cast<int32_t*>(bg + static_cast<size_t>(kSortCap) * 8);
     P3Smem& ps = *reinterpret_cast<P3Smem*>(bg);
-    auto build = [&](int q) {
+    // returns false (every thread alike) when a wait gave up
+    auto build = [&](int q) -> bool {
+      if (q >= 2) {
+        // slot q & 1 last held query q - 2: the gathering warps and the
+        // top-k are done with it (sready, sequence), and the UMMA warp must
+        // have read its length, which nothing else orders when that query
+        // had no tiles
+        const bool w = mbar_wait(&mread[q & 1], ((q - 2) >> 1) & 1, a.err, abort_flag);
+        if (!named_bar_and(2, 128, w)) return false;
+      }
       const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
       const int64_t t = a.pos0 + qi;
       int nC;
@@ -1445,11 +1458,12 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       }
       if (et == 0) meta[q & 1] = n;
       mbar_arrive(&cready[q & 1]);  // after this thread's own list stores
+      return true;
     };
-    if (nq > 0) build(0);
-    for (int q = 0; q < nq; ++q) {
+    const bool started = nq > 0 && build(0);
+    for (int q = 0; started && q < nq; ++q) {
       const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
-      if (q + 1 < nq) build(q + 1);
+      if (q + 1 < nq && !build(q + 1)) break;
       const bool ok = mbar_wait(&sready[q & 1], (q >> 1) & 1, a.err, abort_flag);
       if (!named_bar_and(1, 128, ok)) break;
       tc_fence_after();
