@@ -63,7 +63,7 @@ class AiError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ivf_top_key_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python ivf_top_key_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     sig = {
