@@ -35,7 +35,7 @@ namespace {
 constexpr int kSortCap = 2048;  // ranked clusters per query (size-capped at ~W/m keys each)
 constexpr int kTile = 128;
 constexpr int kStages = 3;
-constexpr int kTcThreads = 288;   // warps 0-3 gather, 4 UMMA, 5-8 epilogue
+constexpr int kTcThreads = 288;   // 9 warps; each tensor-core kernel lists its warp roles
 constexpr int kSimtThreads = 256;
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -924,6 +924,10 @@ __host__ __device__ inline int tc_tmem_cols(int C, int H) {
   return cols;
 }
 
+// Block-sequential tensor-core kernel: one query at a time per CTA.  All
+// warps build the candidate list; then warps 0-3 gather the rows (TMA
+// gather4), warp 4 issues the UMMAs and warps 5-8 run the epilogue into
+// TMEM score columns and, after the last tile, the top-k.
 template <int H, bool kGC>
 __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     k_refine_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
