@@ -1543,17 +1543,17 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     const bool pipe = kind == REFINE_PIPE || kind == REFINE_PIPE_1BUF;
     if ((kind == REFINE_SEQ_GLOBAL || pipe) && !a.cand_scratch) return cudaErrorInvalidValue;
     const int tm = pipe ? pipe_tmem_cols(a.C, a.H, kind == REFINE_PIPE ? 2 : 1) : tc_tmem_cols(a.C, a.H);
-    const size_t smem = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
-    if (smem > kMaxSmem || tm > 512) return cudaErrorInvalidValue;
-    const int per_sm = per_sm_for(smem, tm);
+    const size_t smem_tc = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
+    if (smem_tc > kMaxSmem || tm > 512) return cudaErrorInvalidValue;
+    const int per_sm = per_sm_for(smem_tc, tm);
     const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
     if (grid <= 0) return cudaSuccess;
 #define AI_LAUNCH_REFINE(KERNEL)                                                                         \
   do {                                                                                                   \
-    cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));   \
+    cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_tc)); \
     cudaFuncSetAttribute(KERNEL, cudaFuncAttributePreferredSharedMemoryCarveout, 100);                   \
     count_launch();                                                                                      \
-    KERNEL<<<grid, pipe ? pipe_threads(kPipeNgw) : kTcThreads, smem, st>>>(*kmap, *qmap, a, vt);         \
+    KERNEL<<<grid, pipe ? pipe_threads(kPipeNgw) : kTcThreads, smem_tc, st>>>(*kmap, *qmap, a, vt);      \
   } while (0)
     if (a.H == 32) {
       if (kind == REFINE_PIPE) AI_LAUNCH_REFINE((k_refine_pipe<32, kPipeNgw, 2>));
