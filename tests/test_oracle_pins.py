@@ -388,3 +388,59 @@ def test_recall_definition():
     b = np.array([[3, 2, 9, -1], [7, 6, 5, 4]])
     assert O.recall(a, a) == 1.0
     assert O.recall(b, a) == (2 + 4) / 7
+
+
+# ------------------------------------------------- candidate fill, by hand --
+
+def _hand_index():
+    """A hand-built index state (explainer, 查询时怎么挑候选？ and the version
+    paragraph of 索引怎么边算边建？), S = 4 sinks, 15 keys (ids 0..14).
+
+    Window 1 = keys [4, 8) sealed into clusters c0, c1 -> version (2, 8).
+    Window 2 = keys [8, 12) sealed into c2 (empty), c3, c4 -> version (5, 12).
+    One head, weight 1, query q = (2, 1); route score = ReLU(2 r0 + r1):
+
+      cluster  rep          score  members
+      c0       (0.5, 0)     1.0    4, 6
+      c1       (1.0, 0.5)   2.5    5, 7
+      c2       (2, 2)       6.0    (empty: skipped)
+      c3       (0.25, 0.5)  1.0    8, 10, 11   (ties c0: lower id first)
+      c4       (-1, 0)      0.0    9
+    """
+    idx = O.OracleIndex(d=2, n_sinks=4, window=4, clusters_per_window=2, refit_period=0)
+    idx.keys = np.zeros((15, 2))
+    spec = [((0.5, 0.0), [4, 6]), ((1.0, 0.5), [5, 7]), ((2.0, 2.0), []),
+            ((0.25, 0.5), [8, 10, 11]), ((-1.0, 0.0), [9])]
+    idx.clusters = [O.Cluster(centroid=np.array(r), members=np.array(m, dtype=np.int64),
+                              rep=np.array(r)) for r, m in spec]
+    idx.versions = [O.Version(2, 8), O.Version(5, 12)]
+    return idx, np.array([[2.0, 1.0]]), np.array([1.0])
+
+
+@pytest.mark.parametrize("t,C,want", [
+    # t = 14 uses version (5, 12): sinks, open window 12..14, then
+    # c1 (2.5), c0 (1.0), c3 (1.0, tie -> after c0), c4 (0.0); c2 is empty
+    (14, 100, [0, 1, 2, 3, 12, 13, 14, 5, 7, 4, 6, 8, 10, 11, 9]),
+    (14, 10, [0, 1, 2, 3, 12, 13, 14, 5, 7, 4]),            # rank-2 list cut after one member
+    (14, 13, [0, 1, 2, 3, 12, 13, 14, 5, 7, 4, 6, 8, 10]),  # tie order, rank-3 list cut
+    (14, 5, [0, 1, 2, 3, 12]),                               # budget inside the open window
+    # t = 10 uses version (2, 8) (watermark 12 > t + 1): open window 8..10,
+    # only c1 and c0 visible
+    (10, 100, [0, 1, 2, 3, 8, 9, 10, 5, 7, 4, 6]),
+    (10, 9, [0, 1, 2, 3, 8, 9, 10, 5, 7]),
+    # t = 2: no sealed version yet, sinks cut at t
+    (2, 100, [0, 1, 2]),
+])
+def test_candidate_fill_order_by_hand(t, C, want):
+    """The exact candidate sequence: sinks, open window ascending, member
+    lists in rank order (score desc, cluster id asc) in CSR order, the last
+    list truncated at C, empty clusters contributing nothing, clusters of
+    newer versions invisible."""
+    idx, q, w = _hand_index()
+    cand, sc, v = idx.candidates(t, q, w, C)
+    assert cand.tolist() == want
+    if t >= 11:
+        assert sc.tolist() == [1.0, 2.5, 6.0, 1.0, 0.0]
+    # route+refine on this state returns ids drawn from exactly that list
+    ids, _ = idx.route_refine(q, w, t, k=len(want), C=C)
+    assert sorted(ids[ids >= 0].tolist()) == sorted(want)
