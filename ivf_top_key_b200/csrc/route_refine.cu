@@ -396,13 +396,14 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
 }
 
 // Phase 3: top-k of score[0..n) with ids cand[]; ties go to the lower id.
+// sbuf: shared memory for the output sort (next power of two >= k keys).
 __device__ __forceinline__ void topk_emit(const RefineArgs& a, int qi, const float* score,
-                                          const int32_t* cand, int n, BlockScratch& bs) {
+                                          const int32_t* cand, int n, BlockScratch& bs, uint64_t* sbuf) {
   int32_t* out = a.out + static_cast<int64_t>(qi) * a.k;
   float* outs = a.out_scores ? a.out_scores + static_cast<int64_t>(qi) * a.k : nullptr;
   topk_select_emit(
       n, [&](int i) -> float { return score[i]; }, [&](int i) -> int32_t { return cand[i]; }, a.k,
-      out, outs, bs);
+      out, outs, bs, sbuf);
 }
 
 struct Layout {
@@ -489,7 +490,9 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
       L.score[slot] = sc;
     }
     __syncthreads();
-    topk_emit(a, qi, L.score, L.cand, n, bs);
+    // the query row in the region is dead now: it holds the output sort
+    topk_emit(a, qi, L.score, L.cand, n, bs, L.sortbuf);
+    __syncthreads();
   }
 }
 
@@ -504,10 +507,12 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
 // select over the same items.  Ties at the threshold go to the lower key id.
 constexpr int kNB = 2048;     // histogram bins
 constexpr int kCapB = 2048;   // items of the threshold bin sorted in smem (>= k/2)
+constexpr int kMaxBinSort = 96;  // output sort: largest score bin ranked by comparisons
 
 struct P3Smem {
   uint32_t hist[kNB];
   uint64_t buf[kCapB];
+  int32_t perm[kCapB];   // output sort: staged items grouped by score bin
   float fred[8];
   int ired[8];
   int scal[8];
@@ -805,8 +810,8 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       theta_id = static_cast<int>(~idk);
     }
   }
-  // emission: ids staged in shared memory in thread-major order, then
-  // written out coalesced (deterministic order).  Selection is v >= theta
+  // emission: the selected items are staged in shared memory, sorted into
+  // the output order and written out coalesced.  Selection is v >= theta
   // (everything when all items are kept), except when only some of the
   // items tied at theta are kept: then v > theta or (v == theta and id <=
   // theta_id).  Bodies are branch-free; unselected items write to a
@@ -828,16 +833,18 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   }
   int total;
   int pos = p3_scan(mine, et, &total, ps);
-  int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] slots
-  float* ssc = reinterpret_cast<float*>(ps.buf) + kCapB;       // [k] scores
-  int32_t* dump_id = reinterpret_cast<int32_t*>(ps.hist) + et;
-  float* dump_sc = reinterpret_cast<float*>(ps.hist) + 128 + et;
-  auto stage = [&pos, sid, ssc, dump_id, dump_sc, k](float v, int slot, int f) {
+  // staging: every selected item becomes a 64-bit order key (score desc,
+  // id asc) at its thread-order position; the id load is predicated (an
+  // unselected item reads entry 0), unselected items write a per-thread
+  // dummy slot, so the body stays branch-free
+  static_assert(kCapB >= 2048, "the output sort holds k <= 2048 keys");
+  uint64_t* keys = ps.buf;
+  uint64_t* dump = reinterpret_cast<uint64_t*>(ps.hist) + et;
+  auto stage = [&pos, keys, dump, k, cd, nlast](float v, int slot, int f) {
     const bool w = (f & static_cast<int>(pos < k)) != 0;
-    int32_t* pi = w ? sid + pos : dump_id;
-    float* pv = w ? ssc + pos : dump_sc;
-    *pi = slot;
-    *pv = v;
+    const int sl = (w && slot <= nlast) ? slot : 0;
+    const int32_t id = cd[sl];
+    *(w ? keys + pos : dump) = order_key(v, id);
     pos += f;
   };
   if (!partial_ties) {
@@ -850,25 +857,92 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       stage(v, slot, ok & (static_cast<int>(v > th) | (v == th ? static_cast<int>(cd[sl] <= thid) : 0)));
     });
   }
-  named_bar(1, 128);
+  // output order (score desc, id asc) by a counting sort: the staged keys
+  // are grouped by score bin (highest bin first), then each key takes its
+  // rank inside its bin by comparing with the bin's other keys.  Bins split
+  // the order-preserving integer keys of [lowest selected score, vmax] into
+  // at most kNB equal ranges: about constant relative width, so a few
+  // outlying high scores do not crowd the bulk into one bin.  A bin holding
+  // more than kMaxBinSort keys (near-equal scores) sends the whole list
+  // through a bitonic sort instead.
   const int nw = min(total, k);
-  // the ids of a thread's outputs are all loaded before any is stored (the
-  // stores could alias the list, so the compiler would not reorder them)
-  for (int j0 = et; j0 < k; j0 += 8 * 128) {
-    int32_t id[8];
+  const uint32_t klo = f2key(th == -INFINITY ? vmin : th);
+  const uint32_t krange = f2key(vmax) - klo;
+  int kshift = 0;
+  while (kshift < 32 && (static_cast<uint64_t>(krange) >> kshift) >= static_cast<uint64_t>(kNB)) ++kshift;
+  auto sbin = [=](uint64_t x) -> int {
+    const uint32_t d = ~static_cast<uint32_t>(x >> 32) - klo;  // f2key(score) - klo
+    const uint32_t b = kshift < 32 ? d >> kshift : 0u;
+    return b < static_cast<uint32_t>(kNB) ? static_cast<int>(b) : kNB - 1;
+  };
+  named_bar(1, 128);  // staging done (its dummy slots overlap the histogram)
+  for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
+  named_bar(1, 128);
+  for (int j = et; j < nw; j += 128) atomicAdd(&ps.hist[sbin(keys[j])], 1u);
+  named_bar(1, 128);
+  // bin starts in descending bin order: thread et owns bins 2047 - 16 et - u
+  int cnt16 = 0, cmax = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * 128;
-      id[u] = j < nw ? cd[sid[j]] : -1;
+  for (int u = 0; u < 16; ++u) {
+    const int c = static_cast<int>(ps.hist[kNB - 1 - (16 * et + u)]);
+    cnt16 += c;
+    cmax = max(cmax, c);
+  }
+  int all_total;
+  int run = p3_scan(cnt16, et, &all_total, ps);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int b = kNB - 1 - (16 * et + u);
+    const int c = static_cast<int>(ps.hist[b]);
+    ps.hist[b] = static_cast<uint32_t>(run);  // start of bin b
+    run += c;
+  }
+  for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+  if ((et & 31) == 0) ps.ired[4 + (et >> 5)] = cmax;
+  named_bar(1, 128);
+  const int bin_max = max(max(ps.ired[4], ps.ired[5]), max(ps.ired[6], ps.ired[7]));
+  if (bin_max <= kMaxBinSort) {
+    // group by bin (after this, bin b spans [end of bin b + 1, hist[b]))
+    for (int j = et; j < nw; j += 128) {
+      const int p = static_cast<int>(atomicAdd(&ps.hist[sbin(keys[j])], 1u));
+      ps.perm[p] = j;
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * 128;
-      if (j < k) {
-        out[j] = id[u];
-        if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
+    named_bar(1, 128);
+    for (int p = et; p < nw; p += 128) {
+      const uint64_t x = keys[ps.perm[p]];
+      const int b = sbin(x);
+      const int lo = b == kNB - 1 ? 0 : static_cast<int>(ps.hist[b + 1]);
+      const int hi = static_cast<int>(ps.hist[b]);
+      int r = lo;
+      for (int q = lo; q < hi; ++q) r += keys[ps.perm[q]] < x ? 1 : 0;
+      out[r] = order_key_id(x);
+      if (outs) outs[r] = order_key_score(x);
+    }
+  } else {
+    int np = 1;
+    while (np < nw) np <<= 1;
+    for (int i = nw + et; i < np; i += 128) keys[i] = kOrderPad;
+    named_bar(1, 128);
+    for (int kk = 2; kk <= np; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int p = et; p < (np >> 1); p += 128) {
+          const int i = ((p & ~(j - 1)) << 1) | (p & (j - 1));  // lower element of pair p
+          const uint64_t x = keys[i], y = keys[i + j];
+          const bool swp = ((i & kk) == 0) ? (x > y) : (x < y);
+          keys[i] = swp ? y : x;  // both written: no divergent branch
+          keys[i + j] = swp ? x : y;
+        }
+        named_bar(1, 128);
       }
     }
+    for (int j = et; j < nw; j += 128) {
+      out[j] = order_key_id(keys[j]);
+      if (outs) outs[j] = order_key_score(keys[j]);
+    }
+  }
+  for (int j = nw + et; j < k; j += 128) {
+    out[j] = -1;
+    if (outs) outs[j] = -INFINITY;
   }
   named_bar(1, 128);
 }
@@ -1138,6 +1212,11 @@ __host__ __device__ inline size_t pipe_bg_bytes() {
   const size_t p3 = sizeof(P3Smem);
   return align_up(p1 > p3 ? p1 : p3, 16);
 }
+// the top-k's shared memory (with the output sort) fits in the build's, so
+// the pipelined kernel keeps two CTAs per SM
+static_assert(sizeof(P3Smem) <= ((static_cast<size_t>(kSortCap) * 8 + (kSortCap + 1) * 4 + 15) & ~size_t(15)) +
+                                    sizeof(P1Smem),
+              "top-k shared memory grew past the candidate build's");
 constexpr int kPipeBars = 16;
 // Gathering warps of the pipelined kernel (4 or 8).  Eight measured
 // slower on B200 (128K bf16: 2.21M vs 2.40M query tokens/s): the SM's
@@ -1534,6 +1613,7 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     if (a.d != 128 || !a.q_is_bf16 || (a.key_dtype != KD_BF16 && a.key_dtype != KD_FP8))
       return cudaErrorInvalidValue;
     if (a.H != 32 && a.H != 64) return cudaErrorInvalidValue;
+    if (a.k > kTcMaxK) return cudaErrorInvalidValue;
     const size_t sm_local = tc_smem_bytes(a.C, a.H, false), sm_glob = tc_smem_bytes(a.C, a.H, true);
     const size_t sm_pipe = pipe_smem_bytes(a.H);
     constexpr size_t kMaxSmem = 227 * 1024;
@@ -1568,6 +1648,9 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     }
 #undef AI_LAUNCH_REFINE
   } else {
+    // the output sort reuses the phase-1 region: room for kRowTopkMaxK keys
+    if (a.k > kRowTopkMaxK || region_bytes(a.H, a.d, false) < static_cast<size_t>(kRowTopkMaxK) * 8)
+      return cudaErrorInvalidValue;
     cudaFuncSetAttribute(k_refine_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     int per_sm = 1;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_refine_simt, kSimtThreads, smem);

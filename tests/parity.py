@@ -10,7 +10,10 @@ results correct):
 * candidate lists are equal, or differ only by clusters whose route scores
   are within that tolerance of each other (checked for validity);
 * top-k sets are equal up to swaps whose scores are within tolerance of the
-  k-th score.
+  k-th score;
+* ids come out in (score desc, id asc) order: the library's own scores are
+  sorted with ties broken by id, and the j-th id's float64 score lies
+  within twice the tolerance of the oracle's j-th score.
 """
 from __future__ import annotations
 
@@ -64,12 +67,13 @@ def make_pair(wl: S.Workload, encoder=None, async_refit=True, max_keys=None):
         refit_period=wl.refit_period, refit_new_seeds=wl.refit_new_seeds,
         refit_seed_window=wl.refit_seed_window, seal_iters=wl.seal_iters,
         async_refit=async_refit, max_query_chunk=wl.T, max_budget=max(wl.budget, 64),
-        max_k=wl.k, max_keys=max_keys or wl.L, seed=wl.seed, encoder_weights=encoder)
+        max_k=wl.k, max_keys=max_keys or wl.L, seed=wl.seed, encoder_weights=encoder,
+        block_routing=wl.block_routing)
     orc = O.OracleIndex(d=wl.d, n_sinks=wl.n_sinks, window=wl.window,
                         clusters_per_window=wl.clusters_per_window,
                         refit_period=wl.refit_period, refit_new_seeds=wl.refit_new_seeds,
                         refit_seed_window=wl.refit_seed_window, seal_iters=wl.seal_iters,
-                        seed=wl.seed, encoder=encoder)
+                        seed=wl.seed, encoder=encoder, block_routing=wl.block_routing)
     return gpu, orc
 
 
@@ -105,29 +109,38 @@ def check_index_equal(gpu, orc):
 
 # ----------------------------------------------------------- query checks --
 
-def output_order_key(slots, tile_order):
-    """Sort key of the documented output order: ascending candidate slot s
-    (fp32 path), or ascending (s mod 128, s div 128) (tensor-core path)."""
-    slots = np.asarray(slots, dtype=np.int64)
-    return (slots % 128) * (1 << 32) + slots // 128 if tile_order else slots
+def check_sequence(t, ids, gpu_scores, exact, want_scores, tol_max):
+    """The documented output order (score desc, id asc), position by position.
+
+    ids / gpu_scores: the valid ids and the library's scores for them, in
+    output order; exact: their float64 scores; want_scores: the oracle's
+    top-k scores in its (score desc, id asc) order.  The library's own
+    scores must be sorted with ties broken by id, and the j-th id's exact
+    score must be within 2 * tol_max of the oracle's j-th score (a near-tie
+    swap moves an id only among positions whose scores agree to that)."""
+    gs = np.asarray(gpu_scores, dtype=np.float64)
+    assert np.all(gs[1:] <= gs[:-1]), f"t={t}: scores not in descending order"
+    tie = gs[1:] == gs[:-1]
+    assert np.all(ids[1:][tie] > ids[:-1][tie]), f"t={t}: equal scores not in ascending id order"
+    n = min(ids.size, want_scores.size)
+    dev = np.abs(exact[:n] - want_scores[:n])
+    assert np.all(dev <= 2 * tol_max + 1e-6), \
+        f"t={t}: position {int(np.argmax(dev))} holds a score {dev.max():.3g} from the oracle's"
 
 
-def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats, tile_order=None):
-    """Compare route+refine results of the listed queries with the oracle.
-    tile_order: True / False checks the documented output order (tensor-core
-    / fp32 path) against the GPU's own candidate list; None skips it."""
+def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats):
+    """Compare route+refine results of the listed queries with the oracle:
+    candidate lists, scores, the top-k set and its (score desc, id asc)
+    order."""
     for i, t in enumerate(t_list):
         qi, wi = q[i], w[i]
         o_cand, rs, v = orc.candidates(t, qi, wi, C)
         g_cand = gpu_cand[i][gpu_cand[i] >= 0]
         g_ids = gpu_ids[i]
         valid = g_ids[g_ids >= 0]
+        assert np.all(g_ids[valid.size:] == -1), f"t={t}: padding is not a -1 suffix"
         assert np.all(valid <= t), f"t={t}: selected a future key"
         assert len(set(valid.tolist())) == valid.size, f"t={t}: duplicate ids"
-        if tile_order is not None and valid.size:
-            slot_of = {int(s): j for j, s in enumerate(g_cand.tolist())}
-            key = output_order_key([slot_of[int(s)] for s in valid.tolist()], tile_order)
-            assert np.all(np.diff(key) > 0), f"t={t}: output order"
         # scores of the selected ids agree with float64
         exact = O.indexer_score(qi, wi, orc.keys[valid])
         tol = score_tol(qi, wi, orc.keys[valid])
@@ -143,17 +156,44 @@ def check_queries(orc, t_list, q, w, gpu_ids, gpu_scores, gpu_cand, k, C, stats,
         want, want_sc = O.topk_ids(cs, g_cand, k)
         wv = want[want >= 0]
         assert valid.size == wv.size, f"t={t}: {valid.size} ids vs {wv.size}"
-        if set(valid.tolist()) != set(wv.tolist()):
-            theta = want_sc[wv.size - 1]
-            extra = np.setdiff1d(valid, wv)
-            miss = np.setdiff1d(wv, valid)
-            for s in np.concatenate([extra, miss]):
-                sc = O.indexer_score(qi, wi, orc.keys[[s]])[0]
-                tl = score_tol(qi, wi, orc.keys[[s]])[0]
-                assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: swap of key {s} not a near tie"
-            stats["topk_near_tie"] += 1
-        else:
+        tmax = float(score_tol(qi, wi, orc.keys[g_cand]).max()) if g_cand.size else 0.0
+        check_sequence(t, valid, gs, exact, want_sc[:wv.size], tmax)
+        if np.array_equal(valid, wv):
             stats["topk_equal"] += 1
+        else:
+            if set(valid.tolist()) != set(wv.tolist()):
+                theta = want_sc[wv.size - 1]
+                extra = np.setdiff1d(valid, wv)
+                miss = np.setdiff1d(wv, valid)
+                for s in np.concatenate([extra, miss]):
+                    sc = O.indexer_score(qi, wi, orc.keys[[s]])[0]
+                    tl = score_tol(qi, wi, orc.keys[[s]])[0]
+                    assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: swap of key {s} not a near tie"
+            stats["topk_near_tie"] += 1
+
+
+def check_exhaustive(orc, t, q, w, got, got_sc, k):
+    """Exhaustive selection of query t against the oracle's: the -1 padding,
+    the set up to near-tie swaps at the k-th score, scores within tolerance
+    and the (score desc, id asc) order."""
+    want, want_sc = orc.exhaustive(q, w, t, k)
+    vs = got >= 0
+    assert np.array_equal(vs, np.arange(k) < min(k, t + 1)), f"t={t}: padding"
+    g = got[vs]
+    w_ = want[want >= 0]
+    exact = O.indexer_score(q, w, orc.keys[g])
+    tol = score_tol(q, w, orc.keys[g])
+    assert np.all(np.abs(got_sc[vs] - exact) <= tol + 1e-6), f"t={t}: exhaustive score"
+    tmax = float(score_tol(q, w, orc.keys[:t + 1]).max())
+    check_sequence(t, g, got_sc[vs], exact, want_sc[:w_.size], tmax)
+    if set(g.tolist()) != set(w_.tolist()):
+        theta = want_sc[w_.size - 1]
+        for s in np.setxor1d(g, w_):
+            sc = O.indexer_score(q, w, orc.keys[[s]])[0]
+            tl = score_tol(q, w, orc.keys[[s]])[0]
+            assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: exhaustive swap {s}"
+        return "exh_near_tie"
+    return "exh_equal"
 
 
 def _check_candidate_validity(orc, t, q, w, g_cand, o_cand, rs, v, C):

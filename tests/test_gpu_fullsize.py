@@ -160,23 +160,14 @@ def test_glm_bf16_L1m_sampled_steps():
     gpu.route_refine(qd, wd, p0, wl.k, wl.budget, out=out, out_scores=osc)
     cand, _ = gpu.debug_candidates(qd, wd, p0, wl.budget, with_scores=False)
     eo = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
-    gpu.select_exhaustive(qd, wd, p0, wl.k, out=eo)
+    es = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    gpu.select_exhaustive(qd, wd, p0, wl.k, out=eo, out_scores=es)
     gpu.sync()
     idx = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, size=8, replace=False)]))
     stats = collections.Counter()
     P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], out.cpu().numpy()[idx],
-                    osc.cpu().numpy()[idx], cand.cpu().numpy()[idx], wl.k, wl.budget, stats,
-                    tile_order=wl.key_dtype != "fp32")
-    eo = eo.cpu().numpy()
+                    osc.cpu().numpy()[idx], cand.cpu().numpy()[idx], wl.k, wl.budget, stats)
+    eo, es = eo.cpu().numpy(), es.cpu().numpy()
     for i in idx[:4]:
-        t = p0 + i
-        want_ids, want_sc = orc.exhaustive(qv[i], wv[i], t, wl.k)
-        g = eo[i][eo[i] >= 0]
-        w_ = want_ids[want_ids >= 0]
-        if set(g.tolist()) != set(w_.tolist()):
-            theta = want_sc[w_.size - 1]
-            for s in np.setxor1d(g, w_):
-                sc = O.indexer_score(qv[i], wv[i], keys[[s]])[0]
-                tl = P.score_tol(qv[i], wv[i], keys[[s]])[0]
-                assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: exhaustive swap {s}"
+        P.check_exhaustive(orc, p0 + i, qv[i], wv[i], eo[i], es[i], wl.k)
     gpu.close()
