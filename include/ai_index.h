@@ -20,7 +20,9 @@
  *    gives a message for the calling thread.  A call that fails leaves the
  *    index unchanged unless stated otherwise.
  *  - Layouts are row-major and dense: keys [n, d], queries [T, H, d],
- *    head weights [T, H] float32, outputs [T, k] int32.
+ *    head weights [T, H] float32, outputs [T, k] int32.  With bf16 queries
+ *    the query and head-weight pointers must be 16-byte aligned (they are
+ *    read by bulk tensor copies); AI_ERR_ARG otherwise.
  *  - One handle is one (request, layer) index; handles are independent and
  *    must not be used from two threads at once.
  */
@@ -67,12 +69,19 @@ typedef struct ai_config {
   int32_t async_refit;         /* 1: refit runs on an internal side stream   */
   int32_t max_query_chunk;     /* largest T passed to route/exhaustive calls */
   int32_t max_budget;          /* largest C passed to ai_route_refine        */
-  int32_t max_k;               /* largest k                                  */
+  int32_t max_k;               /* largest k: <= 2048 (bf16 / fp8 keys),      */
+                               /* <= 4096 (fp32 keys)                        */
   int64_t max_keys;            /* capacity of the key store                  */
   uint64_t seed;               /* seed of the refit seed draws (SplitMix64)  */
   const float* encoder_weights_host; /* NULL: plain mean representatives.   */
   /* Else the correction encoder's float32 weights, packed in this order:
    * A [d,d], a [d], B1 [d, 3d+1], b1 [d], B2 [d,d], b2 [d] (copied at create). */
+  int32_t block_routing;       /* 0: the inverted-file index (k-means seal,  */
+  /* refit).  1: the contiguous-block baseline the explainer compares against
+   * ("它到底在解决什么问题？", HiSA): a sealed window is cut into m blocks of
+   * consecutive keys, block j = keys [lo + floor(jW/m), lo + floor((j+1)W/m)),
+   * each represented by its member mean; no refit (refit_period must be 0),
+   * no encoder.  Routing, candidate fill, rescore and top-k are unchanged.  */
 } ai_config;
 
 /* Create an index.  `cuda_stream` is the main stream (cudaStream_t, may be
@@ -118,19 +127,24 @@ int ai_publish(ai_handle h);
  * fills C candidate slots with the sinks, the open window [n_v, t] and
  * whole member lists in rank order (score desc, cluster id asc; the last
  * list is truncated), rescores the candidates exactly and writes the top k
- * ids by (score desc, id asc) to out_dev[T, k], padded with -1.  Their
- * order follows the candidate slots s: ascending s on the fp32 path, and
- * ascending (s mod 128, s div 128) on the tensor-core path (bf16 / fp8
- * keys), the same for every kernel variant.  q_dev: [T, H, d] in q_dtype; w_dev: [T, H] float32;
- * out_scores_dev: [T, k] float32 or NULL.  Errors: AI_ERR_ARG (T, k, C
- * beyond the create-time maxima), AI_ERR_CAUSALITY (pos0 + T - 1 >=
- * appended keys).                                                          */
+ * ids to out_dev[T, k] sorted by score descending, ties by key id
+ * ascending, then -1 padding (fewer than k candidates).  q_dev: [T, H, d]
+ * in q_dtype; w_dev: [T, H] float32; out_scores_dev: [T, k] float32 (the
+ * scores of those ids, -inf on padding) or NULL.
+ * Limit: at most 2048 clusters of one query can reach its budget (the
+ * clusters ranked in shared memory).  Clusters hold ~W/m keys after a seal,
+ * so this binds only when C / (smallest cluster size) exceeds 2048; a
+ * query over the limit ranks only 2048 of them and ai_sync then reports
+ * AI_ERR_DEVICE_CHECK.
+ * Errors: AI_ERR_ARG (T, k, C beyond the create-time maxima),
+ * AI_ERR_CAUSALITY (pos0 + T - 1 >= appended keys).                        */
 int ai_route_refine(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
                     int32_t T, int32_t k, int32_t C, int32_t* out_dev, float* out_scores_dev);
 
 /* Exhaustive selection (explainer, "它到底在解决什么问题？": the indexer
- * scores every key s <= t).  Same arguments and output order rules as
- * ai_route_refine (ids ascending).  The in-library baseline.              */
+ * scores every key s <= t).  Same arguments and output order as
+ * ai_route_refine (score descending, ties by id ascending, -1 padding).
+ * The in-library baseline.                                                */
 int ai_select_exhaustive(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
                          int32_t T, int32_t k, int32_t* out_dev, float* out_scores_dev);
 
@@ -217,17 +231,26 @@ int ai_quantize_fp8(const uint16_t* keys_bf16_dev, int64_t n, int32_t d, uint8_t
  * that loads the library until the process exits.
  *   keys_dev: [n_keys, d] keys owned by the caller: AI_BF16 (d = 128,
  *     H in {32, 64}, bf16 queries) or AI_FP32 (fp32 queries); n_keys at
- *     most 1,048,576 (AI_ERR_ARG beyond).
+ *     most 1,048,576 (AI_ERR_ARG beyond); k at most 4096.
  *   q_dev [T, H, d], w_dev [T, H], pos0, T, k, out_dev [T, k],
- *   out_scores_dev [T, k] or NULL: as for ai_select_exhaustive.
+ *   out_scores_dev [T, k] or NULL: as for ai_select_exhaustive (same
+ *     output order).
+ *   status_dev: NULL, or a device int32 that receives, in stream order
+ *     after the call's kernels, the device flags they raised: 0 when clean,
+ *     else an OR of AI_DEVFLAG_* (the handle-based calls report the same
+ *     flags through ai_sync).  A nonzero status means the output is not
+ *     valid.
  * Enqueued on cuda_stream.  The first call on a device looks up the
  * array's device address (make it before any stream capture).  All calls
  * share the array: calls whose work overlaps on the GPU (other streams,
  * other threads) race and must be serialised by the caller.              */
+#define AI_DEVFLAG_TIMEOUT 1   /* a bounded wait inside a kernel ran out     */
+#define AI_DEVFLAG_RANGE 2     /* an id or offset was out of range           */
+#define AI_DEVFLAG_CAPACITY 4  /* a per-CTA buffer would have overflowed     */
 int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_t n_keys,
                                  int32_t d, int32_t H, const void* q_dev, const float* w_dev,
                                  int64_t pos0, int32_t T, int32_t k, int32_t* out_dev,
-                                 float* out_scores_dev, void* cuda_stream);
+                                 float* out_scores_dev, int32_t* status_dev, void* cuda_stream);
 
 /* ------------------------------------------------ refine kernel variant */
 /* Selects the kernel that runs route+refine on the tensor-core path (bf16

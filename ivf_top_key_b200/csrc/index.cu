@@ -286,11 +286,7 @@ int route_scores(ai_index* h, const void* q, const float* w, int T, int64_t nC) 
     CUtensorMap ma, mb;
     if (!make_map(&ma, b.reps, nC, 128) || !make_map(&mb, q, static_cast<int64_t>(T) * h->cfg.H, 256))
       return fail(AI_ERR_CUDA, "tensor map encoding failed (route)");
-    const int qpt = 256 / h->cfg.H;
-    const int64_t qtiles = (T + qpt - 1) / qpt;
-    const int64_t atiles = (nC + 127) / 128;
-    int64_t apc = (atiles * qtiles + 4 * h->num_sms - 1) / (4 * h->num_sms);
-    apc = std::max<int64_t>(1, std::min(apc, atiles));
+    const int apc = scores_tiles_per_item(nC, T, h->cfg.H, h->num_sms);
     const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
     prof_end(h, pi, h->main);
@@ -324,6 +320,8 @@ int build_version_table(const ai_index* h, int64_t pos0, int T, VersionTable* vt
 
 int check_queries(const ai_index* h, const void* q, const float* w, int64_t pos0, int T, int k) {
   if (!q || !w) return fail(AI_ERR_ARG, "null query or weight pointer");
+  if (tc_route(h) && (reinterpret_cast<uintptr_t>(q) % 16 != 0 || reinterpret_cast<uintptr_t>(w) % 16 != 0))
+    return fail(AI_ERR_ARG, "q_dev and w_dev must be 16-byte aligned (bf16 queries)");
   if (T <= 0 || T > h->cfg.max_query_chunk) return fail(AI_ERR_ARG, "T out of range");
   if (k <= 0 || k > h->cfg.max_k) return fail(AI_ERR_ARG, "k out of range");
   if (pos0 < 0) return fail(AI_ERR_ARG, "negative pos0");
@@ -500,6 +498,7 @@ int seal_group(ai_index* h, int64_t w0, int64_t nw) {
   sa.m = static_cast<int>(m);
   sa.cap = h->cap;
   sa.iters = h->iters;
+  sa.blocks = h->cfg.block_routing;
   sa.first_key = S + w0 * W;
   sa.n_windows = static_cast<int>(nw);
   sa.members = A.members;
@@ -572,11 +571,7 @@ int exhaustive_scores(ai_index* h, const void* q, const float* w, int64_t pos0, 
     CUtensorMap ma, mb;
     if (!make_map(&ma, A, nA, 128) || !make_map(&mb, q, static_cast<int64_t>(T) * h->cfg.H, 256))
       return fail(AI_ERR_CUDA, "tensor map encoding failed (exhaustive)");
-    const int qpt = 256 / h->cfg.H;
-    const int64_t qtiles = (T + qpt - 1) / qpt;
-    const int64_t atiles = (nA + 127) / 128;
-    int64_t apc = (atiles * qtiles + 4 * h->num_sms - 1) / (4 * h->num_sms);
-    apc = std::max<int64_t>(1, std::min(apc, atiles));
+    const int apc = scores_tiles_per_item(nA, T, h->cfg.H, h->num_sms);
     const int pe = prof_begin(h, AI_PHASE_EXH_SCORES, h->main);
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
     prof_end(h, pe, h->main);
@@ -609,6 +604,9 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
     return fail(AI_ERR_ARG, "bad sinks / window / clusters per window");
   if (c.refit_period < 0 || (c.refit_period > 0 && c.refit_period % c.window != 0))
     return fail(AI_ERR_ARG, "refit period must be a multiple of the window");
+  if (c.block_routing != 0 && c.block_routing != 1) return fail(AI_ERR_ARG, "block_routing must be 0 or 1");
+  if (c.block_routing && (c.refit_period != 0 || c.encoder_weights_host))
+    return fail(AI_ERR_ARG, "block routing takes no refit and no encoder");
   if ((c.refit_period > 0 || c.encoder_weights_host) && c.d > 128)
     return fail(AI_ERR_ARG, "refit and the correction encoder support d <= 128");
   if (c.max_keys <= 0 || c.max_keys >= (int64_t(1) << 31)) return fail(AI_ERR_ARG, "bad max_keys");
@@ -624,7 +622,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   const bool tck = tcr && c.key_dtype != AI_FP32;
   if (refine_smem_bytes(c.max_budget, c.H, c.d, tck) > 227 * 1024)
     return fail(AI_ERR_ARG, "max_budget too large for the per-query kernel");
-  if (tck && c.max_k > 2048) return fail(AI_ERR_ARG, "k above 2048 is not supported for bf16/fp8 keys");
+  if (tck && c.max_k > kTcMaxK) return fail(AI_ERR_ARG, "k above 2048 is not supported for bf16/fp8 keys");
+  if (!tck && c.max_k > kRowTopkMaxK) return fail(AI_ERR_ARG, "k above 4096 is not supported for fp32 keys");
 
   ai_index* h = new ai_index();
   h->cfg = c;

@@ -21,13 +21,15 @@ struct ScoreArgs {
   const float* row_scale;  // [nA] per-row positive scale or nullptr
   float* out;              // out[q * ld_out + a]
   int64_t ld_out;
-  int a_tiles_per_cta;
+  int a_tiles_per_cta;      // A tiles per work item (tensor-core path)
   int causal;              // mask a_pos0 + a > q_pos0 + q to -inf
   int64_t a_pos0;
   int64_t q_pos0;
   int* err;
 };
 int scores_smem_bytes();
+// A tiles per work item of launch_scores_tc for nA rows, T queries, H heads.
+int scores_tiles_per_item(int64_t nA, int T, int H, int num_sms);
 cudaError_t launch_scores_tc(const CUtensorMap& mapA, const CUtensorMap& mapB, int H,
                              const ScoreArgs& args, int a_tiles_per_cta, cudaStream_t st);
 cudaError_t launch_scores_simt(const void* A, int a_dtype, const void* Q, int q_is_bf16, int d,
@@ -83,6 +85,12 @@ size_t refine_smem_bytes(int C, int H, int d, bool tc);
 cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUtensorMap* kmap,
                           const CUtensorMap* qmap, int num_sms, cudaStream_t st);
 
+// Largest k of every top-k that sorts its output in shared memory: the
+// exhaustive row top-k and the fp32 (SIMT) route+refine.  The tensor-core
+// route+refine allows 2048.
+constexpr int kRowTopkMaxK = 4096;
+constexpr int kTcMaxK = 2048;
+
 // ------------------------------------------------------- exhaustive top-k
 struct RowTopkArgs {
   const float* scores;  // [T, ld]
@@ -103,6 +111,7 @@ struct SealArgs {
   const float* key_scale;
   int key_dtype;
   int d, W, m, cap, iters;
+  int blocks;               // 1: contiguous blocks with mean representatives (no k-means)
   int64_t first_key;        // window j covers keys [first_key + j W, + W)
   int n_windows;
   int32_t* members;         // output: window j writes members[mem_base + j W ...]

@@ -50,7 +50,7 @@ def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_
         scs = osc.cpu().numpy()[idx]
         cnd = cand.cpu().numpy()[idx]
         P.check_queries(orc, (p0 + idx).tolist(), qv[idx], wv[idx], ids, scs, cnd, wl.k,
-                        wl.budget, stats, tile_order=wl.key_dtype != "fp32")
+                        wl.budget, stats)
         if check_exhaustive is True or (check_exhaustive and c in check_exhaustive):
             eo = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
             es = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
@@ -58,24 +58,7 @@ def _run_prefill(wl, *, sample=None, check_exhaustive=True, encoder=None, async_
             gpu.sync()
             eo, es = eo.cpu().numpy()[idx], es.cpu().numpy()[idx]
             for j, i in enumerate(idx):
-                t = p0 + i
-                want, want_sc = orc.exhaustive(qv[i], wv[i], t, wl.k)
-                got = eo[j]
-                assert np.array_equal(got >= 0, np.arange(wl.k) < min(wl.k, t + 1))
-                assert np.all(np.diff(got[got >= 0]) > 0), "exhaustive ids must ascend"
-                if set(got[got >= 0].tolist()) != set(want[want >= 0].tolist()):
-                    theta = want_sc[(want >= 0).sum() - 1]
-                    for s in np.setxor1d(got[got >= 0], want[want >= 0]):
-                        sc = O.indexer_score(qv[i], wv[i], orc.keys[[s]])[0]
-                        tl = P.score_tol(qv[i], wv[i], orc.keys[[s]])[0]
-                        assert abs(sc - theta) <= 2 * tl + 1e-6, f"t={t}: exhaustive swap {s}"
-                    stats["exh_near_tie"] += 1
-                else:
-                    stats["exh_equal"] += 1
-                vs = got >= 0
-                exact = O.indexer_score(qv[i], wv[i], orc.keys[got[vs]])
-                tol = P.score_tol(qv[i], wv[i], orc.keys[got[vs]])
-                assert np.all(np.abs(es[j][vs] - exact) <= tol + 1e-6)
+                stats[P.check_exhaustive(orc, p0 + i, qv[i], wv[i], eo[j], es[j], wl.k)] += 1
     gpu.close()
     return stats
 
@@ -99,13 +82,51 @@ def test_glm_bf16_scaled_sampled(refine_kernel):
     assert st["cand_near_tie"] <= 0.02 * (st["cand_equal"] + st["cand_near_tie"]), st
 
 
-@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3])
+@pytest.mark.parametrize("refine_kernel", [0, 1, 2, 3, 4])
 def test_v4flash_fp8_scaled_sampled(refine_kernel):
     wl = S.scaled(S.WORKLOADS["v4flash_fp8_L256k"], L=12288, T=2048, refit_period=4096,
                   budget=2500, k=200, M=256)
     st = _run_prefill(wl, sample=32, refine_kernel=refine_kernel,
                       check_exhaustive=True if refine_kernel == 0 else False)
     assert st["cand_equal"] > 0, st
+
+
+def test_v4flash_fp8_largest_budget_automatic_choice():
+    """fp8 keys, H = 64, C = 16384 (the largest budget of that workload):
+    the library picks the pipelined kernel with one TMEM score buffer, and
+    its results match the oracle on sampled queries of every chunk."""
+    wl = S.scaled(S.WORKLOADS["v4flash_fp8_L256k"], L=24576, T=4096, refit_period=8192,
+                  budget=16384, k=1024, M=256)
+    gpu, _ = P.make_pair(wl)
+    assert gpu.refine_kernel_choice(wl.budget) == 4
+    gpu.close()
+    st = _run_prefill(wl, sample=10, check_exhaustive={wl.n_chunks - 1})
+    assert st["cand_equal"] > 0, st
+
+
+def test_cluster_rank_limit_is_reported():
+    """Two-key clusters (W = 64 sealed into m = 32) and a budget of 8192:
+    about 4000 clusters would have to be ranked for one query, above the
+    2048 the kernel ranks in shared memory.  The overflow comes back from
+    ai_sync as AI_ERR_DEVICE_CHECK, and the handle stays usable."""
+    from ivf_top_key_b200 import AiError
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=16384, T=2048, window=64, clusters_per_window=32,
+                  refit_period=0, budget=8192, k=64, M=256)
+    gpu, _ = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        kd, ks, _ = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+    gpu.sync()
+    p0 = wl.L - wl.T
+    qd, wd, _, _ = P.query_inputs(wl, p0, wl.L)
+    gpu.route_refine(qd, wd, p0, wl.k, wl.budget)
+    with pytest.raises(AiError, match="DEVICE_CHECK"):
+        gpu.sync()
+    # a budget that needs few clusters runs clean afterwards
+    gpu.route_refine(qd, wd, p0, wl.k, 1024)
+    gpu.sync()
+    gpu.close()
 
 
 def test_refine_variants_agree_bitwise():
@@ -139,6 +160,16 @@ def test_refine_variants_agree_bitwise():
             assert np.array_equal(r[1].view(np.uint32), res[0][1].view(np.uint32)), \
                 f"scores differ: kernel {kern}, T={T}"
     gpu.close()
+
+
+def test_block_routing_baseline_matches_oracle():
+    """The contiguous-block baseline: blocks of consecutive keys with mean
+    representatives instead of k-means clusters, the rest of the path
+    unchanged; index state exact and sampled queries within tolerance."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=12288, T=2048, refit_period=0, budget=2048,
+                  k=128, M=256, block_routing=True)
+    st = _run_prefill(wl, sample=24, check_exhaustive=False)
+    assert st["cand_equal"] > 0, st
 
 
 def test_synchronous_refit_matches_oracle():
