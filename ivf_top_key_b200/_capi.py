@@ -46,6 +46,7 @@ class AiConfig(ctypes.Structure):
         ("max_budget", ctypes.c_int32), ("max_k", ctypes.c_int32),
         ("max_keys", ctypes.c_int64), ("seed", ctypes.c_uint64),
         ("encoder_weights_host", ctypes.POINTER(ctypes.c_float)),
+        ("block_routing", ctypes.c_int32),
     ]
 
 
@@ -85,7 +86,7 @@ def _load():
         "ai_quantize_fp8": [vp, i64, i32, vp, vp, vp],
         "ai_profile_enable": [vp, ctypes.c_int],
         "ai_profile_read": [vp, vp, vp],
-        "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp],
+        "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp, vp],
         "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
         "ai_debug_refine_kernel": [vp, i32],
         "ai_refine_kernel_choice": [vp, i32, ctypes.POINTER(i32)],
@@ -234,12 +235,13 @@ def ai_kernel_launches() -> int:
 
 
 def ai_select_exhaustive_noalloc(keys, key_dtype: int, q, w, pos0: int, k: int, out,
-                                 out_scores=None, stream=None):
-    """Exhaustive selection without any device allocation (see the header)."""
+                                 out_scores=None, status=None, stream=None):
+    """Exhaustive selection without any device allocation (see the header).
+    status: None or a 1-element int32 device tensor for the device flags."""
     n, d = keys.shape[0], keys.shape[1]
     _check(_lib.ai_select_exhaustive_noalloc(_ptr(keys), key_dtype, n, d, q.shape[1], _ptr(q), _ptr(w),
                                              pos0, q.shape[0], k, _ptr(out), _ptr(out_scores),
-                                             _stream(stream)))
+                                             _ptr(status), _stream(stream)))
     return out
 
 

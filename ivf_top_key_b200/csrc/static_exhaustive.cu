@@ -75,7 +75,8 @@ bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
 extern "C" int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_t n_keys,
                                             int32_t d, int32_t H, const void* q_dev, const float* w_dev,
                                             int64_t pos0, int32_t T, int32_t k, int32_t* out_dev,
-                                            float* out_scores_dev, void* cuda_stream) {
+                                            float* out_scores_dev, int32_t* status_dev,
+                                            void* cuda_stream) {
   using namespace aiidx;
   const bool tc = key_dtype == AI_BF16 && d == 128 && (H == 32 || H == 64);
   const bool simt = key_dtype == AI_FP32 && d > 0 && d % 8 == 0 && H > 0 && H <= 64 &&
@@ -85,7 +86,10 @@ extern "C" int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dt
     return fail_na(AI_ERR_ARG, "keys must be bf16 (d = 128, H in {32, 64}) or fp32 (queries of the same type)");
   if (n_keys <= 0 || n_keys > kMaxKeys) return fail_na(AI_ERR_ARG, "n_keys must be in [1, 1048576] (static scratch)");
   if (T <= 0 || k <= 0 || pos0 < 0) return fail_na(AI_ERR_ARG, "bad T, k or pos0");
+  if (k > kRowTopkMaxK) return fail_na(AI_ERR_ARG, "k above 4096");
   if (pos0 + T > n_keys) return fail_na(AI_ERR_CAUSALITY, "query positions beyond the keys");
+  if (tc && (reinterpret_cast<uintptr_t>(q_dev) % 16 != 0 || reinterpret_cast<uintptr_t>(w_dev) % 16 != 0))
+    return fail_na(AI_ERR_ARG, "q_dev and w_dev must be 16-byte aligned (bf16 keys)");
   float* scratch = nullptr;
   int rc = scratch_for_current_device(&scratch);
   if (rc) return rc;
@@ -122,12 +126,7 @@ extern "C" int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dt
       int dev = 0;
       cudaGetDevice(&dev);
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      const int qpt = 256 / H;
-      const int64_t qtiles = (tb + qpt - 1) / qpt;
-      const int64_t atiles = (nA + 127) / 128;
-      int64_t apc = (atiles * qtiles + 4 * sms - 1) / (4 * sms);
-      apc = apc < 1 ? 1 : (apc > atiles ? atiles : apc);
-      e = launch_scores_tc(ma, mb, H, sa, static_cast<int>(apc), st);
+      e = launch_scores_tc(ma, mb, H, sa, scores_tiles_per_item(nA, tb, H, sms), st);
     } else {
       e = launch_scores_simt(keys_dev, KD_FP32, qb, 0, d, H, sa, st);
     }
@@ -145,5 +144,11 @@ extern "C" int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dt
     e = launch_row_topk(ta, st);
     if (e != cudaSuccess) return fail_na(AI_ERR_CUDA, cudaGetErrorString(e));
   }
+  // the call's device flags (bounded-wait timeout, range, capacity) go to
+  // the caller's status word, in stream order: a 4-byte device-to-device
+  // copy, no allocation
+  if (status_dev &&
+      cudaMemcpyAsync(status_dev, err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return fail_na(AI_ERR_CUDA, "status copy failed");
   return AI_OK;
 }
