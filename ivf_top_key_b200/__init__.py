@@ -26,7 +26,8 @@ class AttentionIndex:
                  cluster_cap: int = 0, refit_period: int = 16384, refit_new_seeds: int = 0,
                  refit_seed_window: int = 0, seal_iters: int = 10, async_refit: bool = True,
                  max_query_chunk: int = 8192, max_budget: int = 8192, max_k: int = 2048,
-                 max_keys: int = 1 << 17, seed: int = 0, encoder_weights=None, stream=None):
+                 max_keys: int = 1 << 17, seed: int = 0, encoder_weights=None, stream=None,
+                 block_routing: bool = False):
         cfg = C.AiConfig()
         cfg.d, cfg.H = d, H
         cfg.key_dtype, cfg.q_dtype = C.DTYPES[key_dtype], C.DTYPES[q_dtype]
@@ -36,6 +37,7 @@ class AttentionIndex:
         cfg.seal_iters, cfg.async_refit = seal_iters, int(async_refit)
         cfg.max_query_chunk, cfg.max_budget, cfg.max_k = max_query_chunk, max_budget, max_k
         cfg.max_keys, cfg.seed = max_keys, seed
+        cfg.block_routing = int(block_routing)
         self._enc = None
         if encoder_weights is not None:
             import numpy as np

@@ -589,6 +589,34 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
   }
 }
 
+// Block seal (the contiguous-block baseline): CTA (window, block j) owns
+// keys [lo + floor(j W / m), lo + floor((j + 1) W / m)); its representative
+// is the float64 mean of those keys in ascending order, rounded once to
+// bf16.  Thread e sums dimensions e, e + blockDim, ...
+__global__ void __launch_bounds__(128) k_seal_blocks(SealArgs a) {
+  const int W = a.W, m = a.m, d = a.d;
+  const int win = blockIdx.x / m, j = blockIdx.x % m;
+  const int64_t lo = a.first_key + static_cast<int64_t>(win) * W;
+  const int b0 = static_cast<int>((static_cast<int64_t>(j) * W) / m);
+  const int b1 = static_cast<int>((static_cast<int64_t>(j + 1) * W) / m);
+  const int64_t mem0 = a.mem_base + static_cast<int64_t>(win) * W;
+  const int64_t cl = a.cl_base + static_cast<int64_t>(win) * m + j;
+  for (int i = b0 + threadIdx.x; i < b1; i += blockDim.x) a.members[mem0 + i] = static_cast<int32_t>(lo + i);
+  if (threadIdx.x == 0) {
+    a.offsets[cl] = static_cast<int32_t>(mem0 + b0);
+    if (blockIdx.x == gridDim.x - 1)
+      a.offsets[a.cl_base + static_cast<int64_t>(a.n_windows) * m] =
+          static_cast<int32_t>(a.mem_base + static_cast<int64_t>(a.n_windows) * W);
+  }
+  for (int e = threadIdx.x; e < d; e += blockDim.x) {
+    double acc = 0.0;
+    for (int i = b0; i < b1; ++i) acc += key_f64(a, lo + i, e);
+    const double c = b1 > b0 ? acc / static_cast<double>(b1 - b0) : 0.0;
+    a.centroids[cl * d + e] = c;
+    a.reps[cl * d + e] = f64_to_bf16_rne(c);
+  }
+}
+
 }  // namespace
 
 size_t seal_smem_bytes(int W, int m, int d) { return seal_layout(nullptr, W, m, d, nullptr) + 16; }
@@ -596,6 +624,11 @@ size_t seal_smem_bytes(int W, int m, int d) { return seal_layout(nullptr, W, m, 
 cudaError_t launch_seal(const SealArgs& a, cudaStream_t st) {
   if (a.n_windows <= 0) return cudaSuccess;
   if (a.m < 1 || a.m > 64 || a.W < 1 || a.W > 32767 || a.d % 8 != 0) return cudaErrorInvalidValue;
+  if (a.blocks) {
+    count_launch();
+    k_seal_blocks<<<a.n_windows * a.m, 128, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = seal_smem_bytes(a.W, a.m, a.d);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaFuncSetAttribute(k_seal, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -172,6 +172,23 @@ def seal_window(X: np.ndarray, m: int, cap: int, iters: int):
     return assign, C
 
 
+def seal_window_blocks(X: np.ndarray, m: int):
+    """The contiguous-block baseline the explainer compares against
+    ("它到底在解决什么问题？": HiSA groups keys by position into blocks, each
+    scored through one representative).  Reading: block j of a window of W
+    keys holds keys [floor(j W / m), floor((j + 1) W / m)), represented by
+    their mean.  Returns (assign [W], centroids [m, d] float64)."""
+    W = X.shape[0]
+    starts = [(j * W) // m for j in range(m + 1)]
+    assign = np.empty(W, dtype=np.int64)
+    C = np.zeros((m, X.shape[1]))
+    for j in range(m):
+        assign[starts[j]:starts[j + 1]] = j
+        if starts[j + 1] > starts[j]:
+            C[j] = X[starts[j]:starts[j + 1]].mean(axis=0)
+    return assign, C
+
+
 # ----------------------------------------------------------------- refit --
 
 def splitmix64(seed: int, ctr: int) -> int:
@@ -283,7 +300,7 @@ class OracleIndex:
 
     def __init__(self, *, d, n_sinks, window, clusters_per_window, refit_period,
                  refit_new_seeds=0, refit_seed_window=0, seal_iters=10, seed=0,
-                 encoder=None, cluster_cap=0):
+                 encoder=None, cluster_cap=0, block_routing=False):
         self.d = d
         self.S = n_sinks
         self.W = window
@@ -295,6 +312,9 @@ class OracleIndex:
         self.iters = seal_iters
         self.seed = seed
         self.encoder = encoder
+        self.block_routing = block_routing
+        if block_routing and (refit_period or encoder is not None):
+            raise ValueError("block routing takes no refit and no encoder")
         self.keys = np.zeros((0, d))
         self.n_windows = 0
         self.clusters: list[Cluster] = []
@@ -323,7 +343,10 @@ class OracleIndex:
         while self.keys.shape[0] >= self.S + (self.n_windows + 1) * self.W:
             lo = self.S + self.n_windows * self.W
             X = self.keys[lo:lo + self.W]
-            assign, C = seal_window(X, self.m, self.cap, self.iters)
+            if self.block_routing:
+                assign, C = seal_window_blocks(X, self.m)
+            else:
+                assign, C = seal_window(X, self.m, self.cap, self.iters)
             for j in range(self.m):
                 mem = lo + np.nonzero(assign == j)[0]
                 self.clusters.append(self._make_cluster(C[j], mem))

@@ -54,6 +54,7 @@ class Workload:
     refit_seed_window: int = 0    # 0 -> R
     seal_iters: int = 10
     encoder: str = "none"         # "none" | "random" | "zero_out"
+    block_routing: bool = False   # contiguous-block baseline instead of the IVF index
 
     @property
     def n_chunks(self) -> int:

@@ -444,3 +444,23 @@ def test_candidate_fill_order_by_hand(t, C, want):
     # route+refine on this state returns ids drawn from exactly that list
     ids, _ = idx.route_refine(q, w, t, k=len(want), C=C)
     assert sorted(ids[ids >= 0].tolist()) == sorted(want)
+
+
+def test_block_seal_by_hand():
+    """Contiguous-block baseline (explainer, 它到底在解决什么问题？: HiSA groups
+    keys by position): a window of 10 one-dimensional keys cut into m = 3
+    blocks of consecutive keys, [0, 3), [3, 6), [6, 10), each represented by
+    its mean."""
+    X = np.array([[1.0], [2.0], [6.0], [0.0], [0.0], [3.0], [4.0], [4.0], [8.0], [-4.0]])
+    assign, C = O.seal_window_blocks(X, 3)
+    assert assign.tolist() == [0, 0, 0, 1, 1, 1, 2, 2, 2, 2]
+    assert C[:, 0].tolist() == [3.0, 1.0, 3.0]
+    idx = O.OracleIndex(d=1, n_sinks=2, window=10, clusters_per_window=3, refit_period=0,
+                        block_routing=True)
+    idx.append(np.concatenate([np.zeros((2, 1)), X, np.ones((3, 1))]))
+    idx.seal()
+    assert [c.members.tolist() for c in idx.clusters] == [[2, 3, 4], [5, 6, 7], [8, 9, 10, 11]]
+    assert [(v.n_clusters, v.n_v) for v in idx.versions] == [(3, 12)]
+    with pytest.raises(ValueError):
+        O.OracleIndex(d=1, n_sinks=2, window=10, clusters_per_window=3, refit_period=10,
+                      block_routing=True)
