@@ -61,6 +61,9 @@ def parse():
                    help="also time one refit (64 seeds from the last 16384 keys) alone, the route "
                         "alone and both together, and report the hidden fraction")
     p.add_argument("--exh-reps", type=int, default=10, help="timed exhaustive calls (after one warm-up)")
+    p.add_argument("--decode", type=int, default=0,
+                   help="also time N decode steps after the prefill (one key appended, one query "
+                        "selected per step) with route+refine and with the exhaustive selection")
     p.add_argument("--no-1m", dest="with_1m", action="store_false",
                    help="skip the 1M-key sub-result of the default workload")
     return p.parse_args()
@@ -557,6 +560,69 @@ def measure_e2e(idx, chunks, wl, out, stream, flush, steps, warmup, world, units
             "ms_per_step": e_ms / steps}
 
 
+def measure_decode(wl, args, dev, stream, n_steps):
+    """Decode after a full prefill of the workload: every step appends the
+    next key, seals (a window completes every W steps; refits follow their
+    period) and selects the top-k of one query at the newest position.
+    The same steps are timed with route+refine and with the exhaustive
+    selection (the index is rolled back between the two); CUDA events
+    around all steps."""
+    import torch
+    from ivf_top_key_b200 import AttentionIndex
+    T, L = wl.T, wl.L
+    wl_d = S.scaled(wl, L=L + n_steps)
+    idx = AttentionIndex(d=wl.d, H=wl.H, key_dtype=wl.key_dtype, q_dtype=wl.q_dtype,
+                         n_sinks=wl.n_sinks, window=wl.window,
+                         clusters_per_window=wl.clusters_per_window,
+                         refit_period=wl.refit_period, seal_iters=wl.seal_iters, async_refit=True,
+                         max_query_chunk=T, max_budget=wl.budget, max_k=wl.k, max_keys=L + n_steps,
+                         seed=wl.seed, block_routing=wl.block_routing)
+    for c in range(wl.n_chunks):
+        kd, ks = chunk_keys_dev(wl, c * T, (c + 1) * T, dev)
+        idx.append_keys(kd, ks)
+        idx.seal()
+    idx.publish()
+    idx.sync()
+    idx.checkpoint()
+    kd, ks = chunk_keys_dev(wl_d, L, L + n_steps, dev)
+    qd, wd = queries_dev(wl_d, L, L + n_steps, dev)
+    out = torch.empty((1, wl.k), dtype=torch.int32, device=dev)
+
+    def run(select, n):
+        for i in range(n):
+            idx.append_keys(kd[i:i + 1], None if ks is None else ks[i:i + 1])
+            idx.seal()
+            select(qd[i:i + 1], wd[i:i + 1], L + i)
+        idx.publish()
+
+    def rr(q, w, t):
+        idx.route_refine(q, w, t, wl.k, wl.budget, out=out)
+
+    def ex(q, w, t):
+        idx.select_exhaustive(q, w, t, wl.k, out=out)
+
+    res = {}
+    for name, fn in (("route_refine", rr), ("exhaustive", ex)):
+        idx.rollback()
+        run(fn, min(8, n_steps))  # warm-up
+        idx.sync()
+        idx.rollback()
+        idx.sync()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(fn, n_steps)
+        e1.record(stream)
+        idx.sync()
+        ms = e0.elapsed_time(e1)
+        res[name] = {"us_per_token": round(ms * 1e3 / n_steps, 2),
+                     "tokens_per_s": round(n_steps / (ms / 1e3), 1)}
+    idx.close()
+    return {"workload": wl.name, "prefix_tokens": L, "steps": n_steps, "batch": 1,
+            "step": "append one key + seal (+ refit on its period) + select for one query",
+            **res, "speedup_vs_exhaustive": round(res["exhaustive"]["us_per_token"] /
+                                                  res["route_refine"]["us_per_token"], 2)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -595,6 +661,7 @@ def run_ours(args):
               "frac": round(ach / l2p, 4),
               "peak_source": "torch copy of a 24 MiB L2-resident buffer, best of 50 (read + write bytes)",
               "note": f"key store {wl.L * wl.d * 2 >> 20} MiB fits L2: rows are served from L2"}
+    dec = measure_decode(wl, args, dev, stream, args.decode) if args.decode else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_baseline(wl, args.cpu_sample)
@@ -617,6 +684,8 @@ def run_ours(args):
             "clocks": r["clocks"], "e2e": r["e2e"], "cpu_baseline": cpu,
             "wall_s_timed_region": round(r["wall_s"], 3),
         }
+        if dec is not None:
+            line["decode"] = dec
         if r1m is not None:
             line["at_1m"] = {
                 "workload": "glm_bf16_L1m", "prefix_tokens": wl1.L, "clusters": r1m["nC"],

@@ -172,6 +172,49 @@ def test_block_routing_baseline_matches_oracle():
     assert st["cand_equal"] > 0, st
 
 
+def test_decode_steps_match_oracle():
+    """Decode (explainer, 我认为它的局限, item 1): after a chunked prefill,
+    every step appends one key, seals when a window completes (and refits
+    on its period), and selects for one query (T = 1) at the newest
+    position.  Index state and sampled steps match the oracle, including
+    the steps right after a seal and a refit."""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=8192, T=2048, window=256, clusters_per_window=2,
+                  refit_period=1024, budget=1500, k=128, M=256)
+    n_dec = 1100
+    gpu, orc = P.make_pair(wl, max_keys=wl.L + n_dec)
+    for c in range(wl.n_chunks):
+        kd, ks, kv = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        orc.append(kv)
+        gpu.seal()
+        orc.seal()
+    wl_d = S.scaled(wl, L=wl.L + n_dec)
+    kd_all, ks_all, kv_all = P.keys_inputs(wl_d, wl.L, wl.L + n_dec)
+    qd_all, wd_all, qv_all, wv_all = P.query_inputs(wl_d, wl.L, wl.L + n_dec)
+    stats = collections.Counter()
+    checked = 0
+    for i in range(n_dec):
+        t = wl.L + i
+        gpu.append_keys(kd_all[i:i + 1], None if ks_all is None else ks_all[i:i + 1])
+        orc.append(kv_all[i:i + 1])
+        gpu.seal()
+        orc.seal()
+        out = torch.full((1, wl.k), -7, dtype=torch.int32, device="cuda")
+        osc = torch.zeros((1, wl.k), dtype=torch.float32, device="cuda")
+        gpu.route_refine(qd_all[i:i + 1], wd_all[i:i + 1], t, wl.k, wl.budget, out=out, out_scores=osc)
+        if i % 97 == 0 or (t + 1 - wl.n_sinks) % wl.window in (0, 1):
+            cand, _ = gpu.debug_candidates(qd_all[i:i + 1], wd_all[i:i + 1], t, wl.budget, with_scores=False)
+            gpu.sync()
+            P.check_queries(orc, [t], qv_all[i:i + 1], wv_all[i:i + 1], out.cpu().numpy(),
+                            osc.cpu().numpy(), cand.cpu().numpy(), wl.k, wl.budget, stats)
+            checked += 1
+    gpu.sync()
+    P.check_index_equal(gpu, orc)
+    assert gpu.stats()["n_refits"] == orc.n_refits > wl.L // wl.refit_period - 1
+    assert checked >= 15 and stats["cand_equal"] > 0, stats
+    gpu.close()
+
+
 def test_synchronous_refit_matches_oracle():
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=10240, T=2048, refit_period=4096,
                   budget=2048, k=128, M=128)
