@@ -205,7 +205,8 @@ int ai_rollback(ai_handle h);
 #define AI_PHASE_PUBLISH 4     /* wait for the refit + tail copy              */
 #define AI_PHASE_EXH_SCORES 5  /* exhaustive score GEMM                       */
 #define AI_PHASE_EXH_TOPK 6    /* exhaustive row top-k                        */
-#define AI_N_PHASES 7
+#define AI_PHASE_ORDER 7       /* route+refine output ordering (tensor core)  */
+#define AI_N_PHASES 8
 int ai_profile_enable(ai_handle h, int enable);
 /* Waits for the handle's streams, then writes the summed milliseconds and
  * the number of timed launches per phase (arrays of AI_N_PHASES, nullable)

@@ -32,7 +32,7 @@ EXPORTED = [
     "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
     "ai_debug_refine_kernel", "ai_refine_kernel_choice",
 ]
-PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk"]
+PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk", "order"]
 
 
 class AiConfig(ctypes.Structure):

@@ -199,6 +199,7 @@ struct ai_index {
   uint16_t* cent_lo = nullptr;
   float* cent_cc = nullptr;
   int32_t* cand_scratch = nullptr;  // tensor-core refine: candidate lists, 4 per SM
+  float* topk_scores = nullptr;      // tensor-core refine: scores for the output ordering [max_query_chunk, max_k]
   int refine_kernel = 0;             // tensor-core refine variant (0 = by occupancy)
   int32_t* upd_chunk_off = nullptr;  // refit update chunks
   double* upd_part = nullptr;
@@ -681,6 +682,7 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   CKC(dalloc(&h->scan_words, 16));
   // one candidate row per refine CTA (at most 4 per SM)
   if (tck) CKC(dalloc(&h->cand_scratch, static_cast<size_t>(h->num_sms) * 4 * c.max_budget));
+  if (tck) CKC(dalloc(&h->topk_scores, static_cast<size_t>(c.max_query_chunk) * c.max_k));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
   CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
   if ((c.key_dtype == AI_BF16 || c.key_dtype == AI_FP8E4M3) && d == 128 && c.refit_period > 0) {
@@ -735,6 +737,7 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->cent_lo);
   cudaFree(h->cent_cc);
   cudaFree(h->cand_scratch);
+  cudaFree(h->topk_scores);
   cudaFree(h->upd_chunk_off);
   cudaFree(h->upd_part);
   cudaFree(h->band_best);
@@ -897,9 +900,22 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
     kmp = &kmap;
     qmp = &qmap;
   }
+  // the tensor-core refine writes each row's ids (and scores) in slot
+  // order; a second kernel puts them in the output order, reading the
+  // scores from the caller's buffer or the handle's scratch
+  const bool order = tc_keys(h) && !cand_out;
+  float* sc_rows = out_scores;
+  if (order && !sc_rows) sc_rows = h->topk_scores;
+  ra.out_scores = order ? sc_rows : out_scores;
   const int pf = prof_begin(h, AI_PHASE_REFINE, h->main);
   CK(launch_refine(ra, vt, kmp, qmp, h->num_sms, h->main));
   prof_end(h, pf, h->main);
+  if (order) {
+    OrderRowsArgs oa{ra.out, sc_rows, ra.out, out_scores, T, k};
+    const int po = prof_begin(h, AI_PHASE_ORDER, h->main);
+    CK(launch_order_rows(oa, h->main));
+    prof_end(h, po, h->main);
+  }
   if (tmp_out) CK(cudaFreeAsync(tmp_out, h->main));
   return AI_OK;
 }

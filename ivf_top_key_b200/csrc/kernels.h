@@ -91,6 +91,19 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
 constexpr int kRowTopkMaxK = 4096;
 constexpr int kTcMaxK = 2048;
 
+// ------------------------------------------------ route+refine output order
+// Sorts each row of [T, k] (ids, scores) -- valid entries a prefix, -1
+// padding after -- by (score desc, id asc).  In place is allowed
+// (ids_out == ids_in, scores_out == scores_in); scores_out may be nullptr.
+struct OrderRowsArgs {
+  const int32_t* ids_in;
+  const float* scores_in;
+  int32_t* ids_out;
+  float* scores_out;
+  int T, k;
+};
+cudaError_t launch_order_rows(const OrderRowsArgs& a, cudaStream_t st);
+
 // ------------------------------------------------------- exhaustive top-k
 struct RowTopkArgs {
   const float* scores;  // [T, ld]

@@ -507,12 +507,10 @@ __global__ void __launch_bounds__(kSimtThreads) k_refine_simt(RefineArgs a, Vers
 // select over the same items.  Ties at the threshold go to the lower key id.
 constexpr int kNB = 2048;     // histogram bins
 constexpr int kCapB = 2048;   // items of the threshold bin sorted in smem (>= k/2)
-constexpr int kMaxBinSort = 96;  // output sort: largest score bin ranked by comparisons
 
 struct P3Smem {
   uint32_t hist[kNB];
   uint64_t buf[kCapB];
-  int32_t perm[kCapB];   // output sort: staged items grouped by score bin
   float fred[8];
   int ired[8];
   int scal[8];
@@ -810,8 +808,9 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       theta_id = static_cast<int>(~idk);
     }
   }
-  // emission: the selected items are staged in shared memory, sorted into
-  // the output order and written out coalesced.  Selection is v >= theta
+  // emission: ids (and scores) staged in shared memory in thread-major
+  // order, then written out coalesced; a follow-up kernel (order_rows.cu)
+  // puts every row in the output order.  Selection is v >= theta
   // (everything when all items are kept), except when only some of the
   // items tied at theta are kept: then v > theta or (v == theta and id <=
   // theta_id).  Bodies are branch-free; unselected items write to a
@@ -833,18 +832,16 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
   }
   int total;
   int pos = p3_scan(mine, et, &total, ps);
-  // staging: every selected item becomes a 64-bit order key (score desc,
-  // id asc) at its thread-order position; the id load is predicated (an
-  // unselected item reads entry 0), unselected items write a per-thread
-  // dummy slot, so the body stays branch-free
-  static_assert(kCapB >= 2048, "the output sort holds k <= 2048 keys");
-  uint64_t* keys = ps.buf;
-  uint64_t* dump = reinterpret_cast<uint64_t*>(ps.hist) + et;
-  auto stage = [&pos, keys, dump, k, cd, nlast](float v, int slot, int f) {
+  int32_t* sid = reinterpret_cast<int32_t*>(ps.buf);          // [k] slots
+  float* ssc = reinterpret_cast<float*>(ps.buf) + kCapB;       // [k] scores
+  int32_t* dump_id = reinterpret_cast<int32_t*>(ps.hist) + et;
+  float* dump_sc = reinterpret_cast<float*>(ps.hist) + 128 + et;
+  auto stage = [&pos, sid, ssc, dump_id, dump_sc, k](float v, int slot, int f) {
     const bool w = (f & static_cast<int>(pos < k)) != 0;
-    const int sl = (w && slot <= nlast) ? slot : 0;
-    const int32_t id = cd[sl];
-    *(w ? keys + pos : dump) = order_key(v, id);
+    int32_t* pi = w ? sid + pos : dump_id;
+    float* pv = w ? ssc + pos : dump_sc;
+    *pi = slot;
+    *pv = v;
     pos += f;
   };
   if (!partial_ties) {
@@ -857,92 +854,25 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
       stage(v, slot, ok & (static_cast<int>(v > th) | (v == th ? static_cast<int>(cd[sl] <= thid) : 0)));
     });
   }
-  // output order (score desc, id asc) by a counting sort: the staged keys
-  // are grouped by score bin (highest bin first), then each key takes its
-  // rank inside its bin by comparing with the bin's other keys.  Bins split
-  // the order-preserving integer keys of [lowest selected score, vmax] into
-  // at most kNB equal ranges: about constant relative width, so a few
-  // outlying high scores do not crowd the bulk into one bin.  A bin holding
-  // more than kMaxBinSort keys (near-equal scores) sends the whole list
-  // through a bitonic sort instead.
+  named_bar(1, 128);
   const int nw = min(total, k);
-  const uint32_t klo = f2key(th == -INFINITY ? vmin : th);
-  const uint32_t krange = f2key(vmax) - klo;
-  int kshift = 0;
-  while (kshift < 32 && (static_cast<uint64_t>(krange) >> kshift) >= static_cast<uint64_t>(kNB)) ++kshift;
-  auto sbin = [=](uint64_t x) -> int {
-    const uint32_t d = ~static_cast<uint32_t>(x >> 32) - klo;  // f2key(score) - klo
-    const uint32_t b = kshift < 32 ? d >> kshift : 0u;
-    return b < static_cast<uint32_t>(kNB) ? static_cast<int>(b) : kNB - 1;
-  };
-  named_bar(1, 128);  // staging done (its dummy slots overlap the histogram)
-  for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
-  named_bar(1, 128);
-  for (int j = et; j < nw; j += 128) atomicAdd(&ps.hist[sbin(keys[j])], 1u);
-  named_bar(1, 128);
-  // bin starts in descending bin order: thread et owns bins 2047 - 16 et - u
-  int cnt16 = 0, cmax = 0;
+  // the ids of a thread's outputs are all loaded before any is stored (the
+  // stores could alias the list, so the compiler would not reorder them)
+  for (int j0 = et; j0 < k; j0 += 8 * 128) {
+    int32_t id[8];
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int c = static_cast<int>(ps.hist[kNB - 1 - (16 * et + u)]);
-    cnt16 += c;
-    cmax = max(cmax, c);
-  }
-  int all_total;
-  int run = p3_scan(cnt16, et, &all_total, ps);
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 128;
+      id[u] = j < nw ? cd[sid[j]] : -1;
+    }
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int b = kNB - 1 - (16 * et + u);
-    const int c = static_cast<int>(ps.hist[b]);
-    ps.hist[b] = static_cast<uint32_t>(run);  // start of bin b
-    run += c;
-  }
-  for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-  if ((et & 31) == 0) ps.ired[4 + (et >> 5)] = cmax;
-  named_bar(1, 128);
-  const int bin_max = max(max(ps.ired[4], ps.ired[5]), max(ps.ired[6], ps.ired[7]));
-  if (bin_max <= kMaxBinSort) {
-    // group by bin (after this, bin b spans [end of bin b + 1, hist[b]))
-    for (int j = et; j < nw; j += 128) {
-      const int p = static_cast<int>(atomicAdd(&ps.hist[sbin(keys[j])], 1u));
-      ps.perm[p] = j;
-    }
-    named_bar(1, 128);
-    for (int p = et; p < nw; p += 128) {
-      const uint64_t x = keys[ps.perm[p]];
-      const int b = sbin(x);
-      const int lo = b == kNB - 1 ? 0 : static_cast<int>(ps.hist[b + 1]);
-      const int hi = static_cast<int>(ps.hist[b]);
-      int r = lo;
-      for (int q = lo; q < hi; ++q) r += keys[ps.perm[q]] < x ? 1 : 0;
-      out[r] = order_key_id(x);
-      if (outs) outs[r] = order_key_score(x);
-    }
-  } else {
-    int np = 1;
-    while (np < nw) np <<= 1;
-    for (int i = nw + et; i < np; i += 128) keys[i] = kOrderPad;
-    named_bar(1, 128);
-    for (int kk = 2; kk <= np; kk <<= 1) {
-      for (int j = kk >> 1; j > 0; j >>= 1) {
-        for (int p = et; p < (np >> 1); p += 128) {
-          const int i = ((p & ~(j - 1)) << 1) | (p & (j - 1));  // lower element of pair p
-          const uint64_t x = keys[i], y = keys[i + j];
-          const bool swp = ((i & kk) == 0) ? (x > y) : (x < y);
-          keys[i] = swp ? y : x;  // both written: no divergent branch
-          keys[i + j] = swp ? x : y;
-        }
-        named_bar(1, 128);
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 128;
+      if (j < k) {
+        out[j] = id[u];
+        if (outs) outs[j] = j < nw ? ssc[j] : -INFINITY;
       }
     }
-    for (int j = et; j < nw; j += 128) {
-      out[j] = order_key_id(keys[j]);
-      if (outs) outs[j] = order_key_score(keys[j]);
-    }
-  }
-  for (int j = nw + et; j < k; j += 128) {
-    out[j] = -1;
-    if (outs) outs[j] = -INFINITY;
   }
   named_bar(1, 128);
 }

@@ -165,69 +165,6 @@ __device__ __forceinline__ void block_sort_u64(uint64_t* buf, int np) {
   }
 }
 
-// Position of element i of a 2048-key array in shared memory: pairs of keys
-// (16 bytes) are XOR-swizzled inside each group of 16 keys, so a warp whose
-// lanes each touch their own 16 consecutive keys spreads over all banks.
-__device__ __forceinline__ int sw2048(int i) { return ((((i >> 1) ^ (i >> 4)) & 7) | ((i >> 1) & ~7)) << 1 | (i & 1); }
-
-__device__ __forceinline__ void cmpx_u64(uint64_t& a, uint64_t& b, bool asc) {
-  const bool swp = asc ? (a > b) : (a < b);
-  const uint64_t lo = swp ? b : a, hi = swp ? a : b;
-  a = lo;
-  b = hi;
-}
-template <int J>
-__device__ __forceinline__ void sort2048_reg_stage(uint64_t (&x)[16], int et, int kk) {
-#pragma unroll
-  for (int e = 0; e < 16; ++e)
-    if ((e & J) == 0) cmpx_u64(x[e], x[e | J], ((16 * et + e) & kk) == 0);
-}
-
-// Bitonic sort, ascending, of 2048 64-bit keys held by the 128 threads
-// et = 0 .. 127 of a named-barrier group, 16 per thread: element
-// i = 16 et + e is x[e].  Stages whose partner lies in the same thread run in
-// registers, those in another lane of the warp use shuffles, and the three
-// whose partner is in another warp exchange through xb (2048 keys of shared
-// memory, swizzled by sw2048).  Afterwards x holds elements 16 et .. 16 et + 15
-// of the sorted order.
-template <int BAR>
-__device__ __forceinline__ void sort2048_regs(uint64_t (&x)[16], uint64_t* xb, int et) {
-  for (int kk = 2; kk <= 2048; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      if (j >= 16) {
-        const int m = j >> 4;  // thread distance
-        const bool keep_min = ((et & m) == 0) == (((16 * et) & kk) == 0);
-        if (m < 32) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t y = __shfl_xor_sync(0xffffffffu, x[e], m);
-            x[e] = keep_min ? (x[e] < y ? x[e] : y) : (x[e] < y ? y : x[e]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) xb[sw2048(16 * et + e)] = x[e];
-          named_bar(BAR, 128);
-          const int pt = et ^ m;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t y = xb[sw2048(16 * pt + e)];
-            x[e] = keep_min ? (x[e] < y ? x[e] : y) : (x[e] < y ? y : x[e]);
-          }
-          named_bar(BAR, 128);
-        }
-      } else if (j == 8) {
-        sort2048_reg_stage<8>(x, et, kk);
-      } else if (j == 4) {
-        sort2048_reg_stage<4>(x, et, kk);
-      } else if (j == 2) {
-        sort2048_reg_stage<2>(x, et, kk);
-      } else {
-        sort2048_reg_stage<1>(x, et, kk);
-      }
-    }
-  }
-}
-
 // Top-k of n items (score(i), id(i)) by (score desc, id asc).  Writes the
 // selected ids (and scores) in that order, then pads with -1 / -inf up to
 // k.  sbuf: shared memory for the next power of two >= k keys.  All
