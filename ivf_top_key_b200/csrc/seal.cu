@@ -58,6 +58,8 @@ struct SealSmem {
   int16_t* prev;     // [W]
   int16_t* mlist;    // [W] members, grouped by cluster, ascending
   int16_t* coll;     // [m, W] proposals in each cluster's target bin
+  uint16_t* bin;     // [m, W] histogram bin of D[j, i] for this pass
+  uint32_t* ord;     // [W] (m <= 8) clusters of key i by (D asc, j asc), 4 bits each
 };
 
 // Lays the arrays out from p; returns the bytes used.  Shared by the kernel
@@ -89,6 +91,8 @@ __host__ __device__ inline size_t seal_layout(uint8_t* p, int W, int m, int d, S
   uint8_t* prev = take(static_cast<size_t>(W) * 2);
   uint8_t* mlist = take(static_cast<size_t>(W) * 2);
   uint8_t* coll = take(static_cast<size_t>(W) * m * 2);
+  uint8_t* bin = take(static_cast<size_t>(W) * m * 2);
+  uint8_t* ord = take(static_cast<size_t>(W) * 4);
   if (s) {
     s->D = reinterpret_cast<double*>(D);
     s->cent = reinterpret_cast<double*>(cent);
@@ -110,6 +114,8 @@ __host__ __device__ inline size_t seal_layout(uint8_t* p, int W, int m, int d, S
     s->prev = reinterpret_cast<int16_t*>(prev);
     s->mlist = reinterpret_cast<int16_t*>(mlist);
     s->coll = reinterpret_cast<int16_t*>(coll);
+    s->bin = reinterpret_cast<uint16_t*>(bin);
+    s->ord = reinterpret_cast<uint32_t*>(ord);
   }
   return o;
 }
@@ -200,14 +206,21 @@ __device__ __forceinline__ void seal_dist(const SealArgs& a, const SealSmem& s, 
       acc0[j] = 0.0;
       acc1[j] = 0.0;
     }
+    // bf16 rows: the next 8-element block of both rows is loaded while the
+    // current one is used (the rows come from L2 on every pass)
+    const uint4* kp = kBf16 ? reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.keys) +
+                                                             (lo + i0) * d)
+                            : nullptr;
+    uint4 n0 = kBf16 ? __ldg(kp) : make_uint4(0, 0, 0, 0);
+    uint4 n1 = kBf16 && two ? __ldg(kp + d / 8) : make_uint4(0, 0, 0, 0);
     for (int e0 = 0; e0 < d; e0 += 8) {
       double x0[8], x1[8];
       if (kBf16) {
-        // both rows' 16-byte loads issued before any use
-        const uint4* kp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.keys) +
-                                                         (lo + i0) * d + e0);
-        const uint4 v0 = __ldg(kp);
-        const uint4 v1 = two ? __ldg(kp + d / 8) : make_uint4(0, 0, 0, 0);
+        const uint4 v0 = n0, v1 = n1;
+        if (e0 + 8 < d) {
+          n0 = __ldg(kp + (e0 + 8) / 8);
+          if (two) n1 = __ldg(kp + d / 8 + (e0 + 8) / 8);
+        }
         const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -339,6 +352,40 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       }
     }
     __syncthreads();
+    // fixed for the pass: every pair's histogram bin and (m <= 8) every
+    // key's clusters in (distance, cluster) order, so that a round only
+    // skips the clusters that have filled
+    for (int e = tid; e < m * W; e += blockDim.x) s.bin[e] = static_cast<uint16_t>(dist_bin(s, e / W, s.D[e]));
+    if (m <= 8) {
+      for (int i = tid; i < W; i += blockDim.x) {
+        double dv[8];
+        int jv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          dv[j] = j < m ? s.D[j * W + i] : INFINITY;
+          jv[j] = j;
+        }
+        // insertion by (distance, cluster): the order of the first-minimum scan
+#pragma unroll
+        for (int a1 = 1; a1 < 8; ++a1) {
+#pragma unroll
+          for (int b1 = a1; b1 > 0; --b1) {
+            const bool sw = dv[b1] < dv[b1 - 1];
+            const double td = sw ? dv[b1 - 1] : dv[b1];
+            const int tj = sw ? jv[b1 - 1] : jv[b1];
+            dv[b1 - 1] = sw ? dv[b1] : dv[b1 - 1];
+            jv[b1 - 1] = sw ? jv[b1] : jv[b1 - 1];
+            dv[b1] = td;
+            jv[b1] = tj;
+          }
+        }
+        uint32_t o = 0;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) o = (o << 4) | static_cast<uint32_t>(jv[j]);
+        s.ord[i] = o;
+      }
+    }
+    __syncthreads();
 
     // greedy capacity assignment in rounds (see the file comment)
     for (int round = 0; round <= m && s.misc[2] > 0; ++round) {
@@ -346,19 +393,28 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       // B. proposals: best open cluster of every free key, counted per bin
       for (int i = tid; i < W; i += blockDim.x) {
         int bj = -1;
-        double bd = 0.0;
         if (s.assign[i] < 0) {
-          for (int j = 0; j < m; ++j) {
-            if ((fullm >> j) & 1ull) continue;
-            const double v = s.D[j * W + i];
-            if (bj < 0 || v < bd) {
-              bj = j;
-              bd = v;
+          if (m <= 8) {
+            // pop the clusters that filled since the last round (they stay full)
+            uint32_t o = s.ord[i];
+            for (int g = 0; g < m && ((fullm >> (o & 15u)) & 1ull); ++g) o >>= 4;
+            s.ord[i] = o;
+            const int oj = static_cast<int>(o & 15u);
+            bj = (oj < m && !((fullm >> oj) & 1ull)) ? oj : -1;
+          } else {
+            double bd = 0.0;
+            for (int j = 0; j < m; ++j) {
+              if ((fullm >> j) & 1ull) continue;
+              const double v = s.D[j * W + i];
+              if (bj < 0 || v < bd) {
+                bj = j;
+                bd = v;
+              }
             }
           }
         }
         s.prop[i] = static_cast<int8_t>(bj);
-        if (bj >= 0) atomicAdd(&s.hist[bj * kBins + dist_bin(s, bj, bd)], 1);
+        if (bj >= 0) atomicAdd(&s.hist[bj * kBins + s.bin[bj * W + i]], 1);
       }
       __syncthreads();
       // C. per open cluster, the bin where the running count reaches the
@@ -370,12 +426,11 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         if (!((fullm >> j) & 1ull)) {
           const int need = a.cap - s.cnt[j];
           int* hj = s.hist + j * kBins;
+          // lane l sums chunk l (bins 32 l .. 32 l + 31), reading the bins in
+          // a lane-skewed order so the warp's loads hit 32 different banks
           int csum = 0;
 #pragma unroll 8
-          for (int c = 0; c < 32; ++c) {
-            const int t = __reduce_add_sync(0xffffffffu, hj[c * 32 + lane]);
-            if (lane == c) csum = t;
-          }
+          for (int u = 0; u < 32; ++u) csum += hj[lane * 32 + ((u + lane) & 31)];
           int cin = csum;
           for (int o = 1; o < 32; o <<= 1) {
             const int t = __shfl_up_sync(0xffffffffu, cin, o);
@@ -411,7 +466,7 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
       // D. collect, per cluster, the proposals lying in its target bin
       for (int i = tid; i < W; i += blockDim.x) {
         const int j = s.prop[i];
-        if (j >= 0 && s.tb[j] >= 0 && dist_bin(s, j, s.D[j * W + i]) == s.tb[j])
+        if (j >= 0 && s.tb[j] >= 0 && static_cast<int>(s.bin[j * W + i]) == s.tb[j])
           s.coll[j * W + atomicAdd(&s.ncoll[j], 1)] = static_cast<int16_t>(i);
       }
       __syncthreads();
@@ -533,14 +588,25 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         if (a.key_dtype == KD_BF16) {
           // raw bf16 pairs: the loads of a batch are issued back to back
           const uint32_t* kp = reinterpret_cast<const uint32_t*>(a.keys) + (lo * d + e) / 2;
-          for (; q + 16 <= b1; q += 16) {
-            uint32_t r[16];
+          // batches of 16 member rows; the next batch is loaded while the
+          // current one is summed (in member order)
+          uint32_t r[16];
+          if (q + 16 <= b1) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) r[u] = __ldg(kp + static_cast<int64_t>(s.mlist[q + u]) * (d / 2));
+          }
+          for (; q + 16 <= b1; q += 16) {
+            uint32_t c[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) c[u] = r[u];
+            if (q + 32 <= b1) {
+#pragma unroll
+              for (int u = 0; u < 16; ++u) r[u] = __ldg(kp + static_cast<int64_t>(s.mlist[q + 16 + u]) * (d / 2));
+            }
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-              s0 += static_cast<double>(__uint_as_float(r[u] << 16));
-              s1 += static_cast<double>(__uint_as_float(r[u] & 0xFFFF0000u));
+              s0 += static_cast<double>(__uint_as_float(c[u] << 16));
+              s1 += static_cast<double>(__uint_as_float(c[u] & 0xFFFF0000u));
             }
           }
         }

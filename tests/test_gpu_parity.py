@@ -215,6 +215,40 @@ def test_decode_steps_match_oracle():
     gpu.close()
 
 
+@pytest.mark.parametrize("variant", ["ivf_refit", "ivf_seal_only", "blocks"])
+def test_recall_ablation_agrees_with_oracle(variant):
+    """The recall behind the ablation tables (refit vs seal only vs the
+    contiguous-block baseline; explainer, 实验结果, ablation paragraph, and
+    它到底在解决什么问题？): recall of route+refine against exhaustive
+    selection on sampled queries of the last chunk, measured on the GPU
+    (library exhaustive) and by the oracle on the same queries, agree
+    within half a point."""
+    base = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=24576, T=4096, refit_period=8192, budget=2048,
+                    k=256, M=512)
+    wl = {"ivf_refit": base, "ivf_seal_only": S.scaled(base, refit_period=0),
+          "blocks": S.scaled(base, refit_period=0, block_routing=True)}[variant]
+    gpu, orc = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        kd, ks, kv = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        orc.append(kv)
+        gpu.seal()
+        orc.seal()
+    p0 = wl.L - wl.T
+    qd, wd, qv, wv = P.query_inputs(wl, p0, wl.L)
+    sel = gpu.route_refine(qd, wd, p0, wl.k, wl.budget)
+    exh = gpu.select_exhaustive(qd, wd, p0, wl.k)
+    gpu.sync()
+    idx = np.random.default_rng(7).choice(wl.T, size=24, replace=False)
+    sel, exh = sel.cpu().numpy()[idx], exh.cpu().numpy()[idx]
+    r_gpu = O.recall(sel, exh)
+    o_sel = np.stack([orc.route_refine(qv[i], wv[i], p0 + i, wl.k, wl.budget)[0] for i in idx])
+    o_exh = np.stack([orc.exhaustive(qv[i], wv[i], p0 + i, wl.k)[0] for i in idx])
+    r_orc = O.recall(o_sel, o_exh)
+    assert abs(r_gpu - r_orc) <= 0.005, (variant, r_gpu, r_orc)
+    gpu.close()
+
+
 def test_synchronous_refit_matches_oracle():
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=10240, T=2048, refit_period=4096,
                   budget=2048, k=128, M=128)
