@@ -66,6 +66,10 @@ def parse():
     p.add_argument("--decode", type=int, default=0,
                    help="also time N decode steps after the prefill (one key appended, one query "
                         "selected per step) with route+refine and with the exhaustive selection")
+    p.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+                   help="N > 1: replicas = an independent request per rank (weak scaling); sharded = one "
+                        "request, every rank rescoring its share of each candidate list, partial top-k "
+                        "all-gathered over NCCL and merged (strong scaling)")
     p.add_argument("--no-1m", dest="with_1m", action="store_false",
                    help="skip the 1M-key sub-result of the default workload")
     return p.parse_args()
@@ -82,7 +86,7 @@ def chunks_per_step(wl):
     return max(1, wl.refit_period // wl.T) if wl.refit_period else 1
 
 
-def config_block(wl, n):
+def config_block(wl, n, mode="replicas"):
     return {"workload": wl.name, "chunks_per_step": chunks_per_step(wl),
             "queries_per_step": chunks_per_step(wl) * wl.T, "prefix_tokens": wl.L, "chunk_queries": wl.T, "heads": wl.H,
             "head_dim": wl.d, "key_dtype": wl.key_dtype, "k": wl.k, "budget_C": wl.budget,
@@ -90,13 +94,15 @@ def config_block(wl, n):
             "refit_period_R": wl.refit_period, "sinks": wl.n_sinks,
             "routing": "contiguous blocks (baseline)" if wl.block_routing else "ivf",
             "step": "last R/T chunks: per chunk append + seal (+side-stream refit) + route/refine; then publish",
-            "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{n}"}
+            "l2": "flushed between steps (256 MiB write)",
+            "parallelism": f"cluster-sharded rescore x{n}" if mode == "sharded" and n > 1 else f"replicas x{n}"}
 
 
-def wl_for_rank(name, rank, budget=0, refit_period=-1, routing="ivf"):
-    """Every rank runs an independent request: same shapes, its own seed.
-    budget / refit_period / routing override the workload's (ablations)."""
-    wl = S.scaled(S.WORKLOADS[name], seed=rank)
+def wl_for_rank(name, rank, budget=0, refit_period=-1, routing="ivf", sharded=False):
+    """Every rank runs an independent request: same shapes, its own seed (or,
+    sharded, the same request on every rank).  budget / refit_period /
+    routing override the workload's (ablations)."""
+    wl = S.scaled(S.WORKLOADS[name], seed=0 if sharded else rank)
     if budget:
         wl = S.scaled(wl, budget=budget)
     if routing == "blocks":
@@ -331,11 +337,18 @@ def measure_workload(wl, args, dev, stream, world, steps, warmup, e2e_on, overla
     out = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    sharded = getattr(args, "mode", "replicas") == "sharded" and world > 1
+    if sharded:
+        from ivf_top_key_b200 import sharded as shd
+
     def step():
         for a, kd_, ks_, qd_, wd_ in chunks:
             idx.append_keys(kd_, ks_)
             idx.seal()
-            idx.route_refine(qd_, wd_, a, wl.k, wl.budget, out=out)
+            if sharded:
+                out.copy_(shd.sharded_route_refine(idx, qd_, wd_, a, wl.k, wl.budget))
+            else:
+                idx.route_refine(qd_, wd_, a, wl.k, wl.budget, out=out)
         idx.publish()
 
     for _ in range(warmup):
@@ -371,7 +384,8 @@ def measure_workload(wl, args, dev, stream, world, steps, warmup, e2e_on, overla
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(float(np.sum(step_ms)), dev)
     units = T * ncs                # query tokens per step
-    value = weak_scaling_value(units, steps, world, total_ms)
+    # sharded: the ranks share one request, so its queries count once
+    value = weak_scaling_value(units, steps, 1 if sharded else world, total_ms)
     st = idx.stats()
     nC = st["n_clusters"]
 
@@ -461,7 +475,8 @@ def measure_workload(wl, args, dev, stream, world, steps, warmup, e2e_on, overla
                     "ms_per_chunk": round(exh_ph["exh_scores"], 4)}
 
     # end to end through the public API with host buffers
-    e2e = measure_e2e(idx, chunks, wl, out, stream, flush, steps, warmup, world, units) if e2e_on else None
+    e2e = measure_e2e(idx, chunks, wl, out, stream, flush, steps, warmup, world, units) \
+        if e2e_on and not sharded else None
     refit_overlap = None
     if overlap_on:  # last: it moves the checkpoint to the full prefix
         refit_overlap = measure_refit_overlap(idx, chunks, wl, out, stream)
@@ -645,7 +660,8 @@ def run_ours(args):
     main_stream = torch.cuda.Stream(device=dev, priority=hi_pri)
     torch.cuda.set_stream(main_stream)
     stream = torch.cuda.current_stream()
-    wl = wl_for_rank(args.workload, rank, args.budget, args.refit_period, args.routing)
+    wl = wl_for_rank(args.workload, rank, args.budget, args.refit_period, args.routing,
+                     sharded=args.mode == "sharded" and world > 1)
     r = measure_workload(wl, args, dev, stream, world, args.steps, args.warmup, not args.no_e2e,
                          args.refit_overlap)
     # the 1M-key prefix (one final chunk routed over ~8200 clusters, plus
@@ -653,7 +669,7 @@ def run_ours(args):
     r1m = None
     if args.with_1m and args.workload == "glm_bf16_L128k" and args.routing == "ivf" and args.refit_period < 0 \
             and not args.budget:
-        wl1 = wl_for_rank("glm_bf16_L1m", rank, 0)
+        wl1 = wl_for_rank("glm_bf16_L1m", rank, 0, sharded=args.mode == "sharded" and world > 1)
         r1m = measure_workload(wl1, args, dev, stream, world, max(3, args.steps // 2), max(3, args.warmup),
                                False, True)
     l2 = None
@@ -675,9 +691,10 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if args.mode == "sharded" and world > 1 else "weak", "vs_baseline": None,
             "dtype": wl.key_dtype, "data": "synthetic (seeded Gaussian-mixture keys/queries)",
-            "config": config_block(wl, world),
+            "config": config_block(wl, world, args.mode),
             "recall_vs_exhaustive": round(r["recall"], 4) if r["recall"] is not None else None,
             "exhaustive": r["exhaustive"],
             "roofline": r["roofline"], "l2": l2, "roofline_route_gemm": r["roofline_route_gemm"],

@@ -141,6 +141,33 @@ int ai_publish(ai_handle h);
 int ai_route_refine(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
                     int32_t T, int32_t k, int32_t C, int32_t* out_dev, float* out_scores_dev);
 
+/* Sharded rescore for a cluster-sharded, several-GPU deployment (the
+ * review's "tensor-parallel index ownership", Impact Assessment: Core
+ * Contribution item 3; the explainer, 我认为它的局限 item 2, names the
+ * cross-GPU synchronisation).  Every rank holds the same index (maintenance
+ * is deterministic); for each query it builds the same candidate list and
+ * rescores only its share: the contiguous range of the list's 128-slot
+ * tiles with index shard of n_shards.  It writes that share's top k to
+ * out_dev / out_scores_dev [T, k] (both required), in (score desc, id asc)
+ * order, -1 / -inf padded.  The shards' lists hold disjoint ids and the
+ * union of their top k holds the query's top k: gathering the n_shards
+ * partial results and merging them with ai_merge_topk gives exactly
+ * ai_route_refine's output.  bf16 / fp8 keys (pipelined refine kernels)
+ * only; n_shards = 1 is ai_route_refine.  Errors as ai_route_refine, and
+ * AI_ERR_ARG for a bad shard.                                              */
+int ai_route_refine_shard(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0,
+                          int32_t T, int32_t k, int32_t C, int32_t shard, int32_t n_shards,
+                          int32_t* out_dev, float* out_scores_dev);
+
+/* Merge n_parts partial top-k results per query: ids_dev / scores_dev are
+ * [n_parts, T, k] (ids -1 where a part has fewer than k); writes the top k
+ * of each query's union by (score desc, id asc) to out_dev [T, k] (and
+ * out_scores_dev, nullable), -1 padded.  The parts must hold disjoint ids.
+ * Enqueued on cuda_stream; needs no handle and allocates nothing.  Limits:
+ * k <= 2048, (n_parts + 1) * k <= 29,000 (AI_ERR_ARG).                    */
+int ai_merge_topk(const int32_t* ids_dev, const float* scores_dev, int32_t n_parts, int32_t T,
+                  int32_t k, int32_t* out_dev, float* out_scores_dev, void* cuda_stream);
+
 /* Exhaustive selection (explainer, "它到底在解决什么问题？": the indexer
  * scores every key s <= t).  Same arguments and output order as
  * ai_route_refine (score descending, ties by id ascending, -1 padding).

@@ -15,7 +15,7 @@ import torch
 from . import _capi as C
 from ._capi import AiError  # noqa: F401
 
-__all__ = ["AttentionIndex", "AiError", "quantize_fp8", "C"]
+__all__ = ["AttentionIndex", "AiError", "quantize_fp8", "merge_topk", "C"]
 
 
 class AttentionIndex:
@@ -80,6 +80,16 @@ class AttentionIndex:
             out = torch.empty((q.shape[0], k), dtype=torch.int32, device=q.device)
         return C.ai_route_refine(self.h, q, w, pos0, k, C_budget, out, out_scores)
 
+    def route_refine_shard(self, q, w, pos0: int, k: int, C_budget: int, shard: int, n_shards: int,
+                           out=None, out_scores=None):
+        """This shard's top k of the sharded rescore (see ai_route_refine_shard)."""
+        T = q.shape[0]
+        if out is None:
+            out = torch.empty((T, k), dtype=torch.int32, device=q.device)
+        if out_scores is None:
+            out_scores = torch.empty((T, k), dtype=torch.float32, device=q.device)
+        return C.ai_route_refine_shard(self.h, q, w, pos0, k, C_budget, shard, n_shards, out, out_scores)
+
     def select_exhaustive(self, q, w, pos0: int, k: int, out=None, out_scores=None):
         if out is None:
             out = torch.empty((q.shape[0], k), dtype=torch.int32, device=q.device)
@@ -133,6 +143,14 @@ class AttentionIndex:
 
     def rollback(self):
         C.ai_rollback(self.h)
+
+
+def merge_topk(ids: torch.Tensor, scores: torch.Tensor, k: int, out=None, out_scores=None, stream=None):
+    """Top k of the union of n_parts partial results [n_parts, T, k] (library kernel)."""
+    T = ids.shape[1]
+    if out is None:
+        out = torch.empty((T, k), dtype=torch.int32, device=ids.device)
+    return C.ai_merge_topk(ids, scores, k, out, out_scores, stream)
 
 
 def quantize_fp8(keys_bf16: torch.Tensor, stream=None):

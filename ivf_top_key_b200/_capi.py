@@ -30,6 +30,7 @@ EXPORTED = [
     "ai_get_stats", "ai_export_index", "ai_debug_candidates", "ai_debug_scores",
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
     "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
+    "ai_route_refine_shard", "ai_merge_topk",
     "ai_debug_refine_kernel", "ai_refine_kernel_choice",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk", "order"]
@@ -87,6 +88,8 @@ def _load():
         "ai_profile_enable": [vp, ctypes.c_int],
         "ai_profile_read": [vp, vp, vp],
         "ai_select_exhaustive_noalloc": [vp, i32, i64, i32, i32, vp, vp, i64, i32, i32, vp, vp, vp, vp],
+        "ai_route_refine_shard": [vp, vp, vp, i64, i32, i32, i32, i32, i32, vp, vp],
+        "ai_merge_topk": [vp, vp, i32, i32, i32, vp, vp, vp],
         "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
         "ai_debug_refine_kernel": [vp, i32],
         "ai_refine_kernel_choice": [vp, i32, ctypes.POINTER(i32)],
@@ -242,6 +245,19 @@ def ai_select_exhaustive_noalloc(keys, key_dtype: int, q, w, pos0: int, k: int, 
     _check(_lib.ai_select_exhaustive_noalloc(_ptr(keys), key_dtype, n, d, q.shape[1], _ptr(q), _ptr(w),
                                              pos0, q.shape[0], k, _ptr(out), _ptr(out_scores),
                                              _ptr(status), _stream(stream)))
+    return out
+
+
+def ai_route_refine_shard(h, q, w, pos0: int, k: int, C: int, shard: int, n_shards: int, out, out_scores):
+    _check(_lib.ai_route_refine_shard(h, _ptr(q), _ptr(w), pos0, q.shape[0], k, C, shard, n_shards,
+                                      _ptr(out), _ptr(out_scores)))
+    return out, out_scores
+
+
+def ai_merge_topk(ids, scores, k: int, out, out_scores=None, stream=None):
+    """ids / scores: [n_parts, T, k] device tensors."""
+    _check(_lib.ai_merge_topk(_ptr(ids), _ptr(scores), ids.shape[0], ids.shape[1], k, _ptr(out),
+                              _ptr(out_scores), _stream(stream)))
     return out
 
 

@@ -839,7 +839,7 @@ int ai_publish(ai_handle h) {
 
 static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t pos0, int T, int k,
                              int C, int32_t* out, float* out_scores, int32_t* cand_out,
-                             float* cluster_scores_out) {
+                             float* cluster_scores_out, int shard = 0, int n_shards = 1) {
   int rc = check_queries(h, q, w, pos0, T, k);
   if (rc) return rc;
   if (C <= 0 || C > h->cfg.max_budget) return fail(AI_ERR_ARG, "C out of range");
@@ -878,6 +878,8 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
   ra.cand_out = cand_out;
   ra.cand_scratch = h->cand_scratch;
   ra.refine_kernel = h->refine_kernel;
+  ra.shard = shard;
+  ra.n_shards = n_shards;
   ra.err = h->err_dev;
   int32_t* tmp_out = nullptr;
   if (!out) {  // debug call: outputs still need a home
@@ -924,6 +926,19 @@ int ai_route_refine(ai_handle h, const void* q_dev, const float* w_dev, int64_t 
                     int32_t k, int32_t C, int32_t* out_dev, float* out_scores_dev) {
   if (!h || !out_dev) return fail(AI_ERR_ARG, "null handle or output");
   return route_refine_impl(h, q_dev, w_dev, pos0, T, k, C, out_dev, out_scores_dev, nullptr, nullptr);
+}
+
+int ai_route_refine_shard(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0, int32_t T,
+                          int32_t k, int32_t C, int32_t shard, int32_t n_shards, int32_t* out_dev,
+                          float* out_scores_dev) {
+  if (!h || !out_dev || !out_scores_dev) return fail(AI_ERR_ARG, "null handle or output");
+  if (n_shards < 1 || shard < 0 || shard >= n_shards) return fail(AI_ERR_ARG, "bad shard");
+  if (n_shards > 1 && !tc_keys(h)) return fail(AI_ERR_ARG, "sharded rescore needs bf16 or fp8 keys");
+  if (n_shards > 1 && h->refine_kernel != REFINE_AUTO && h->refine_kernel != REFINE_PIPE &&
+      h->refine_kernel != REFINE_PIPE_1BUF)
+    return fail(AI_ERR_ARG, "sharded rescore runs on the pipelined refine kernels only");
+  return route_refine_impl(h, q_dev, w_dev, pos0, T, k, C, out_dev, out_scores_dev, nullptr, nullptr, shard,
+                           n_shards);
 }
 
 int ai_debug_candidates(ai_handle h, const void* q_dev, const float* w_dev, int64_t pos0, int32_t T,

@@ -67,6 +67,7 @@ struct RefineArgs {
   int32_t* cand_out;         // debug: [T, C] candidate lists or nullptr
   int32_t* cand_scratch;     // tensor-core path: candidate lists, [4 * num_sms, C]
   int refine_kernel;         // REFINE_* (tensor-core path; AUTO picks by occupancy)
+  int shard, n_shards;       // rescore only this shard's tile range of each list (n_shards <= 1: all)
   int* err;
 };
 enum RefineKernel {

@@ -12,6 +12,7 @@
 // position is its bin's start plus its rank among the bin's keys.  A bin
 // holding more than kMaxBin keys (near-equal scores) sends the row through a
 // bitonic sort instead.
+#include "../../include/ai_index.h"
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
@@ -150,7 +151,61 @@ __global__ void __launch_bounds__(kThreads) k_order_rows(OrderRowsArgs a) {
   }
 }
 
+// Merge of P partial top-k lists per row (the shards of a sharded rescore):
+// the valid (id >= 0) entries of the row's P lists are compacted into
+// shared memory, and the block selects their top k by (score desc, id asc),
+// written in that order and padded with -1.  The partial lists hold
+// disjoint ids, and each holds its shard's top k, so the union holds the
+// row's top k.
+__global__ void __launch_bounds__(1024) k_merge_rows(const int32_t* __restrict__ ids,
+                                                    const float* __restrict__ scores, int P, int T, int k,
+                                                    int32_t* out, float* out_scores) {
+  extern __shared__ __align__(16) uint8_t raw[];
+  int np = 1;
+  while (np < k) np <<= 1;
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(raw);        // output sort [np]
+  uint64_t* items = sbuf + np;                              // [P * k] valid entries
+  __shared__ BlockScratch bs;
+  __shared__ int s_n;
+  const int row = blockIdx.x, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) s_n = 0;
+  __syncthreads();
+  const int L = P * k;
+  const int Lr = (L + 31) & ~31;  // whole warps for the ballots
+  for (int e = threadIdx.x; e < Lr; e += blockDim.x) {
+    int32_t id = -1;
+    float v = 0.f;
+    if (e < L) {
+      const int p = e / k, j = e % k;
+      const int64_t o = (static_cast<int64_t>(p) * T + row) * k + j;
+      id = ids[o];
+      v = scores[o];
+    }
+    const bool ok = id >= 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, ok);
+    int base = 0;
+    if (bal) {
+      const int lead = __ffs(bal) - 1;
+      if (lane == lead) base = atomicAdd(&s_n, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, lead);
+    }
+    if (ok) items[base + __popc(bal & ((1u << lane) - 1u))] = order_key(v, id);
+  }
+  __syncthreads();
+  const int n = s_n;
+  topk_select_emit(
+      n, [&](int i) -> float { return order_key_score(items[i]); },
+      [&](int i) -> int32_t { return order_key_id(items[i]); }, k, out + static_cast<int64_t>(row) * k,
+      out_scores ? out_scores + static_cast<int64_t>(row) * k : nullptr, bs, sbuf);
+}
+
 }  // namespace
+
+size_t merge_smem_bytes(int P, int k) {
+  size_t np = 1;
+  while (np < static_cast<size_t>(k)) np <<= 1;
+  return (np + static_cast<size_t>(P) * k) * 8;
+}
 
 cudaError_t launch_order_rows(const OrderRowsArgs& a, cudaStream_t st) {
   if (a.T <= 0) return cudaSuccess;
@@ -161,3 +216,33 @@ cudaError_t launch_order_rows(const OrderRowsArgs& a, cudaStream_t st) {
 }
 
 }  // namespace aiidx
+
+// ------------------------------------------------------------------ C ABI
+extern "C" int ai_merge_topk(const int32_t* ids_dev, const float* scores_dev, int32_t n_parts, int32_t T,
+                             int32_t k, int32_t* out_dev, float* out_scores_dev, void* cuda_stream) {
+  using namespace aiidx;
+  if (!ids_dev || !scores_dev || !out_dev) {
+    set_last_error("null pointer argument");
+    return AI_ERR_ARG;
+  }
+  if (n_parts < 1 || T < 0 || k < 1 || k > kTcMaxK) {
+    set_last_error("n_parts >= 1, T >= 0 and 1 <= k <= 2048 required");
+    return AI_ERR_ARG;
+  }
+  const size_t smem = merge_smem_bytes(n_parts, k);
+  if (smem > 227 * 1024) {
+    set_last_error("n_parts * k too large for one block (n_parts * k + k <= 29000)");
+    return AI_ERR_ARG;
+  }
+  if (T == 0) return AI_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaFuncSetAttribute(k_merge_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  count_launch();
+  k_merge_rows<<<T, 1024, smem, st>>>(ids_dev, scores_dev, n_parts, T, k, out_dev, out_scores_dev);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error(cudaGetErrorString(e));
+    return AI_ERR_CUDA;
+  }
+  return AI_OK;
+}

@@ -75,6 +75,23 @@ __device__ __forceinline__ void bitonic_sort_u64(uint64_t* buf, int n, const G& 
   }
 }
 
+// The share of a candidate list of n slots that one shard rescores: the
+// whole list, or (n_shards > 1) a contiguous range of its 128-slot tiles.
+// The rescore and the top-k run on the list shifted to that range.
+__device__ __forceinline__ void shard_span(const RefineArgs& a, int n, int* off, int* n_loc) {
+  if (a.n_shards <= 1) {
+    *off = 0;
+    *n_loc = n;
+    return;
+  }
+  const int tiles = (n + kTile - 1) / kTile;
+  const int t0 = static_cast<int>(static_cast<int64_t>(a.shard) * tiles / a.n_shards);
+  const int t1 = static_cast<int>(static_cast<int64_t>(a.shard + 1) * tiles / a.n_shards);
+  const int e = n < t1 * kTile ? n : t1 * kTile;
+  *off = t0 * kTile;
+  *n_loc = e > t0 * kTile ? e - t0 * kTile : 0;
+}
+
 __device__ __forceinline__ void version_of(const VersionTable& vt, int64_t t, int* nC,
                                            int64_t* n_v) {
   int idx = 0;
@@ -1285,9 +1302,10 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       // orders the previous query's reads of wsh before its rewrite
       if (!named_bar_and(3, 128, ok)) break;
       tc_fence_after();
-      const int n = meta[b];
+      int off, n;
+      shard_span(a, meta[b], &off, &n);
       const int nt = (n + kTile - 1) / kTile;
-      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C;
+      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C + off;
       for (int h = row; h < H; h += 128) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
       named_bar(3, 128);
       const int sb = q % NSB;  // score buffer of this query
@@ -1365,7 +1383,9 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
         const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
         const int b = q & 1;
         if (!mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag)) break;
-        const int nt = (meta[b] + kTile - 1) / kTile;
+        int off, n_loc;
+        shard_span(a, meta[b], &off, &n_loc);
+        const int nt = (n_loc + kTile - 1) / kTile;
         mbar_arrive(&mread[b]);  // the slot's length is read; it may be rebuilt
         // the head tile is rewritten once the previous query's UMMAs are done
         if (q > 0 && !mbar_wait(qempty, (commits - 1) & 1, a.err, abort_flag)) break;
@@ -1415,9 +1435,10 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       const int b = q & 1;
       const bool ok = mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const int n = meta[b];
+      int off, n;
+      shard_span(a, meta[b], &off, &n);
       const int nt = (n + kTile - 1) / kTile;
-      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C;
+      const int32_t* cl = rows + static_cast<int64_t>(b) * a.C + off;
       int gid = next_gid(-1, gw, n, cl);
       bool good = true;
       for (int j = 0; j < nt; ++j) {
@@ -1484,9 +1505,10 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       P3Ctx c;
       c.row = quarter * 32 + lane;
       c.tcol = tmem_base + 2 * H + (q % NSB) * sc_cols + (static_cast<uint32_t>(quarter * 32) << 16);
-      c.n = meta[q & 1];
+      int off;
+      shard_span(a, meta[q & 1], &off, &c.n);
       c.ntiles = (c.n + kTile - 1) / kTile;
-      c.cand = rows + static_cast<int64_t>(q & 1) * a.C;
+      c.cand = rows + static_cast<int64_t>(q & 1) * a.C + off;
       p3_topk(a, qi, c, c.row, ps);  // c.row == et: rows in thread order
       tc_fence_before();
       mbar_arrive(&sfree[q % NSB]);
@@ -1551,6 +1573,7 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
                                                     : a.refine_kernel;
     if (kind < REFINE_SEQ_SMEM || kind > REFINE_PIPE_1BUF) return cudaErrorInvalidValue;
     const bool pipe = kind == REFINE_PIPE || kind == REFINE_PIPE_1BUF;
+    if (a.n_shards > 1 && !pipe) return cudaErrorInvalidValue;  // sharded rescore: pipelined kernels only
     if ((kind == REFINE_SEQ_GLOBAL || pipe) && !a.cand_scratch) return cudaErrorInvalidValue;
     const int tm = pipe ? pipe_tmem_cols(a.C, a.H, kind == REFINE_PIPE ? 2 : 1) : tc_tmem_cols(a.C, a.H);
     const size_t smem_tc = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
@@ -1578,6 +1601,7 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     }
 #undef AI_LAUNCH_REFINE
   } else {
+    if (a.n_shards > 1) return cudaErrorInvalidValue;
     // the output sort reuses the phase-1 region: room for kRowTopkMaxK keys
     if (a.k > kRowTopkMaxK || region_bytes(a.H, a.d, false) < static_cast<size_t>(kRowTopkMaxK) * 8)
       return cudaErrorInvalidValue;

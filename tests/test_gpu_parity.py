@@ -249,6 +249,46 @@ def test_recall_ablation_agrees_with_oracle(variant):
     gpu.close()
 
 
+@pytest.mark.parametrize("name,budget,kern", [("glm_bf16_L128k", 3000, 0), ("v4flash_fp8_L256k", 2500, 0),
+                                              ("v4flash_fp8_L256k", 2500, 4)])
+def test_sharded_rescore_and_merge_equal_route_refine(name, budget, kern):
+    """Cluster-sharded selection (review, Impact Assessment: Core
+    Contribution item 3): every shard rescores its range of each candidate
+    list, and merging the shards' top k (ai_merge_topk) gives exactly the
+    single-call result, ids and scores bit for bit, for 1 to 4 shards.  The
+    shards run one after another here (one GPU); on several GPUs an
+    all-gather moves the partial results (sharded.exchange_and_merge, tested
+    with gloo ranks on CPU)."""
+    from ivf_top_key_b200 import merge_topk
+    wl = S.scaled(S.WORKLOADS[name], L=12288, T=2048, refit_period=4096, budget=budget, k=200, M=256)
+    gpu, _ = P.make_pair(wl)
+    if kern:
+        gpu.debug_refine_kernel(kern)
+    for c in range(wl.n_chunks):
+        kd, ks, _ = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+    p0 = wl.L - wl.T
+    qd, wd, _, _ = P.query_inputs(wl, p0, wl.L)
+    ref = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    ref_sc = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    gpu.route_refine(qd, wd, p0, wl.k, wl.budget, out=ref, out_scores=ref_sc)
+    for n in (1, 2, 3, 4):
+        parts = [gpu.route_refine_shard(qd, wd, p0, wl.k, wl.budget, r, n) for r in range(n)]
+        ids = torch.stack([p_[0] for p_ in parts])
+        sc = torch.stack([p_[1] for p_ in parts])
+        out = torch.full((wl.T, wl.k), -7, dtype=torch.int32, device="cuda")
+        out_sc = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
+        merge_topk(ids, sc, wl.k, out=out, out_scores=out_sc)
+        gpu.sync()
+        assert torch.equal(out, ref), n
+        assert torch.equal(out_sc.view(torch.int32), ref_sc.view(torch.int32)), n
+        if n > 1:  # every shard did part of the work: disjoint, non-empty shares
+            got = [set(p_[0][p_[0] >= 0].cpu().numpy().ravel().tolist()) for p_ in parts]
+            assert all(len(g) > 0 for g in got)
+    gpu.close()
+
+
 def test_synchronous_refit_matches_oracle():
     wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=10240, T=2048, refit_period=4096,
                   budget=2048, k=128, M=128)
