@@ -213,6 +213,9 @@ struct ai_index {
   int64_t max_seeds = 0;
   // route / exhaustive scratch
   float* route = nullptr;          // [max_query_chunk, maxC_pad]
+  uint32_t* route_kmin = nullptr;  // [max_query_chunk] per-query route score range (tensor-core route)
+  uint32_t* route_kmax = nullptr;
+  bool route_range = false;        // the last route call filled route_kmin / route_kmax
   float* exh = nullptr;            // [exh_rows, exh_ld]
   int64_t exh_rows = 0, exh_ld = 0;
   int* err_dev = nullptr;
@@ -288,10 +291,18 @@ int route_scores(ai_index* h, const void* q, const float* w, int T, int64_t nC) 
     if (!make_map(&ma, b.reps, nC, 128) || !make_map(&mb, q, static_cast<int64_t>(T) * h->cfg.H, 256))
       return fail(AI_ERR_CUDA, "tensor map encoding failed (route)");
     const int apc = scores_tiles_per_item(nC, T, h->cfg.H, h->num_sms);
+    // per-query score range, collected by the GEMM's epilogue (the candidate
+    // build bins the scores over it)
+    sa.row_kmin = h->route_kmin;
+    sa.row_kmax = h->route_kmax;
     const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
+    CK(cudaMemsetAsync(h->route_kmin, 0xff, static_cast<size_t>(T) * 4, h->main));
+    CK(cudaMemsetAsync(h->route_kmax, 0, static_cast<size_t>(T) * 4, h->main));
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
     prof_end(h, pi, h->main);
+    h->route_range = true;
   } else {
+    h->route_range = false;
     const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
     CK(launch_scores_simt(b.reps, KD_BF16, q, h->cfg.q_dtype == AI_BF16, h->cfg.d, h->cfg.H, sa, h->main));
     prof_end(h, pi, h->main);
@@ -683,6 +694,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   // one candidate row per refine CTA (at most 4 per SM)
   if (tck) CKC(dalloc(&h->cand_scratch, static_cast<size_t>(h->num_sms) * 4 * c.max_budget));
   if (tck) CKC(dalloc(&h->topk_scores, static_cast<size_t>(c.max_query_chunk) * c.max_k));
+  if (tcr) CKC(dalloc(&h->route_kmin, static_cast<size_t>(c.max_query_chunk)));
+  if (tcr) CKC(dalloc(&h->route_kmax, static_cast<size_t>(c.max_query_chunk)));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
   CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
   if ((c.key_dtype == AI_BF16 || c.key_dtype == AI_FP8E4M3) && d == 128 && c.refit_period > 0) {
@@ -738,6 +751,8 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->cent_cc);
   cudaFree(h->cand_scratch);
   cudaFree(h->topk_scores);
+  cudaFree(h->route_kmin);
+  cudaFree(h->route_kmax);
   cudaFree(h->upd_chunk_off);
   cudaFree(h->upd_part);
   cudaFree(h->band_best);
@@ -864,6 +879,8 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
   ra.w = w;
   ra.route = h->route;
   ra.ld_route = h->maxC_pad;
+  ra.route_kmin = nC > 0 && h->route_range ? h->route_kmin : nullptr;
+  ra.route_kmax = nC > 0 && h->route_range ? h->route_kmax : nullptr;
   ra.offsets = b.offsets;
   ra.members = b.members;
   ra.pos0 = pos0;

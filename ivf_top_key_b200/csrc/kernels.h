@@ -20,6 +20,8 @@ struct ScoreArgs {
   const float* w;          // [T, H] head weights
   const float* row_scale;  // [nA] per-row positive scale or nullptr
   float* out;              // out[q * ld_out + a]
+  uint32_t* row_kmin;      // per query: min / max over a of f2key(out[q][a]) (atomic;
+  uint32_t* row_kmax;      //   pre-set to 0xffffffff / 0), or nullptr
   int64_t ld_out;
   int a_tiles_per_cta;      // A tiles per work item (tensor-core path)
   int causal;              // mask a_pos0 + a > q_pos0 + q to -inf
@@ -57,6 +59,8 @@ struct RefineArgs {
   int q_is_bf16;
   const float* w;            // [T, H]
   const float* route;        // [T, ld_route] cluster scores
+  const uint32_t* route_kmin;  // per query: order-preserving keys of the min / max route score
+  const uint32_t* route_kmax;  //   over all clusters, or nullptr (then computed by the kernel)
   int64_t ld_route;
   const int32_t* offsets;    // CSR offsets [nC + 1]
   const int32_t* members;    // CSR members

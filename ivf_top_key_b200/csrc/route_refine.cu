@@ -111,6 +111,7 @@ __device__ __forceinline__ void version_of(const VersionTable& vt, int64_t t, in
 // crosses the remaining budget; clusters in that bin or above are sorted
 // exactly and the fill stops at C.
 constexpr int kNB1 = 2048;
+constexpr int kLightBin = 512;  // members in a boundary bin taken whole (no level-2 pass)
 struct P1Smem {
   union {                    // the histogram is dead before the offsets are written
     int32_t coff[kSortCap];  // member offset of each ranked cluster
@@ -186,38 +187,49 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
       (reinterpret_cast<uintptr_t>(pref + kSortCap + 1) + 15) & ~uintptr_t(15));
   const float* rs = a.route + static_cast<int64_t>(qi) * a.ld_route;
   const int32_t* off = a.offsets;
-  // pass A: score range and total size of the non-empty clusters
   float vmin = INFINITY, vmax = -INFINITY;
   unsigned long long wsum = 0;
+  if (a.route_kmin) {
+    // score range from the route GEMM (over all clusters of the buffer: a
+    // superset of this query's visible ones, which only widens the bins)
+    // and the total size of the visible clusters (telescoping offsets)
+    vmin = key2f(__ldg(a.route_kmin + qi));
+    vmax = key2f(__ldg(a.route_kmax + qi));
+    wsum = static_cast<unsigned long long>(__ldg(off + nC) - __ldg(off));
+    for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
+    g.sync();
+  } else {
+    // pass A: score range and total size of the non-empty clusters
 #pragma unroll 4
-  for (int c = tid; c < nC; c += nthr) {
-    const int sz = __ldg(off + c + 1) - __ldg(off + c);
-    const float v = __ldg(rs + c);
-    if (sz > 0) {
-      vmin = fminf(vmin, v);
-      vmax = fmaxf(vmax, v);
-      wsum += static_cast<unsigned long long>(sz);
+    for (int c = tid; c < nC; c += nthr) {
+      const int sz = __ldg(off + c + 1) - __ldg(off + c);
+      const float v = __ldg(rs + c);
+      if (sz > 0) {
+        vmin = fminf(vmin, v);
+        vmax = fmaxf(vmax, v);
+        wsum += static_cast<unsigned long long>(sz);
+      }
     }
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  }
-  if (lane == 0) {
-    ps.fred[warp] = vmin;
-    ps.fred[16 + warp] = vmax;
-    ps.wred[warp] = wsum;
-  }
-  for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
-  g.sync();
-  vmin = INFINITY;
-  vmax = -INFINITY;
-  wsum = 0;
-  for (int w = 0; w < nwarps; ++w) {
-    vmin = fminf(vmin, ps.fred[w]);
-    vmax = fmaxf(vmax, ps.fred[16 + w]);
-    wsum += ps.wred[w];
+    for (int o = 16; o > 0; o >>= 1) {
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    }
+    if (lane == 0) {
+      ps.fred[warp] = vmin;
+      ps.fred[16 + warp] = vmax;
+      ps.wred[warp] = wsum;
+    }
+    for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
+    g.sync();
+    vmin = INFINITY;
+    vmax = -INFINITY;
+    wsum = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      vmin = fminf(vmin, ps.fred[w]);
+      vmax = fmaxf(vmax, ps.fred[16 + w]);
+      wsum += ps.wred[w];
+    }
   }
   const bool take_all = wsum <= static_cast<unsigned long long>(rem);
   const float scale = vmax > vmin ? static_cast<float>(kNB1) / (vmax - vmin) : 0.f;
@@ -254,7 +266,12 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     int above1 = 0;
     p1_find_bin(ps, rem, &bstar, &above1, g);
     // pass B2: the boundary bin split into kNB1 sub-bins (a long score tail
-    // leaves most clusters in few level-1 bins)
+    // leaves most clusters in few level-1 bins).  A light boundary bin (few
+    // members, hence few clusters) is instead taken whole: the exact sort
+    // below ranks its clusters.
+    const bool light = ps.hist[bstar] <= static_cast<uint32_t>(kLightBin);
+    g.sync();
+    if (!light) {
     for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
     g.sync();
     for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
@@ -273,6 +290,7 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     g.sync();
     int above2 = 0;
     p1_find_bin(ps, rem - above1, &bstar2, &above2, g);
+    }  // !light (else bstar2 = 0: every cluster of the boundary bin)
   }
   auto selected = [=](float v) -> bool {
     if (take_all) return true;

@@ -254,6 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the weights land with the query tile
       if (!mbar_wait(&bfull[b], (k >> 1) & 1, args.err, sm.abort)) break;
       const float* wk = sm.w + b * kBN + qh * QPW * H;
+      uint32_t kmn[QPW], kmx[QPW];
+#pragma unroll
+      for (int qi = 0; qi < QPW; ++qi) {
+        kmn[qi] = 0xffffffffu;
+        kmx[qi] = 0u;
+      }
       for (int jj = 0; jj < te - tb; ++jj, ++g) {
         const int i = rotated_tile(tb, te, jj);
         const int acc = g & 1;
@@ -292,8 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
         const int a = i * kBM + row_in_tile;
+        const float sc = a < args.nA && args.row_scale ? args.row_scale[a] : 1.f;
         if (a < args.nA) {
-          const float sc = args.row_scale ? args.row_scale[a] : 1.f;
 #pragma unroll
           for (int qi = 0; qi < QPW; ++qi) {
             const int q = q0 + qh * QPW + qi;
@@ -304,8 +310,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        // running per-query score range (order-preserving keys) over the
+        // item's rows; reduced once at the end of the item
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const uint32_t key = f2key(res[qi] * sc);
+          const bool ok = a < args.nA;
+          kmn[qi] = ok && key < kmn[qi] ? key : kmn[qi];
+          kmx[qi] = ok && key > kmx[qi] ? key : kmx[qi];
+        }
       }
       mbar_arrive(&bempty[b]);  // done with this item's weights
+      // (after an aborted wait the warp skips the range: the call reports
+      // the timeout and its outputs are not used)
+      if (__all_sync(0xffffffffu, ok) && args.row_kmin) {
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const int q = q0 + qh * QPW + qi;
+          const uint32_t mn = __reduce_min_sync(0xffffffffu, kmn[qi]);
+          const uint32_t mx = __reduce_max_sync(0xffffffffu, kmx[qi]);
+          if (lane == 0 && q < args.T) {
+            atomicMin(args.row_kmin + q, mn);
+            atomicMax(args.row_kmax + q, mx);
+          }
+        }
+      }
       ++k;
     }
   }
