@@ -162,6 +162,43 @@ __device__ __forceinline__ void p1_find_bin(P1Smem& ps, int need, int* bstar, in
   g.sync();
 }
 
+// f(c, score, size) for every cluster c < nC: blocks of four clusters with
+// 16-byte loads of their offsets and route scores (both arrays 16-byte
+// aligned), two blocks in flight per thread, then the ragged tail.
+template <class F>
+__device__ __forceinline__ void for_clusters(const int32_t* off, const float* rs, int nC, int tid, int nthr,
+                                             F f) {
+  const int nb = nC >> 2;
+  for (int i0 = tid; i0 < nb; i0 += 2 * nthr) {
+    int4 o[2];
+    int o4[2];
+    float4 v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * nthr;
+      o[u] = make_int4(0, 0, 0, 0);
+      o4[u] = 0;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < nb) {
+        o[u] = __ldg(reinterpret_cast<const int4*>(off) + i);
+        o4[u] = __ldg(off + 4 * i + 4);
+        v[u] = __ldg(reinterpret_cast<const float4*>(rs) + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * nthr;
+      if (i < nb) {
+        f(4 * i, v[u].x, o[u].y - o[u].x);
+        f(4 * i + 1, v[u].y, o[u].z - o[u].y);
+        f(4 * i + 2, v[u].z, o[u].w - o[u].z);
+        f(4 * i + 3, v[u].w, o4[u] - o[u].w);
+      }
+    }
+  }
+  for (int c = 4 * nb + tid; c < nC; c += nthr) f(c, __ldg(rs + c), __ldg(off + c + 1) - __ldg(off + c));
+}
+
 // The list is written to shared memory (kGlobal = false) or to the CTA's
 // global scratch row (kGlobal = true).
 template <bool kGlobal, class G>
@@ -249,19 +286,9 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   if (!take_all) {
     // pass B: size-weighted histogram; the bin where the weight from the top
     // reaches the remaining budget
-    for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
-      float v[4];
-      int sz[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * nthr;
-        sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
-        v[u] = c < nC ? __ldg(rs + c) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (sz[u] > 0) atomicAdd(&ps.hist[binof(v[u])], static_cast<uint32_t>(sz[u]));
-    }
+    for_clusters(off, rs, nC, tid, nthr, [&](int, float v, int sz) {
+      if (sz > 0) atomicAdd(&ps.hist[binof(v)], static_cast<uint32_t>(sz));
+    });
     g.sync();
     int above1 = 0;
     p1_find_bin(ps, rem, &bstar, &above1, g);
@@ -274,19 +301,9 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     if (!light) {
     for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
     g.sync();
-    for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
-      float v[4];
-      int sz[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * nthr;
-        sz[u] = c < nC ? __ldg(off + c + 1) - __ldg(off + c) : 0;
-        v[u] = c < nC ? __ldg(rs + c) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (sz[u] > 0 && binof(v[u]) == bstar) atomicAdd(&ps.hist[bin2(v[u], bstar)], static_cast<uint32_t>(sz[u]));
-    }
+    for_clusters(off, rs, nC, tid, nthr, [&](int, float v, int sz) {
+      if (sz > 0 && binof(v) == bstar) atomicAdd(&ps.hist[bin2(v, bstar)], static_cast<uint32_t>(sz));
+    });
     g.sync();
     int above2 = 0;
     p1_find_bin(ps, rem - above1, &bstar2, &above2, g);
@@ -301,25 +318,12 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   // pass C: clusters at or above the boundary bin (any order: sorted next)
   if (tid == 0) ps.scal[1] = 0;
   g.sync();
-  for (int c0 = tid; c0 < nC; c0 += 4 * nthr) {
-    float v[4];
-    int sz[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * nthr;
-      sz[u] = c < nC ? off[c + 1] - off[c] : 0;
-      v[u] = c < nC ? rs[c] : 0.f;
+  for_clusters(off, rs, nC, tid, nthr, [&](int c, float v, int sz) {
+    if (sz > 0 && selected(v)) {
+      const int pos = atomicAdd(&ps.scal[1], 1);
+      if (pos < kSortCap) sortbuf[pos] = (static_cast<uint64_t>(~f2key(v)) << 32) | static_cast<uint32_t>(c);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * nthr;
-      if (sz[u] > 0 && selected(v[u])) {
-        const int pos = atomicAdd(&ps.scal[1], 1);
-        if (pos < kSortCap)
-          sortbuf[pos] = (static_cast<uint64_t>(~f2key(v[u])) << 32) | static_cast<uint32_t>(c);
-      }
-    }
-  }
+  });
   g.sync();
   int nsel = ps.scal[1];
   if (nsel > kSortCap) {
