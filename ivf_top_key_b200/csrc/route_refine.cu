@@ -382,7 +382,7 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
   if (kGlobal) {
     // fill of a list in global memory: one warp per ranked cluster, four
     // clusters per warp at a time (their run bounds are independent shared
-    // loads, their first 64 members eight coalesced loads per lane in
+    // loads, their first 128 members sixteen coalesced loads per lane in
     // flight), cut at C
     for (int r0 = warp; r0 < nsel; r0 += 4 * nwarps) {
       int d0[4], sz[4], src[4];
@@ -398,24 +398,40 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
           src[u] = coff[r];
         }
       }
-      int32_t v[4][2];
+      // the first 128 members of the four clusters: 16 loads in flight per
+      // lane (clusters hold ~W/m = 128 keys after a seal)
+      int32_t v[4][4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
           const int l = lane + 32 * h;
           v[u][h] = l < sz[u] ? __ldg(a.members + src[u] + l) : 0;
         }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
           const int l = lane + 32 * h;
           if (l < sz[u]) cand[d0[u] + l] = v[u][h];
         }
+      // larger (refit) clusters: the rest, four loads in flight per lane
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        for (int l = 64 + lane; l < sz[u]; l += 32) cand[d0[u] + l] = __ldg(a.members + src[u] + l);
+      for (int u = 0; u < 4; ++u) {
+        for (int l0 = 128; l0 < sz[u]; l0 += 128) {
+          int32_t w4[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int l = l0 + lane + 32 * h;
+            w4[h] = l < sz[u] ? __ldg(a.members + src[u] + l) : 0;
+          }
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int l = l0 + lane + 32 * h;
+            if (l < sz[u]) cand[d0[u] + l] = w4[h];
+          }
+        }
+      }
     }
   } else {
     // fill of a list in shared memory: one warp per ranked cluster copies
@@ -553,7 +569,7 @@ struct P3Smem {
   float fred[8];
   int ired[8];
   int scal[8];
-  unsigned long long cnt;
+  int cnt32;   // items of the threshold bin appended so far
 };
 
 struct P3Ctx {
@@ -724,7 +740,7 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
     // the k-th score into kNB sub-bins (a long score tail leaves the bulk
     // in few level-1 bins)
     for (int i = et; i < kNB; i += 128) ps.hist[i] = 0;
-    if (et == 0) ps.cnt = 0;
+    if (et == 0) ps.cnt32 = 0;
     named_bar(1, 128);
     // (an add of 0 for slots past the list keeps the body branch-free)
     p3_for_each_all(c, [&ps, binof](float v, int, int ok) {
@@ -780,21 +796,26 @@ __device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3S
           m |= static_cast<uint32_t>(f) << u;
         }
         if (__any_sync(0xffffffffu, m != 0u)) {
+          // one scan of the per-thread hit counts and one counter update per
+          // warp; each thread then writes its hits with predicated stores
           const int lane = threadIdx.x & 31;
+          const int h = __popc(m);
+          int incl = h;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t2;
+          }
+          int base = 0;
+          if (lane == 31) base = atomicAdd(&ps.cnt32, incl);
+          int pos = __shfl_sync(0xffffffffu, base, 31) + incl - h;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            const int f = static_cast<int>((m >> u) & 1u);
-            const unsigned bal = __ballot_sync(0xffffffffu, f);
-            if (bal) {
-              const int lead = __ffs(bal) - 1;
-              unsigned long long base = 0;
-              if (lane == lead) base = atomicAdd(&ps.cnt, static_cast<unsigned long long>(__popc(bal)));
-              base = __shfl_sync(0xffffffffu, base, lead);
-              if (f)
-                ps.buf[base + __popc(bal & ((1u << lane) - 1u))] =
-                    (static_cast<uint64_t>(~f2key(v[u])) << 32) |
-                    static_cast<uint32_t>((c0 + u) * 128 + c.row);
-            }
+            const bool f = (m >> u) & 1u;
+            if (f)
+              ps.buf[pos] = (static_cast<uint64_t>(~f2key(v[u])) << 32) |
+                            static_cast<uint32_t>((c0 + u) * 128 + c.row);
+            pos += f ? 1 : 0;
           }
         }
       }
