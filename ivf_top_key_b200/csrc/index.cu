@@ -213,7 +213,7 @@ struct ai_index {
   int64_t max_seeds = 0;
   // route / exhaustive scratch
   float* route = nullptr;          // [max_query_chunk, maxC_pad]
-  uint32_t* route_kmin = nullptr;  // [max_query_chunk] per-query route score range (tensor-core route)
+  uint32_t* route_kmin = nullptr;  // [max_query_chunk, 4] route score range partials (tensor-core route)
   uint32_t* route_kmax = nullptr;
   bool route_range = false;        // the last route call filled route_kmin / route_kmax
   float* exh = nullptr;            // [exh_rows, exh_ld]
@@ -296,8 +296,10 @@ int route_scores(ai_index* h, const void* q, const float* w, int T, int64_t nC) 
     sa.row_kmin = h->route_kmin;
     sa.row_kmax = h->route_kmax;
     const int pi = prof_begin(h, AI_PHASE_ROUTE, h->main);
-    CK(cudaMemsetAsync(h->route_kmin, 0xff, static_cast<size_t>(T) * 4, h->main));
-    CK(cudaMemsetAsync(h->route_kmax, 0, static_cast<size_t>(T) * 4, h->main));
+    if (apc < (nC + 127) / 128) {  // several items per query: atomic slots, pre-set
+      CK(cudaMemsetAsync(h->route_kmin, 0xff, static_cast<size_t>(T) * 16, h->main));
+      CK(cudaMemsetAsync(h->route_kmax, 0, static_cast<size_t>(T) * 16, h->main));
+    }
     CK(launch_scores_tc(ma, mb, h->cfg.H, sa, static_cast<int>(apc), h->main));
     prof_end(h, pi, h->main);
     h->route_range = true;
@@ -694,8 +696,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   // one candidate row per refine CTA (at most 4 per SM)
   if (tck) CKC(dalloc(&h->cand_scratch, static_cast<size_t>(h->num_sms) * 4 * c.max_budget));
   if (tck) CKC(dalloc(&h->topk_scores, static_cast<size_t>(c.max_query_chunk) * c.max_k));
-  if (tcr) CKC(dalloc(&h->route_kmin, static_cast<size_t>(c.max_query_chunk)));
-  if (tcr) CKC(dalloc(&h->route_kmax, static_cast<size_t>(c.max_query_chunk)));
+  if (tcr) CKC(dalloc(&h->route_kmin, static_cast<size_t>(c.max_query_chunk) * 4));
+  if (tcr) CKC(dalloc(&h->route_kmax, static_cast<size_t>(c.max_query_chunk) * 4));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
   CKC(dalloc(&h->upd_part, static_cast<size_t>(N / refit_update_chunk() + h->maxC + 1) * d));
   if ((c.key_dtype == AI_BF16 || c.key_dtype == AI_FP8E4M3) && d == 128 && c.refit_period > 0) {

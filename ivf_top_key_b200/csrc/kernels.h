@@ -20,8 +20,11 @@ struct ScoreArgs {
   const float* w;          // [T, H] head weights
   const float* row_scale;  // [nA] per-row positive scale or nullptr
   float* out;              // out[q * ld_out + a]
-  uint32_t* row_kmin;      // per query: min / max over a of f2key(out[q][a]) (atomic;
-  uint32_t* row_kmax;      //   pre-set to 0xffffffff / 0), or nullptr
+  uint32_t* row_kmin;      // [T, 4] per query and TMEM lane quarter: min / max of
+  uint32_t* row_kmax;      //   f2key(out[q][a]) over the quarter's rows, or nullptr;
+                           //   stored directly when one work item covers every A tile
+                           //   (a_tiles_per_cta >= A tiles), else atomic (pre-set to
+                           //   0xffffffff / 0)
   int64_t ld_out;
   int a_tiles_per_cta;      // A tiles per work item (tensor-core path)
   int causal;              // mask a_pos0 + a > q_pos0 + q to -inf
@@ -59,8 +62,8 @@ struct RefineArgs {
   int q_is_bf16;
   const float* w;            // [T, H]
   const float* route;        // [T, ld_route] cluster scores
-  const uint32_t* route_kmin;  // per query: order-preserving keys of the min / max route score
-  const uint32_t* route_kmax;  //   over all clusters, or nullptr (then computed by the kernel)
+  const uint32_t* route_kmin;  // [T, 4] partial order-preserving keys of the min / max route
+  const uint32_t* route_kmax;  //   score over all clusters, or nullptr (then computed here)
   int64_t ld_route;
   const int32_t* offsets;    // CSR offsets [nC + 1]
   const int32_t* members;    // CSR members

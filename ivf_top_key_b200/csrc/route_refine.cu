@@ -230,8 +230,10 @@ __device__ int build_candidates(const RefineArgs& a, int qi, int64_t t, int nC, 
     // score range from the route GEMM (over all clusters of the buffer: a
     // superset of this query's visible ones, which only widens the bins)
     // and the total size of the visible clusters (telescoping offsets)
-    vmin = key2f(__ldg(a.route_kmin + qi));
-    vmax = key2f(__ldg(a.route_kmax + qi));
+    const uint4 mn4 = __ldg(reinterpret_cast<const uint4*>(a.route_kmin) + qi);
+    const uint4 mx4 = __ldg(reinterpret_cast<const uint4*>(a.route_kmax) + qi);
+    vmin = key2f(min(min(mn4.x, mn4.y), min(mn4.z, mn4.w)));
+    vmax = key2f(max(max(mx4.x, mx4.y), max(mx4.z, mx4.w)));
     wsum = static_cast<unsigned long long>(__ldg(off + nC) - __ldg(off));
     for (int i = tid; i < kNB1; i += nthr) ps.hist[i] = 0;
     g.sync();

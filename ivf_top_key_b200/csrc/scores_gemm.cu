@@ -329,9 +329,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int q = q0 + qh * QPW + qi;
           const uint32_t mn = __reduce_min_sync(0xffffffffu, kmn[qi]);
           const uint32_t mx = __reduce_max_sync(0xffffffffu, kmx[qi]);
+          // one slot per (query, lane quarter): a plain store when this item
+          // is the query's only one, else an atomic into a pre-set slot
           if (lane == 0 && q < args.T) {
-            atomicMin(args.row_kmin + q, mn);
-            atomicMax(args.row_kmax + q, mx);
+            uint32_t* pmn = args.row_kmin + static_cast<int64_t>(q) * 4 + quarter;
+            uint32_t* pmx = args.row_kmax + static_cast<int64_t>(q) * 4 + quarter;
+            if (im.apc >= im.n_atiles) {
+              *pmn = mn;
+              *pmx = mx;
+            } else {
+              atomicMin(pmn, mn);
+              atomicMax(pmx, mx);
+            }
           }
         }
       }
