@@ -12,7 +12,9 @@
 //   h      = ReLU(B1 f + b1);   t = tanh(B2 h + b2)
 //   corr   = t * min(1, 0.25 ||mu|| / ||t||)  (0 if t = 0)
 //   rep    = bf16(mu + corr)
-// One CTA of d threads per cluster; thread o owns output feature o.
+// One CTA of d threads per cluster; thread o owns output feature o.  The
+// per-key transform phi is computed once per key when it is appended
+// (k_phi) and pooled from that cache at every seal and refit.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -52,9 +54,28 @@ __global__ void __launch_bounds__(kEncThreads) k_encoder(EncoderArgs a) {
     if (act) a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu);
     return;
   }
+  double psum = 0.0, pmax = 0.0;  // phi >= 0, so 0 starts the max
+  if (a.phi) {
+    // phi of every key was computed when it arrived (launch_phi, same
+    // arithmetic): pool the members' rows in member order
+    if (act) {
+      for (int p0 = o0; p0 < o1; p0 += kBatch) {
+        double ph[kBatch];
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r)
+          ph[r] = p0 + r < o1 ? a.phi[static_cast<int64_t>(a.members[p0 + r]) * d + o] : 0.0;
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {
+          if (p0 + r < o1) {
+            psum += ph[r];
+            pmax = ph[r] > pmax ? ph[r] : pmax;
+          }
+        }
+      }
+    }
+  } else {
   for (int e = o; e < d * d; e += blockDim.x) As[(e / d) * (d + 1) + (e % d)] = A[e];
   const double ao = act ? static_cast<double>(av[o]) : 0.0;
-  double psum = 0.0, pmax = 0.0;  // phi >= 0, so 0 starts the max
   for (int p0 = o0; p0 < o1; p0 += kBatch) {
     const int nb = min(kBatch, o1 - p0);
     __syncthreads();
@@ -82,6 +103,7 @@ __global__ void __launch_bounds__(kEncThreads) k_encoder(EncoderArgs a) {
       }
     }
   }
+  }  // phi computed here
   __syncthreads();
   if (act) {
     f[o] = psum / static_cast<double>(n);
@@ -136,14 +158,71 @@ __global__ void __launch_bounds__(kEncThreads) k_encoder(EncoderArgs a) {
   if (act) a.reps[static_cast<int64_t>(c) * d + o] = f64_to_bf16_rne(mu + corr);
 }
 
+// phi(k) = ReLU(A k + a) for 64 keys per CTA (thread o = output feature),
+// 8 at a time, with exactly the arithmetic of k_encoder's own loop (same
+// float64 FMA order), so cached and recomputed values are identical.
+constexpr int kPhiKeys = 64;
+__global__ void __launch_bounds__(kEncThreads) k_phi(const void* keys, const float* key_scale, int key_dtype,
+                                                     int d, const float* wts, int64_t s0, int64_t s1,
+                                                     double* phi) {
+  extern __shared__ double sh[];
+  double* keyb = sh;                                        // [kBatch][d]
+  float* As = reinterpret_cast<float*>(keyb + kBatch * d);  // [d][d + 1]
+  const int o = threadIdx.x;
+  const bool act = o < d;
+  const int64_t b0 = s0 + static_cast<int64_t>(blockIdx.x) * kPhiKeys;
+  const int64_t b1 = b0 + kPhiKeys < s1 ? b0 + kPhiKeys : s1;
+  for (int e = o; e < d * d; e += blockDim.x) As[(e / d) * (d + 1) + (e % d)] = wts[e];
+  const double ao = act ? static_cast<double>(wts[d * d + o]) : 0.0;
+  for (int64_t p0 = b0; p0 < b1; p0 += kBatch) {
+    const int nb = static_cast<int>(b1 - p0 < kBatch ? b1 - p0 : kBatch);
+    __syncthreads();
+    for (int e = o; e < nb * d; e += blockDim.x) {
+      const int r = e / d, i = e % d;
+      const int64_t s = p0 + r;
+      double v = key_elem(keys, key_dtype, s, d, i);
+      if (key_dtype == KD_FP8) v *= static_cast<double>(key_scale[s]);
+      keyb[r * d + i] = v;
+    }
+    __syncthreads();
+    if (act) {
+      double z[kBatch];
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) z[r] = ao;
+      for (int i = 0; i < d; ++i) {
+        const double w = static_cast<double>(As[o * (d + 1) + i]);
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) z[r] = fma(w, keyb[r * d + i], z[r]);
+      }
+      for (int r = 0; r < nb; ++r) phi[(p0 + r) * d + o] = z[r] > 0.0 ? z[r] : 0.0;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_phi(const void* keys, const float* key_scale, int key_dtype, int d, const float* wts,
+                       int64_t s0, int64_t s1, double* phi, cudaStream_t st) {
+  if (s1 <= s0) return cudaSuccess;
+  if (d > kEncThreads) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(kBatch) * d * 8 + static_cast<size_t>(d) * (d + 1) * 4;
+  const cudaError_t e = cudaFuncSetAttribute(k_phi, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (s1 - s0 + kPhiKeys - 1) / kPhiKeys;
+  count_launch();
+  k_phi<<<static_cast<unsigned>(blocks), kEncThreads, smem, st>>>(keys, key_scale, key_dtype, d, wts, s0, s1, phi);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_encoder(const EncoderArgs& a, cudaStream_t st) {
   const int n = a.cl_end - a.cl_begin;
   if (n <= 0) return cudaSuccess;
   if (a.d > kEncThreads) return cudaErrorInvalidValue;
+  // with cached phi the weight staging is not needed: a smaller footprint
+  // lets the encoder share SMs with other kernels
   const size_t smem = static_cast<size_t>(kBatch * a.d + 3 * a.d + 1 + a.d + 8) * 8 +
-                      static_cast<size_t>(a.d) * (a.d + 1) * 4;
+                      (a.phi ? 0 : static_cast<size_t>(a.d) * (a.d + 1) * 4);
   const cudaError_t e = cudaFuncSetAttribute(k_encoder, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
   if (e != cudaSuccess) return e;

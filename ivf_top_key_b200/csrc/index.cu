@@ -221,6 +221,7 @@ struct ai_index {
   int* err_dev = nullptr;
   int* err_host = nullptr;         // pinned
   float* enc_wts = nullptr;
+  double* phi = nullptr;           // [max_keys, d] encoder transform per key (encoder only)
   // phase timing (CUDA events on the launching stream)
   bool prof = false;
   std::vector<ProfRec> recs;
@@ -484,6 +485,7 @@ int start_refit(ai_index* h, int64_t n_seed, int64_t seed_window, int64_t window
     ea.cl_begin = 0;
     ea.cl_end = static_cast<int>(K);
     ea.wts = h->enc_wts;
+    ea.phi = h->phi;
     ea.reps = B.reps;
     ea.err = h->err_dev;
     CK(launch_encoder(ea, st));
@@ -536,6 +538,7 @@ int seal_group(ai_index* h, int64_t w0, int64_t nw) {
     ea.cl_begin = static_cast<int>(A.nC);
     ea.cl_end = static_cast<int>(A.nC + nw * m);
     ea.wts = h->enc_wts;
+    ea.phi = h->phi;
     ea.reps = A.reps;
     ea.err = h->err_dev;
     CK(launch_encoder(ea, h->main));
@@ -722,6 +725,7 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
                       static_cast<size_t>(d) * d + d;
     CKC(dalloc(&h->enc_wts, nw));
     CKC(cudaMemcpy(h->enc_wts, c.encoder_weights_host, nw * sizeof(float), cudaMemcpyHostToDevice));
+    CKC(dalloc(&h->phi, static_cast<size_t>(c.max_keys) * c.d));
     h->cfg.encoder_weights_host = nullptr;
   }
   CKC(cudaDeviceSynchronize());
@@ -774,6 +778,7 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->err_dev);
   if (h->err_host) cudaFreeHost(h->err_host);
   cudaFree(h->enc_wts);
+  cudaFree(h->phi);
   cudaFree(h->ck_assign);
   cudaFree(h->ck_ub);
   cudaFree(h->ck_lb);
@@ -802,6 +807,10 @@ int ai_append_keys(ai_handle h, const void* keys_dev, const float* scales_dev, i
                      cudaMemcpyDeviceToDevice, h->main));
   if (h->cfg.key_dtype == AI_FP8E4M3)
     CK(cudaMemcpyAsync(h->scales + h->n_keys, scales_dev, n * sizeof(float), cudaMemcpyDeviceToDevice, h->main));
+  if (h->phi) {
+    const int kd = h->cfg.key_dtype == AI_FP8E4M3 ? KD_FP8 : (h->cfg.key_dtype == AI_BF16 ? KD_BF16 : KD_FP32);
+    CK(launch_phi(h->keys, h->scales, kd, h->cfg.d, h->enc_wts, h->n_keys, h->n_keys + n, h->phi, h->main));
+  }
   h->n_keys += n;
   // the tensor-core refit screen reads fp8 keys through their bf16 copy
   if (h->cfg.key_dtype == AI_FP8E4M3 && h->cent_hi) return ensure_codes_bf16(h);

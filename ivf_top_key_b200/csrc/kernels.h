@@ -208,10 +208,15 @@ struct EncoderArgs {
   const double* centroids; // [.., d]
   int cl_begin, cl_end;    // clusters to (re)compute
   const float* wts;        // packed A [d,d], a [d], B1 [d, 3d+1], b1 [d], B2 [d,d], b2 [d]
+  const double* phi;       // [N, d] cached phi(k) per key (launch_phi), or nullptr
   uint16_t* reps;          // bf16 output
   int* err;
 };
 cudaError_t launch_encoder(const EncoderArgs& a, cudaStream_t st);
+// phi(k_s) = ReLU(A k_s + a) (float64) for keys s in [s0, s1) into phi[s]:
+// the per-key transform the encoder pools, computed once when keys arrive.
+cudaError_t launch_phi(const void* keys, const float* key_scale, int key_dtype, int d, const float* wts,
+                       int64_t s0, int64_t s1, double* phi, cudaStream_t st);
 
 // ---------------------------------------------------------------- formats
 cudaError_t launch_quantize_fp8(const uint16_t* keys_bf16, int64_t n, int d, uint8_t* codes,
