@@ -515,7 +515,10 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
             bj = j;
           }
         }
-        for (int o = 16; o > 0; o >>= 1) {
+        // lanes below m hold the candidates: the first step pairs lanes o0 apart
+        int o0 = 1;
+        while (2 * o0 < m && o0 < 16) o0 <<= 1;
+        for (int o = o0; o > 0; o >>= 1) {
           const uint64_t od = __shfl_xor_sync(0xffffffffu, bd, o);
           const uint32_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
           const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
