@@ -40,6 +40,10 @@ constexpr int kMaxBin = 64;                  // largest bin ranked by comparison
 static_assert(kCand >= kRowTopkMaxK, "the fallback sorts k keys in the same buffer");
 constexpr size_t kSmem = static_cast<size_t>(kCand) * 8 * 2 + static_cast<size_t>(kBins) * 4;
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Bin of hist[0 .. kBins) where the running count from bin 0 first reaches
 // target (1 <= target <= total), and the count before that bin.  All
 // threads call it; wt: 32 words of scratch.
@@ -178,6 +182,10 @@ __global__ void __launch_bounds__(kThreads) k_row_topk(RowTopkArgs a) {
   const float4* row4 = reinterpret_cast<const float4*>(row);
   const int n4r = (n4 + kThreads - 1) / kThreads * kThreads;  // whole warps for the votes
   for (int i = tid; i < n4r; i += 2 * kThreads) {
+    // the rows come from DRAM: the lines two iterations ahead are requested
+    // into L2 now, so more of the row is in flight than the loads below hold
+    if (i + 4 * kThreads < n4) prefetch_l2(row4 + i + 4 * kThreads);
+    if (i + 5 * kThreads < n4) prefetch_l2(row4 + i + 5 * kThreads);
     float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
     const bool ok0 = i < n4, ok1 = i + kThreads < n4;
     if (ok0) v0 = row4[i];
