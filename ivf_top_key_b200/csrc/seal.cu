@@ -28,6 +28,10 @@
 // histogram over the cluster's distance range (bins are a monotone function
 // of the distance, so the element lies in the bin where the running count
 // reaches it) and an exact rank among the few proposals of that one bin.
+// The histograms are built from every key's proposal in a pass's first
+// round and then kept current by the commit step: a committed key's count
+// is removed, and a free key whose cluster has just filled moves its count
+// to its next open cluster (the only proposals that change between rounds).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -311,8 +315,6 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
     s.cent[e] = key_f64(a, lo + ((2 * j + 1) * W) / (2 * m), i);
   }
   for (int i = tid; i < W; i += blockDim.x) s.prev[i] = -1;
-  // the histograms start at zero; the scan that reads a row clears it
-  for (int e = tid; e < m * kBins; e += blockDim.x) s.hist[e] = 0;
   __syncthreads();
 
   for (int it = 0; it < a.iters; ++it) {
@@ -329,6 +331,7 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
     else seal_dist_any(a, s, lo);
     for (int i = tid; i < W; i += blockDim.x) s.assign[i] = -1;
     for (int j = tid; j < m; j += blockDim.x) s.cnt[j] = 0;
+    for (int e = tid; e < m * kBins; e += blockDim.x) s.hist[e] = 0;
     if (tid == 0) {
       *s.fullmask = 0ull;
       s.misc[2] = W;
@@ -390,8 +393,9 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
     // greedy capacity assignment in rounds (see the file comment)
     for (int round = 0; round <= m && s.misc[2] > 0; ++round) {
       const unsigned long long fullm = *s.fullmask;
-      // B. proposals: best open cluster of every free key, counted per bin
-      for (int i = tid; i < W; i += blockDim.x) {
+      // B. (first round) proposals: best open cluster of every free key,
+      //    counted per bin; later rounds' proposals are kept by step G
+      for (int i = tid; i < (round == 0 ? W : 0); i += blockDim.x) {
         int bj = -1;
         if (s.assign[i] < 0) {
           if (m <= 8) {
@@ -416,11 +420,11 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         s.prop[i] = static_cast<int8_t>(bj);
         if (bj >= 0) atomicAdd(&s.hist[bj * kBins + s.bin[bj * W + i]], 1);
       }
-      __syncthreads();
+      if (round == 0) __syncthreads();
       // C. per open cluster, the bin where the running count reaches the
       //    (cap - count)-th proposal (none if the cluster cannot fill now):
       //    32-bin chunk sums, a scan over the chunks, a scan inside the one
-      //    chunk.  The row is cleared for the next round as it is read.
+      //    chunk.
       for (int j = warp; j < m; j += nwarps) {
         int found = -1, before = 0;
         if (!((fullm >> j) & 1ull)) {
@@ -451,8 +455,6 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
             found = c * 32 + first;
             before = base + __shfl_sync(0xffffffffu, incl - v, first);
           }
-          __syncwarp();
-          for (int c = 0; c < 32; ++c) hj[c * 32 + lane] = 0;
         }
         if (lane == 0) {
           s.tb[j] = found;
@@ -534,17 +536,47 @@ __global__ void __launch_bounds__(kThreads) k_seal(SealArgs a) {
         }
       }
       __syncthreads();
-      // G. commit every proposal up to the filling pair (all if none)
+      // G. commit every proposal up to the filling pair (all if none), and
+      //    keep the proposals and their counts current for the next round: a
+      //    committed key leaves its cluster's histogram (rows of full
+      //    clusters are not read again), and a free key whose cluster has
+      //    just filled proposes its next open cluster
       const int best = s.misc[0];
       const uint64_t bk1 = best >= 0 ? s.fk1[best] : 0;
       const uint32_t bi = best >= 0 ? (s.fk2[best] >> 16) : 0;
+      const unsigned long long fulln = *s.fullmask;  // now includes best
       for (int i0 = warp * 32; i0 < Wr; i0 += blockDim.x) {
         const int i = i0 + lane;
         const int j = i < W ? s.prop[i] : -1;
         bool take = false;
         if (j >= 0)
           take = best < 0 || pair_le(dbits(s.D[j * W + i]), i, j, bk1, bi, static_cast<uint32_t>(best));
-        if (take) s.assign[i] = static_cast<int16_t>(j);
+        if (take) {
+          s.assign[i] = static_cast<int16_t>(j);
+          s.prop[i] = -1;
+          if (best >= 0 && j != best) atomicSub(&s.hist[j * kBins + s.bin[j * W + i]], 1);
+        } else if (j >= 0 && j == best) {
+          int bj = -1;
+          if (m <= 8) {
+            uint32_t o = s.ord[i];
+            for (int g = 0; g < m && ((fulln >> (o & 15u)) & 1ull); ++g) o >>= 4;
+            s.ord[i] = o;
+            const int oj = static_cast<int>(o & 15u);
+            bj = (oj < m && !((fulln >> oj) & 1ull)) ? oj : -1;
+          } else {
+            double bd = 0.0;
+            for (int jj = 0; jj < m; ++jj) {
+              if ((fulln >> jj) & 1ull) continue;
+              const double v = s.D[jj * W + i];
+              if (bj < 0 || v < bd) {
+                bj = jj;
+                bd = v;
+              }
+            }
+          }
+          s.prop[i] = static_cast<int8_t>(bj);
+          if (bj >= 0) atomicAdd(&s.hist[bj * kBins + s.bin[bj * W + i]], 1);
+        }
         const int tj = take ? j : -1;
         const unsigned grp = __match_any_sync(0xffffffffu, tj);
         if (take && lane == __ffs(grp) - 1) atomicAdd(&s.cnt[j], __popc(grp));

@@ -493,3 +493,60 @@ def test_refine_kernel_choice():
     assert gpu.refine_kernel_choice(16384) == 4
     assert gpu.refine_kernel_choice(8192) == 3
     gpu.close()
+
+
+def test_exhaustive_row_topk_equal_score_paths():
+    """Rows whose top k holds many exactly equal scores (duplicated keys),
+    through the exhaustive selection (explainer, 它到底在解决什么问题？: the
+    indexer scores every key before the query and the k highest are kept;
+    equal scores go by key id ascending).  Rows 0..255 point along u0: 300
+    copies of one key lead their top k, so 300 equal keys share one bin of
+    the row top-k's ordering and that row takes the bitonic order.  Rows
+    256..511 point along u1: 9000 copies of another key lead, more keys lie
+    at or above the sampled threshold than the collecting buffer holds, and
+    the row takes the radix-select path.  Sampled rows agree with the
+    oracle's (its BLAS scores of equal keys may differ in the last bit, so
+    swaps among them are within the score tolerance); on the GPU the equal
+    keys score bit-equal and come out by id ascending."""
+    import types
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=20480, T=512, k=2048, budget=2048)
+    T, H, d, k = wl.T, wl.H, wl.d, wl.k
+    g = np.random.default_rng(11)
+    kf = S.keys_f64(wl, 0, wl.L)
+    u = g.standard_normal((2, d))
+    u[0] /= np.linalg.norm(u[0])
+    u[1] -= (u[1] @ u[0]) * u[0]
+    u[1] /= np.linalg.norm(u[1])
+    hi = 4.0 * np.linalg.norm(kf, axis=1).max()
+    pos = g.permutation(wl.L - T)            # keys every query of the chunk sees
+    a_pos, b_pos = np.sort(pos[:300]), np.sort(pos[300:9300])
+    kf[a_pos] = hi * u[0]
+    kf[b_pos] = hi * u[1]
+    bits = S.to_bf16_bits(kf)
+    keys = S.bf16_bits_to_f64(bits)
+    gpu, _ = P.make_pair(wl)
+    gpu.append_keys(torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16))
+    grp = (np.arange(T) >= T // 2).astype(int)
+    qb = S.to_bf16_bits(u[grp][:, None, :] + 0.02 * g.standard_normal((T, H, d)))
+    q = S.bf16_bits_to_f64(qb)
+    w = (np.abs(g.standard_normal((T, H))) / np.sqrt(H)).astype(np.float32)
+    qd = torch.from_numpy(qb.view(np.int16)).cuda().view(torch.bfloat16)
+    wd = torch.from_numpy(w).cuda()
+    p0 = wl.L - T
+    out = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    osc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    gpu.select_exhaustive(qd, wd, p0, k, out=out, out_scores=osc)
+    gpu.sync()
+    got, gs = out.cpu().numpy(), osc.cpu().numpy()
+    gpu.close()
+    w64 = w.astype(np.float64)
+    orc = types.SimpleNamespace(keys=keys,
+                                exhaustive=lambda qq, ww, t, kk: O.exhaustive_select(qq, ww, keys, t, kk))
+    for i in list(range(0, T // 2, 17)) + list(range(T // 2, T, 17)):
+        P.check_exhaustive(orc, p0 + i, q[i], w64[i], got[i], gs[i], k)
+    for i in range(T // 2):                   # 300 equal top scores, ids ascending
+        assert np.array_equal(got[i, :300], a_pos), f"row {i}"
+        assert np.all(gs[i, :300] == gs[i, 0]) and gs[i, 300] < gs[i, 0], f"row {i}"
+    for i in range(T // 2, T):                # the k smallest ids of 9000 equal scores
+        assert np.array_equal(got[i], b_pos[:k]), f"row {i}"
+        assert np.all(gs[i] == gs[i, 0]), f"row {i}"
