@@ -164,7 +164,7 @@ int ai_route_refine_shard(ai_handle h, const void* q_dev, const float* w_dev, in
  * of each query's union by (score desc, id asc) to out_dev [T, k] (and
  * out_scores_dev, nullable), -1 padded.  The parts must hold disjoint ids.
  * Enqueued on cuda_stream; needs no handle and allocates nothing.  Limits:
- * k <= 2048, (n_parts + 1) * k <= 29,000 (AI_ERR_ARG).                    */
+ * k <= 2048, n_parts * k <= 19,840 (AI_ERR_ARG).                          */
 int ai_merge_topk(const int32_t* ids_dev, const float* scores_dev, int32_t n_parts, int32_t T,
                   int32_t k, int32_t* out_dev, float* out_scores_dev, void* cuda_stream);
 
@@ -295,6 +295,19 @@ int ai_select_exhaustive_noalloc(const void* keys_dev, int32_t key_dtype, int64_
  * those calls fail with AI_ERR_CUDA.  Returns AI_OK, or AI_ERR_ARG for a
  * null handle or a kernel outside 0..4.                                   */
 int ai_debug_refine_kernel(ai_handle h, int32_t kernel);
+
+/* Parts per query for later ai_route_refine calls on h (tensor-core path,
+ * pipelined refine kernels).  A chunk of T queries with 2 * T at most the
+ * pipelined kernel's CTA count (two per SM) would leave most SMs idle, one
+ * CTA gathering each query's whole candidate list; instead each list's
+ * 128-slot tiles are divided among `split` CTAs (contiguous ranges, at
+ * least two tiles each) and their partial top-k merged by a second kernel
+ * into the documented output order.  Every tile, and so every score, is
+ * the same as undivided: results are identical either way.  split: 0 =
+ * chosen by chunk size (the default: up to 8 parts, and at most the CTA
+ * count divided by T), 1 = never divide, 2..8 = at most that many parts.
+ * Returns AI_OK, or AI_ERR_ARG for a null handle or split outside 0..8.   */
+int ai_debug_refine_split(ai_handle h, int32_t split);
 
 /* The refine kernel ai_route_refine launches on h for budget C:
  * *kernel_out = 0 for the fp32 (SIMT) path, else the tensor-core variant

@@ -125,6 +125,12 @@ class AttentionIndex:
         computes the same result."""
         C.ai_debug_refine_kernel(self.h, kernel)
 
+    def debug_refine_split(self, split: int):
+        """Parts per query of small chunks (0 = by chunk size, 1 = never
+        divide, 2..8 = at most that many); results are identical either
+        way."""
+        C.ai_debug_refine_split(self.h, split)
+
     def refine_kernel_choice(self, C_budget: int) -> int:
         """The refine kernel route_refine launches for this budget (0 = fp32
         SIMT path, 1 / 2 = one query per CTA, 3 / 4 = pipelined with two /

@@ -31,7 +31,7 @@ EXPORTED = [
     "ai_checkpoint", "ai_rollback", "ai_quantize_fp8", "ai_profile_enable", "ai_profile_read",
     "ai_kernel_launches", "ai_select_exhaustive_noalloc", "ai_debug_wait_timeout",
     "ai_route_refine_shard", "ai_merge_topk",
-    "ai_debug_refine_kernel", "ai_refine_kernel_choice",
+    "ai_debug_refine_kernel", "ai_refine_kernel_choice", "ai_debug_refine_split",
 ]
 PHASES = ["route", "refine", "seal", "refit", "publish", "exh_scores", "exh_topk", "order"]
 
@@ -92,6 +92,7 @@ def _load():
         "ai_merge_topk": [vp, vp, i32, i32, i32, vp, vp, vp],
         "ai_debug_wait_timeout": [i32, ctypes.POINTER(i32), vp],
         "ai_debug_refine_kernel": [vp, i32],
+        "ai_debug_refine_split": [vp, i32],
         "ai_refine_kernel_choice": [vp, i32, ctypes.POINTER(i32)],
     }
     for name, args in sig.items():
@@ -274,6 +275,12 @@ def ai_debug_refine_kernel(h, kernel: int):
     list in shared memory, 2 sequential with a global list, 3 pipelined,
     4 pipelined with one TMEM score buffer)."""
     _check(_lib.ai_debug_refine_kernel(h, kernel))
+
+
+def ai_debug_refine_split(h, split: int):
+    """Parts per query of small chunks on the pipelined refine (0 = by
+    chunk size, 1 = never divide, 2..8 = at most that many)."""
+    _check(_lib.ai_debug_refine_split(h, split))
 
 
 def ai_refine_kernel_choice(h, C: int) -> int:

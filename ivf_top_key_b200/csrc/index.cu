@@ -200,7 +200,10 @@ struct ai_index {
   float* cent_cc = nullptr;
   int32_t* cand_scratch = nullptr;  // tensor-core refine: candidate lists, 4 per SM
   float* topk_scores = nullptr;      // tensor-core refine: scores for the output ordering [max_query_chunk, max_k]
+  int32_t* split_ids = nullptr;      // split refine of small chunks: partial top-k [2 * num_sms, max_k]
+  float* split_sc = nullptr;
   int refine_kernel = 0;             // tensor-core refine variant (0 = by occupancy)
+  int refine_split = 0;              // parts per query of a small chunk (0 = by chunk size, 1 = none)
   int32_t* upd_chunk_off = nullptr;  // refit update chunks
   double* upd_part = nullptr;
   float* band_best = nullptr;  // near-tie bands of the tensor-core refit scan
@@ -699,6 +702,8 @@ int ai_index_create(const ai_config* cfg, void* cuda_stream, ai_handle* out) {
   // one candidate row per refine CTA (at most 4 per SM)
   if (tck) CKC(dalloc(&h->cand_scratch, static_cast<size_t>(h->num_sms) * 4 * c.max_budget));
   if (tck) CKC(dalloc(&h->topk_scores, static_cast<size_t>(c.max_query_chunk) * c.max_k));
+  if (tck) CKC(dalloc(&h->split_ids, static_cast<size_t>(2 * h->num_sms) * c.max_k));
+  if (tck) CKC(dalloc(&h->split_sc, static_cast<size_t>(2 * h->num_sms) * c.max_k));
   if (tcr) CKC(dalloc(&h->route_kmin, static_cast<size_t>(c.max_query_chunk) * 4));
   if (tcr) CKC(dalloc(&h->route_kmax, static_cast<size_t>(c.max_query_chunk) * 4));
   CKC(dalloc(&h->upd_chunk_off, h->maxC + 1));
@@ -757,6 +762,8 @@ int ai_index_destroy(ai_handle h) {
   cudaFree(h->cent_cc);
   cudaFree(h->cand_scratch);
   cudaFree(h->topk_scores);
+  cudaFree(h->split_ids);
+  cudaFree(h->split_sc);
   cudaFree(h->route_kmin);
   cudaFree(h->route_kmax);
   cudaFree(h->upd_chunk_off);
@@ -863,6 +870,23 @@ int ai_publish(ai_handle h) {
   return publish(h);
 }
 
+// Parts per query of a chunk on the pipelined refine.  A chunk with at
+// most half as many queries as the kernel's CTAs (two per SM) would leave
+// most SMs idle, each query's 128-slot tiles gathered by one CTA; its list
+// is divided instead among `split` CTAs (contiguous tile ranges, at least
+// two tiles each, at most kMaxSplit parts) and their partial top-k merged.
+// The tiles and so every score are the same as undivided.
+constexpr int kMaxSplit = 8;
+static int refine_split_for(const ai_index* h, int T, int C, int k) {
+  const int cap = 2 * h->num_sms;
+  if (h->refine_split == 1 || T <= 0 || 2 * T > cap) return 1;
+  int S = h->refine_split > 1 ? h->refine_split : kMaxSplit;
+  S = std::min(S, cap / T);
+  S = std::min(S, ((C + 127) / 128) / 2);
+  while (S > 1 && merge_smem_bytes(S, k) > 227 * 1024) --S;
+  return S < 2 ? 1 : S;
+}
+
 static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t pos0, int T, int k,
                              int C, int32_t* out, float* out_scores, int32_t* cand_out,
                              float* cluster_scores_out, int shard = 0, int n_shards = 1) {
@@ -929,6 +953,27 @@ static int route_refine_impl(ai_handle h, const void* q, const float* w, int64_t
       return fail(AI_ERR_CUDA, "tensor map encoding failed (key store / queries)");
     kmp = &kmap;
     qmp = &qmap;
+  }
+  // a small chunk on the pipelined refine: each query's list divided among
+  // CTAs, the partial top-k merged into the output order
+  int split = 1;
+  if (tc_keys(h) && !cand_out && out && n_shards <= 1 && h->split_ids) {
+    const int kind = h->refine_kernel == REFINE_AUTO
+                         ? pick_refine_kernel(C, h->cfg.H, h->cand_scratch != nullptr)
+                         : h->refine_kernel;
+    if (kind == REFINE_PIPE || kind == REFINE_PIPE_1BUF) split = refine_split_for(h, T, C, k);
+  }
+  if (split > 1) {
+    ra.split = split;
+    ra.out = h->split_ids;
+    ra.out_scores = h->split_sc;
+    const int pf = prof_begin(h, AI_PHASE_REFINE, h->main);
+    CK(launch_refine(ra, vt, kmp, qmp, h->num_sms, h->main));
+    prof_end(h, pf, h->main);
+    const int po = prof_begin(h, AI_PHASE_ORDER, h->main);
+    CK(launch_merge_rows(h->split_ids, h->split_sc, split, T, k, out, out_scores, h->main));
+    prof_end(h, po, h->main);
+    return AI_OK;
   }
   // the tensor-core refine writes each row's ids (and scores) in slot
   // order; a second kernel puts them in the output order, reading the
@@ -1146,6 +1191,13 @@ int ai_debug_refine_kernel(ai_handle h, int32_t kernel) {
   if (!h) return fail(AI_ERR_ARG, "null handle");
   if (kernel < 0 || kernel > 4) return fail(AI_ERR_ARG, "refine kernel must be 0..4");
   h->refine_kernel = kernel;
+  return AI_OK;
+}
+
+int ai_debug_refine_split(ai_handle h, int32_t split) {
+  if (!h) return fail(AI_ERR_ARG, "null handle");
+  if (split < 0 || split > kMaxSplit) return fail(AI_ERR_ARG, "refine split must be 0..8");
+  h->refine_split = split;
   return AI_OK;
 }
 

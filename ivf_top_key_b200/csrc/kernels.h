@@ -75,6 +75,9 @@ struct RefineArgs {
   int32_t* cand_scratch;     // tensor-core path: candidate lists, [4 * num_sms, C]
   int refine_kernel;         // REFINE_* (tensor-core path; AUTO picks by occupancy)
   int shard, n_shards;       // rescore only this shard's tile range of each list (n_shards <= 1: all)
+  int split;                 // pipelined kernels: > 1 divides each list's tiles among `split` work
+                             // items; item sp of query i writes row sp * T + i of out / out_scores
+                             // ([split, T, k]), to be merged
   int* err;
 };
 enum RefineKernel {
@@ -111,6 +114,13 @@ struct OrderRowsArgs {
   int T, k;
 };
 cudaError_t launch_order_rows(const OrderRowsArgs& a, cudaStream_t st);
+// Merge of P partial top-k lists per row, ids / scores [P, T, k] (valid
+// entries id >= 0, disjoint ids across parts): the top k of their union by
+// (score desc, id asc), written in that order to out / out_scores [T, k]
+// and padded with -1 / -inf.  k <= kTcMaxK; shared memory merge_smem_bytes.
+size_t merge_smem_bytes(int P, int k);
+cudaError_t launch_merge_rows(const int32_t* ids, const float* scores, int P, int T, int k, int32_t* out,
+                              float* out_scores, cudaStream_t st);
 
 // ------------------------------------------------------- exhaustive top-k
 struct RowTopkArgs {

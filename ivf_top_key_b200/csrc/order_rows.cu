@@ -22,6 +22,15 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxK = 2048;
+
+// Slots for the valid entries of a merge row: all P * k, and room for the
+// power of two the bitonic fallback of emit_sorted_prefix sorts in place.
+__host__ __device__ inline int merge_items_cap(int P, int k) {
+  const int L = P * k;
+  int np = 1;
+  while (np < (L < 8192 ? L : 8192)) np <<= 1;
+  return L > np ? L : np;
+}
 constexpr int kBins = 2048;
 constexpr int kMaxBin = 64;
 
@@ -151,26 +160,30 @@ __global__ void __launch_bounds__(kThreads) k_order_rows(OrderRowsArgs a) {
   }
 }
 
-// Merge of P partial top-k lists per row (the shards of a sharded rescore):
-// the valid (id >= 0) entries of the row's P lists are compacted into
-// shared memory, and the block selects their top k by (score desc, id asc),
-// written in that order and padded with -1.  The partial lists hold
-// disjoint ids, and each holds its shard's top k, so the union holds the
-// row's top k.
+// Merge of P partial top-k lists per row (the shards of a sharded rescore,
+// or the parts of a divided one): the valid (id >= 0) entries of the row's
+// P lists are compacted into shared memory as order keys, and the block
+// writes the first k of them in order (score desc, id asc), padded with -1.
+// The partial lists hold disjoint ids, and each holds its part's top k, so
+// the union holds the row's top k.  Up to kMergeSort valid entries are
+// ordered by the counting sort of emit_sorted_prefix; more take a radix
+// select of the top k and a bitonic sort.
+constexpr int kMergeSort = 8192;
+
 __global__ void __launch_bounds__(1024) k_merge_rows(const int32_t* __restrict__ ids,
                                                     const float* __restrict__ scores, int P, int T, int k,
                                                     int32_t* out, float* out_scores) {
   extern __shared__ __align__(16) uint8_t raw[];
-  int np = 1;
-  while (np < k) np <<= 1;
-  uint64_t* sbuf = reinterpret_cast<uint64_t*>(raw);        // output sort [np]
-  uint64_t* items = sbuf + np;                              // [P * k] valid entries
+  const int L = P * k;
+  const int cap = merge_items_cap(P, k);
+  uint64_t* items = reinterpret_cast<uint64_t*>(raw);       // [cap] valid entries
+  uint64_t* grp = items + cap;                              // [kMergeSort] grouping / output sort
+  uint32_t* hist = reinterpret_cast<uint32_t*>(grp + kMergeSort);  // [kPrefixBins]
   __shared__ BlockScratch bs;
   __shared__ int s_n;
   const int row = blockIdx.x, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) s_n = 0;
   __syncthreads();
-  const int L = P * k;
   const int Lr = (L + 31) & ~31;  // whole warps for the ballots
   for (int e = threadIdx.x; e < Lr; e += blockDim.x) {
     int32_t id = -1;
@@ -193,18 +206,38 @@ __global__ void __launch_bounds__(1024) k_merge_rows(const int32_t* __restrict__
   }
   __syncthreads();
   const int n = s_n;
-  topk_select_emit(
-      n, [&](int i) -> float { return order_key_score(items[i]); },
-      [&](int i) -> int32_t { return order_key_id(items[i]); }, k, out + static_cast<int64_t>(row) * k,
-      out_scores ? out_scores + static_cast<int64_t>(row) * k : nullptr, bs, sbuf);
+  int32_t* o_ids = out + static_cast<int64_t>(row) * k;
+  float* o_sc = out_scores ? out_scores + static_cast<int64_t>(row) * k : nullptr;
+  if (n <= kMergeSort) {
+    const int nw = n < k ? n : k;
+    emit_sorted_prefix(items, n, nw, grp, hist, o_ids, o_sc);
+    for (int j = nw + threadIdx.x; j < k; j += blockDim.x) {
+      o_ids[j] = -1;
+      if (o_sc) o_sc[j] = -INFINITY;
+    }
+  } else {
+    topk_select_emit(
+        n, [&](int i) -> float { return order_key_score(items[i]); },
+        [&](int i) -> int32_t { return order_key_id(items[i]); }, k, o_ids, o_sc, bs, grp);
+  }
 }
 
 }  // namespace
 
 size_t merge_smem_bytes(int P, int k) {
-  size_t np = 1;
-  while (np < static_cast<size_t>(k)) np <<= 1;
-  return (np + static_cast<size_t>(P) * k) * 8;
+  return static_cast<size_t>(merge_items_cap(P, k)) * 8 + static_cast<size_t>(kMergeSort) * 8 +
+         static_cast<size_t>(kPrefixBins) * 4;
+}
+
+cudaError_t launch_merge_rows(const int32_t* ids, const float* scores, int P, int T, int k, int32_t* out,
+                              float* out_scores, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const size_t smem = merge_smem_bytes(P, k);
+  if (P < 1 || k < 1 || k > kTcMaxK || smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaFuncSetAttribute(k_merge_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  count_launch();
+  k_merge_rows<<<T, 1024, smem, st>>>(ids, scores, P, T, k, out, out_scores);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_order_rows(const OrderRowsArgs& a, cudaStream_t st) {
@@ -231,15 +264,12 @@ extern "C" int ai_merge_topk(const int32_t* ids_dev, const float* scores_dev, in
   }
   const size_t smem = merge_smem_bytes(n_parts, k);
   if (smem > 227 * 1024) {
-    set_last_error("n_parts * k too large for one block (n_parts * k + k <= 29000)");
+    set_last_error("n_parts * k too large for one block (n_parts * k <= 19840)");
     return AI_ERR_ARG;
   }
   if (T == 0) return AI_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  cudaFuncSetAttribute(k_merge_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  count_launch();
-  k_merge_rows<<<T, 1024, smem, st>>>(ids_dev, scores_dev, n_parts, T, k, out_dev, out_scores_dev);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_merge_rows(ids_dev, scores_dev, n_parts, T, k, out_dev, out_scores_dev,
+                                          static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) {
     set_last_error(cudaGetErrorString(e));
     return AI_ERR_CUDA;

@@ -75,18 +75,36 @@ __device__ __forceinline__ void bitonic_sort_u64(uint64_t* buf, int n, const G& 
   }
 }
 
-// The share of a candidate list of n slots that one shard rescores: the
-// whole list, or (n_shards > 1) a contiguous range of its 128-slot tiles.
-// The rescore and the top-k run on the list shifted to that range.
-__device__ __forceinline__ void shard_span(const RefineArgs& a, int n, int* off, int* n_loc) {
-  if (a.n_shards <= 1) {
+// Work item q of this CTA in the pipelined kernel: query qi, and (split > 1)
+// the part sp of its list that this item rescores.  Items run query-major:
+// the split parts of a query go to neighbouring CTAs.
+struct RefineItem {
+  int qi, sp;
+};
+__device__ __forceinline__ int refine_split(const RefineArgs& a) { return a.split > 1 ? a.split : 1; }
+__device__ __forceinline__ RefineItem refine_item(const RefineArgs& a, int q) {
+  const int S = refine_split(a);
+  const int v = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+  return RefineItem{v / S, v % S};
+}
+
+// The share of a candidate list of n slots that one item rescores: the
+// whole list, or a contiguous range of its 128-slot tiles when the list is
+// divided among shards (ranks; n_shards > 1) and, inside this launch, among
+// the split parts of the query (part sp of split).  The rescore and the
+// top-k run on the list shifted to that range.
+__device__ __forceinline__ void shard_span(const RefineArgs& a, int sp, int n, int* off, int* n_loc) {
+  const int S = refine_split(a);
+  const int parts = (a.n_shards > 1 ? a.n_shards : 1) * S;
+  if (parts <= 1) {
     *off = 0;
     *n_loc = n;
     return;
   }
+  const int part = (a.n_shards > 1 ? a.shard : 0) * S + sp;
   const int tiles = (n + kTile - 1) / kTile;
-  const int t0 = static_cast<int>(static_cast<int64_t>(a.shard) * tiles / a.n_shards);
-  const int t1 = static_cast<int>(static_cast<int64_t>(a.shard + 1) * tiles / a.n_shards);
+  const int t0 = static_cast<int>(static_cast<int64_t>(part) * tiles / parts);
+  const int t1 = static_cast<int>(static_cast<int64_t>(part + 1) * tiles / parts);
   const int e = n < t1 * kTile ? n : t1 * kTile;
   *off = t0 * kTile;
   *n_loc = e > t0 * kTile ? e - t0 * kTile : 0;
@@ -703,10 +721,10 @@ __device__ __forceinline__ void p3_find_bin(P3Smem& ps, int et, int k, int* bsta
   named_bar(1, 128);
 }
 
-__device__ void p3_topk(const RefineArgs& a, int qi, const P3Ctx& c, int et, P3Smem& ps) {
+__device__ void p3_topk(const RefineArgs& a, int orow, const P3Ctx& c, int et, P3Smem& ps) {
   const int k = a.k;
-  int32_t* out = a.out + static_cast<int64_t>(qi) * k;
-  float* outs = a.out_scores ? a.out_scores + static_cast<int64_t>(qi) * k : nullptr;
+  int32_t* out = a.out + static_cast<int64_t>(orow) * k;
+  float* outs = a.out_scores ? a.out_scores + static_cast<int64_t>(orow) * k : nullptr;
   // range of the valid scores
   float vmin = INFINITY, vmax = -INFINITY;
   p3_for_each(c, [&](float v, int) {
@@ -1299,7 +1317,8 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int nq = static_cast<int>(blockIdx.x) < a.T ? (a.T - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+  const int n_items = a.T * refine_split(a);
+  const int nq = static_cast<int>(blockIdx.x) < n_items ? (n_items - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
 
   // Gathering warp gw (0 .. NGW-1) owns rows [gw * RPW, gw * RPW + RPW) of
   // every tile; lane l holds the id of row gw * RPW + l % RPW and lanes
@@ -1339,7 +1358,8 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     int64_t last_issued = -1;
     bool dead = false;
     for (int q = 0; q < nq; ++q) {
-      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const RefineItem it = refine_item(a, q);
+      const int qi = it.qi;
       const int64_t t = a.pos0 + qi;
       const int b = q & 1;
       const bool ok = !dead && mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
@@ -1348,7 +1368,7 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       if (!named_bar_and(3, 128, ok)) break;
       tc_fence_after();
       int off, n;
-      shard_span(a, meta[b], &off, &n);
+      shard_span(a, it.sp, meta[b], &off, &n);
       const int nt = (n + kTile - 1) / kTile;
       const int32_t* cl = rows + static_cast<int64_t>(b) * a.C + off;
       for (int h = row; h < H; h += 128) wsh[h] = a.w[static_cast<int64_t>(qi) * H + h];
@@ -1425,11 +1445,12 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       uint32_t g = 0;
       int commits = 0;
       for (int q = 0; q < nq; ++q) {
-        const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+        const RefineItem it = refine_item(a, q);
+        const int qi = it.qi;
         const int b = q & 1;
         if (!mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag)) break;
         int off, n_loc;
-        shard_span(a, meta[b], &off, &n_loc);
+        shard_span(a, it.sp, meta[b], &off, &n_loc);
         const int nt = (n_loc + kTile - 1) / kTile;
         mbar_arrive(&mread[b]);  // the slot's length is read; it may be rebuilt
         // the head tile is rewritten once the previous query's UMMAs are done
@@ -1475,13 +1496,14 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     uint32_t g = 0;
     int64_t last_issued = -1;
     for (int q = 0; q < nq; ++q) {
-      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const RefineItem it = refine_item(a, q);
+      const int qi = it.qi;
       const int64_t t = a.pos0 + qi;
       const int b = q & 1;
       const bool ok = mbar_wait(&cready[b], (q >> 1) & 1, a.err, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       int off, n;
-      shard_span(a, meta[b], &off, &n);
+      shard_span(a, it.sp, meta[b], &off, &n);
       const int nt = (n + kTile - 1) / kTile;
       const int32_t* cl = rows + static_cast<int64_t>(b) * a.C + off;
       int gid = next_gid(-1, gw, n, cl);
@@ -1525,14 +1547,15 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
         const bool w = mbar_wait(&mread[q & 1], ((q - 2) >> 1) & 1, a.err, abort_flag);
         if (!named_bar_and(2, 128, w)) return false;
       }
-      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const RefineItem it = refine_item(a, q);
+      const int qi = it.qi;
       const int64_t t = a.pos0 + qi;
       int nC;
       int64_t n_v;
       version_of(vt, t, &nC, &n_v);
       int32_t* cl = rows + static_cast<int64_t>(q & 1) * a.C;
       const int n = build_candidates<true>(a, qi, t, nC, n_v, cl, sortbuf, pref, grp);
-      if (a.cand_out) {
+      if (a.cand_out && it.sp == 0) {
         for (int i = et; i < a.C; i += 128) a.cand_out[static_cast<int64_t>(qi) * a.C + i] = i < n ? cl[i] : -1;
       }
       if (et == 0) meta[q & 1] = n;
@@ -1541,7 +1564,8 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
     };
     const bool started = nq > 0 && build(0);
     for (int q = 0; started && q < nq; ++q) {
-      const int qi = static_cast<int>(blockIdx.x) + q * static_cast<int>(gridDim.x);
+      const RefineItem it = refine_item(a, q);
+      const int qi = it.qi;
       if (q + 1 < nq && !build(q + 1)) break;
       const bool ok = mbar_wait(&sready[q & 1], (q >> 1) & 1, a.err, abort_flag);
       if (!named_bar_and(1, 128, ok)) break;
@@ -1551,10 +1575,11 @@ __global__ void __launch_bounds__(pipe_threads(NGW), kTcCtasPerSm)
       c.row = quarter * 32 + lane;
       c.tcol = tmem_base + 2 * H + (q % NSB) * sc_cols + (static_cast<uint32_t>(quarter * 32) << 16);
       int off;
-      shard_span(a, meta[q & 1], &off, &c.n);
+      shard_span(a, it.sp, meta[q & 1], &off, &c.n);
       c.ntiles = (c.n + kTile - 1) / kTile;
       c.cand = rows + static_cast<int64_t>(q & 1) * a.C + off;
-      p3_topk(a, qi, c, c.row, ps);  // c.row == et: rows in thread order
+      // output row: the query's, or (split) its part's row of [split, T, k]
+      p3_topk(a, it.sp * a.T + qi, c, c.row, ps);  // c.row == et: rows in thread order
       tc_fence_before();
       mbar_arrive(&sfree[q % NSB]);
     }
@@ -1618,13 +1643,14 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
                                                     : a.refine_kernel;
     if (kind < REFINE_SEQ_SMEM || kind > REFINE_PIPE_1BUF) return cudaErrorInvalidValue;
     const bool pipe = kind == REFINE_PIPE || kind == REFINE_PIPE_1BUF;
-    if (a.n_shards > 1 && !pipe) return cudaErrorInvalidValue;  // sharded rescore: pipelined kernels only
+    if ((a.n_shards > 1 || a.split > 1) && !pipe) return cudaErrorInvalidValue;  // pipelined kernels only
     if ((kind == REFINE_SEQ_GLOBAL || pipe) && !a.cand_scratch) return cudaErrorInvalidValue;
     const int tm = pipe ? pipe_tmem_cols(a.C, a.H, kind == REFINE_PIPE ? 2 : 1) : tc_tmem_cols(a.C, a.H);
     const size_t smem_tc = kind == REFINE_SEQ_SMEM ? sm_local : kind == REFINE_SEQ_GLOBAL ? sm_glob : sm_pipe;
     if (smem_tc > kMaxSmem || tm > 512) return cudaErrorInvalidValue;
     const int per_sm = per_sm_for(smem_tc, tm);
-    const int grid = a.T < num_sms * per_sm ? a.T : num_sms * per_sm;
+    const int items = pipe ? a.T * (a.split > 1 ? a.split : 1) : a.T;
+    const int grid = items < num_sms * per_sm ? items : num_sms * per_sm;
     if (grid <= 0) return cudaSuccess;
 #define AI_LAUNCH_REFINE(KERNEL)                                                                         \
   do {                                                                                                   \
@@ -1646,7 +1672,7 @@ cudaError_t launch_refine(const RefineArgs& a, const VersionTable& vt, const CUt
     }
 #undef AI_LAUNCH_REFINE
   } else {
-    if (a.n_shards > 1) return cudaErrorInvalidValue;
+    if (a.n_shards > 1 || a.split > 1) return cudaErrorInvalidValue;
     // the output sort reuses the phase-1 region: room for kRowTopkMaxK keys
     if (a.k > kRowTopkMaxK || region_bytes(a.H, a.d, false) < static_cast<size_t>(kRowTopkMaxK) * 8)
       return cudaErrorInvalidValue;

@@ -5,15 +5,20 @@
 // cluster threshold of the candidate fill.
 #pragma once
 
+#include <cstddef>
+
 #include "common.cuh"
 
 namespace aiidx {
 
-struct BlockScratch {
+// 16-byte aligned: bcast[2 .. 3] also holds a 64-bit value (offset 1192),
+// which needs an 8-byte aligned address whatever else the block declares.
+struct __align__(16) BlockScratch {
   uint32_t hist[256];     // radix histogram (counts or weights)
   int warp_tot[40];       // per-warp totals for ordered compaction
   int bcast[8];           // broadcast slots
 };
+static_assert(offsetof(BlockScratch, bcast) % 8 == 0, "bcast[2] holds a 64-bit value");
 
 // Exclusive prefix of `pred` over the block in thread order.  Returns this
 // thread's rank among the threads with pred set; *total receives the count.
@@ -218,6 +223,174 @@ __device__ void topk_select_emit(int n, ScoreF score, IdF id, int k, int32_t* ou
     const uint64_t x = v ? sbuf[j] : kOrderPad;
     out[j] = v ? order_key_id(x) : -1;
     if (outs) outs[j] = v ? order_key_score(x) : -INFINITY;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------- sorted prefix of a key set
+// For blocks of exactly 1024 threads.  keys[0 .. c) hold c distinct order
+// keys (any order); their first nw (nw <= c) in ascending order -- score
+// descending, id ascending -- are written to out[0 .. nw) (ids) and
+// outs[0 .. nw) (scores, if outs).  A counting sort: the keys are grouped
+// by bin of their score key over the set's range (kPrefixBins equal integer
+// ranges of the order-preserving key, about constant relative width), and a
+// key's position is its bin's start plus its rank among the bin's keys;
+// only the bins that start before nw are grouped and ranked.  One of those
+// holding more than 64 keys (near-equal scores) sends the block to a
+// bitonic sort of keys instead, which needs keys to hold the next power of
+// two >= c slots.  grp: c slots of scratch; hist: kPrefixBins words.  Ends
+// with the block synchronised; keys and grp are clobbered.
+constexpr int kPrefixBins = 2048;
+
+__device__ inline void emit_sorted_prefix(uint64_t* keys, int c, int nw, uint64_t* grp, uint32_t* hist, int32_t* out,
+                                   float* outs) {
+  constexpr int kMaxBin = 64;
+  __shared__ uint32_t s_wt[32], s_red[2][32];
+  __shared__ int s_bmax, s_bend;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // score-key range of the keys (high words: ~f2key(score))
+  uint32_t hmn = 0xffffffffu, hmx = 0u;
+  for (int j = tid; j < c; j += 1024) {
+    const uint32_t h = static_cast<uint32_t>(keys[j] >> 32);
+    hmn = min(hmn, h);
+    hmx = max(hmx, h);
+  }
+  for (int i = tid; i < kPrefixBins; i += 1024) hist[i] = 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    hmn = min(hmn, __shfl_xor_sync(0xffffffffu, hmn, o));
+    hmx = max(hmx, __shfl_xor_sync(0xffffffffu, hmx, o));
+  }
+  if (lane == 0) {
+    s_red[0][warp] = hmn;
+    s_red[1][warp] = hmx;
+  }
+  __syncthreads();
+  hmn = s_red[0][0];
+  hmx = s_red[1][0];
+  for (int w = 1; w < 32; ++w) {
+    hmn = min(hmn, s_red[0][w]);
+    hmx = max(hmx, s_red[1][w]);
+  }
+  // Keys are binned by (hi - hmn) >> sh over [hmn, hhi]; keys above hhi
+  // (lower scores) get bin kPrefixBins.  After the first histogram the
+  // first nw keys are known to lie in bins [0, b_end); when that is a small
+  // part of the range (a wide range: outliers, scores of both signs) the
+  // histogram is taken once more over just that part.
+  uint32_t hhi = hmx;
+  int sh = 0;
+  auto bin = [&](uint64_t x) -> int {
+    const uint32_t h = static_cast<uint32_t>(x >> 32);
+    return h > hhi ? kPrefixBins : static_cast<int>((h - hmn) >> sh);
+  };
+  for (int round = 0;; ++round) {
+    sh = 0;
+    while (sh < 32 && (static_cast<uint64_t>(hhi - hmn) >> sh) >= static_cast<uint64_t>(kPrefixBins)) ++sh;
+    if (round > 0) {
+      for (int i = tid; i < kPrefixBins; i += 1024) hist[i] = 0;
+      __syncthreads();
+    }
+    for (int j = tid; j < c; j += 1024) {
+      const int b = bin(keys[j]);
+      if (b < kPrefixBins) atomicAdd(&hist[b], 1u);
+    }
+    __syncthreads();
+    // exclusive scan of the counts (thread t owns bins 2t, 2t + 1)
+    const uint32_t c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
+    const uint32_t loc = c0 + c1;
+    uint32_t incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t tt = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += tt;
+    }
+    if (lane == 31) s_wt[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t v = s_wt[lane];
+      uint32_t in2 = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t tt = __shfl_up_sync(0xffffffffu, in2, o);
+        if (lane >= o) in2 += tt;
+      }
+      s_wt[lane] = in2 - v;
+    }
+    __syncthreads();
+    const uint32_t st0 = s_wt[warp] + incl - loc, st1 = st0 + c0;  // bin starts
+    // Only the bins starting before nw hold any of the first nw keys (bins
+    // run from the highest scores down): b_end is the first bin starting at
+    // or after nw, and the largest count among the bins before it decides
+    // between the counting sort and the bitonic sort.
+    uint32_t cm = max(st0 < static_cast<uint32_t>(nw) ? c0 : 0u, st1 < static_cast<uint32_t>(nw) ? c1 : 0u);
+    uint32_t be = st0 >= static_cast<uint32_t>(nw) ? 2 * tid
+                                                    : (st1 >= static_cast<uint32_t>(nw) ? 2 * tid + 1 : kPrefixBins);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+      be = min(be, __shfl_xor_sync(0xffffffffu, be, o));
+    }
+    if (lane == 0) {
+      s_red[0][warp] = cm;
+      s_red[1][warp] = be;
+    }
+    hist[2 * tid] = st0;
+    hist[2 * tid + 1] = st1;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t m2 = s_red[0][lane], b2 = s_red[1][lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        m2 = max(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+        b2 = min(b2, __shfl_xor_sync(0xffffffffu, b2, o));
+      }
+      if (lane == 0) {
+        s_bmax = static_cast<int>(m2);
+        s_bend = static_cast<int>(b2);
+      }
+    }
+    __syncthreads();
+    const int be_all = s_bend;
+    if (round > 0 || sh == 0 || be_all > kPrefixBins / 4) break;
+    // the keys of bins [0, be_all) span hi in [hmn, hmn + (be_all << sh) - 1]
+    const uint64_t top = static_cast<uint64_t>(hmn) + (static_cast<uint64_t>(be_all) << sh) - 1;
+    hhi = top < hhi ? static_cast<uint32_t>(top) : hhi;
+    __syncthreads();  // every thread has read s_bend before the next round
+  }
+  const int b_end = s_bend;
+  // keys of bins [0, b_end) fill grp[0 .. n_rel) after grouping
+  const int n_rel = b_end < kPrefixBins ? static_cast<int>(hist[b_end]) : c;
+  if (s_bmax <= kMaxBin) {
+    // group the keys of bins before b_end; afterwards such a bin b spans
+    // [end(b - 1), hist[b]) with end(-1) = 0
+    for (int j = tid; j < c; j += 1024) {
+      const uint64_t x = keys[j];
+      const int b = bin(x);
+      if (b < b_end) grp[atomicAdd(&hist[b], 1u)] = x;
+    }
+    __syncthreads();
+    for (int p = tid; p < n_rel; p += 1024) {
+      const uint64_t x = grp[p];
+      const int b = bin(x);
+      const int lo = b == 0 ? 0 : static_cast<int>(hist[b - 1]);
+      const int hi = static_cast<int>(hist[b]);
+      int rk = lo;
+      for (int q = lo; q < hi; ++q) rk += grp[q] < x ? 1 : 0;
+      if (rk < nw) {
+        out[rk] = order_key_id(x);
+        if (outs) outs[rk] = order_key_score(x);
+      }
+    }
+  } else {
+    int np = 1;
+    while (np < c) np <<= 1;
+    for (int j = c + tid; j < np; j += 1024) keys[j] = kOrderPad;
+    __syncthreads();
+    block_sort_u64(keys, np);
+    for (int j = tid; j < nw; j += 1024) {
+      out[j] = order_key_id(keys[j]);
+      if (outs) outs[j] = order_key_score(keys[j]);
+    }
   }
   __syncthreads();
 }

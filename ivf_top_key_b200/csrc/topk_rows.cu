@@ -35,8 +35,7 @@ constexpr int kThreads = 1024;
 constexpr int kCand = 8192;                  // collected keys held in shared memory
 constexpr int kPerThread = 8;                // sampled scores per thread
 constexpr int kSample = kThreads * kPerThread;
-constexpr int kBins = 2048;                  // histogram bins (2 per thread)
-constexpr int kMaxBin = 64;                  // largest bin ranked by comparisons
+constexpr int kBins = kPrefixBins;          // histogram bins (2 per thread)
 static_assert(kCand >= kRowTopkMaxK, "the fallback sorts k keys in the same buffer");
 constexpr size_t kSmem = static_cast<size_t>(kCand) * 8 * 2 + static_cast<size_t>(kBins) * 4;
 
@@ -90,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) k_row_topk(RowTopkArgs a) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(grp + kCand);  // [kBins]
   __shared__ BlockScratch bs;
   __shared__ uint32_t s_wt[32], s_red[2][32];
-  __shared__ int s_cnt, s_bin, s_bmax;
+  __shared__ int s_cnt, s_bin;
   __shared__ uint32_t s_before;
   const int qi = blockIdx.x;
   const int64_t t = a.q_pos0 + qi;
@@ -213,102 +212,7 @@ __global__ void __launch_bounds__(kThreads) k_row_topk(RowTopkArgs a) {
   if (c >= (k < n ? k : n) && c <= kCand) {
     // 3. the first k collected keys in order
     const int nw = k < c ? k : c;
-    // score-key range of the collected keys (high words: ~f2key(score))
-    uint32_t hmn = 0xffffffffu, hmx = 0u;
-    for (int j = tid; j < c; j += kThreads) {
-      const uint32_t h = static_cast<uint32_t>(cand[j] >> 32);
-      hmn = min(hmn, h);
-      hmx = max(hmx, h);
-    }
-    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      hmn = min(hmn, __shfl_xor_sync(0xffffffffu, hmn, o));
-      hmx = max(hmx, __shfl_xor_sync(0xffffffffu, hmx, o));
-    }
-    if (lane == 0) {
-      s_red[0][warp] = hmn;
-      s_red[1][warp] = hmx;
-    }
-    __syncthreads();
-    hmn = s_red[0][0];
-    hmx = s_red[1][0];
-    for (int w = 1; w < kThreads / 32; ++w) {
-      hmn = min(hmn, s_red[0][w]);
-      hmx = max(hmx, s_red[1][w]);
-    }
-    const uint32_t hr = hmx - hmn;
-    int sh = 0;
-    while (sh < 32 && (static_cast<uint64_t>(hr) >> sh) >= static_cast<uint64_t>(kBins)) ++sh;
-    auto bin = [=](uint64_t x) -> int {
-      return sh < 32 ? static_cast<int>((static_cast<uint32_t>(x >> 32) - hmn) >> sh) : 0;
-    };
-    for (int j = tid; j < c; j += kThreads) atomicAdd(&hist[bin(cand[j])], 1u);
-    __syncthreads();
-    // exclusive scan of the counts (thread t owns bins 2t, 2t + 1), largest bin
-    const uint32_t c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
-    const uint32_t loc = c0 + c1;
-    uint32_t incl = loc, cm = max(c0, c1);
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t tt = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += tt;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-    if (lane == 31) s_wt[warp] = incl;
-    if (lane == 0) s_red[0][warp] = cm;
-    __syncthreads();
-    if (warp == 0) {
-      const uint32_t v = s_wt[lane];
-      uint32_t in2 = v, m2 = s_red[0][lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t tt = __shfl_up_sync(0xffffffffu, in2, o);
-        if (lane >= o) in2 += tt;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m2 = max(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-      s_wt[lane] = in2 - v;
-      if (lane == 0) s_bmax = static_cast<int>(m2);
-    }
-    __syncthreads();
-    const uint32_t pre = s_wt[warp] + incl - loc;
-    hist[2 * tid] = pre;  // start of each bin
-    hist[2 * tid + 1] = pre + c0;
-    __syncthreads();
-    if (s_bmax <= kMaxBin) {
-      // group by bin; afterwards bin b spans [end(b - 1), hist[b]) with
-      // end(-1) = 0
-      for (int j = tid; j < c; j += kThreads) {
-        const uint64_t x = cand[j];
-        grp[atomicAdd(&hist[bin(x)], 1u)] = x;
-      }
-      __syncthreads();
-      for (int p = tid; p < c; p += kThreads) {
-        const uint64_t x = grp[p];
-        const int b = bin(x);
-        const int lo = b == 0 ? 0 : static_cast<int>(hist[b - 1]);
-        if (lo >= nw) continue;  // the whole bin lies past the first k
-        const int hi = static_cast<int>(hist[b]);
-        int rk = lo;
-        for (int q = lo; q < hi; ++q) rk += grp[q] < x ? 1 : 0;
-        if (rk < nw) {
-          out[rk] = order_key_id(x);
-          if (outs) outs[rk] = order_key_score(x);
-        }
-      }
-    } else {
-      int np = 1;
-      while (np < c) np <<= 1;
-      for (int j = c + tid; j < np; j += kThreads) cand[j] = kOrderPad;
-      __syncthreads();
-      block_sort_u64(cand, np);
-      for (int j = tid; j < nw; j += kThreads) {
-        out[j] = order_key_id(cand[j]);
-        if (outs) outs[j] = order_key_score(cand[j]);
-      }
-    }
+    emit_sorted_prefix(cand, c, nw, grp, hist, out, outs);
     for (int j = nw + tid; j < k; j += kThreads) {
       out[j] = -1;
       if (outs) outs[j] = -INFINITY;

@@ -550,3 +550,36 @@ def test_exhaustive_row_topk_equal_score_paths():
     for i in range(T // 2, T):                # the k smallest ids of 9000 equal scores
         assert np.array_equal(got[i], b_pos[:k]), f"row {i}"
         assert np.all(gs[i] == gs[i, 0]), f"row {i}"
+
+
+@pytest.mark.parametrize("T", [1, 3, 37, 148])
+def test_refine_split_is_bitwise_undivided(T):
+    """Small chunks on the pipelined refine: each query's candidate list
+    divided among CTAs (contiguous ranges of its 128-slot tiles, the partial
+    top-k merged into the output order) gives the same ids and scores, bit
+    for bit, as one CTA per list, for the automatic and the forced splits.
+    (The decode test checks the divided path against the oracle.)"""
+    wl = S.scaled(S.WORKLOADS["glm_bf16_L128k"], L=32768, T=4096, refit_period=8192, budget=4096,
+                  k=1024, M=512)
+    gpu, _ = P.make_pair(wl)
+    for c in range(wl.n_chunks):
+        kd, ks, _ = P.keys_inputs(wl, c * wl.T, (c + 1) * wl.T)
+        gpu.append_keys(kd, ks)
+        gpu.seal()
+    gpu.publish()
+    p0 = wl.L - 200
+    qd, wd, _, _ = P.query_inputs(wl, p0, p0 + T)
+    res = {}
+    for split in (1, 0, 2, 5, 8):
+        gpu.debug_refine_split(split)
+        out = torch.full((T, wl.k), -7, dtype=torch.int32, device="cuda")
+        osc = torch.zeros((T, wl.k), dtype=torch.float32, device="cuda")
+        gpu.route_refine(qd, wd, p0, wl.k, wl.budget, out=out, out_scores=osc)
+        gpu.sync()
+        res[split] = (out.cpu().numpy(), osc.cpu().numpy())
+    gpu.close()
+    ids1, sc1 = res[1]
+    assert (ids1 >= 0).sum() == T * wl.k
+    for split in (0, 2, 5, 8):
+        assert np.array_equal(res[split][0], ids1), f"split {split}: ids"
+        assert np.array_equal(res[split][1].view(np.uint32), sc1.view(np.uint32)), f"split {split}: scores"
