@@ -246,7 +246,7 @@ __device__ inline void emit_sorted_prefix(uint64_t* keys, int c, int nw, uint64_
                                    float* outs) {
   constexpr int kMaxBin = 64;
   __shared__ uint32_t s_wt[32], s_red[2][32];
-  __shared__ int s_bmax, s_bend;
+  __shared__ int s_bmax, s_bend, s_nbin;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // score-key range of the keys (high words: ~f2key(score))
   uint32_t hmn = 0xffffffffu, hmx = 0u;
@@ -334,6 +334,7 @@ __device__ inline void emit_sorted_prefix(uint64_t* keys, int c, int nw, uint64_
       s_red[0][warp] = cm;
       s_red[1][warp] = be;
     }
+    if (tid == 1023) s_nbin = static_cast<int>(st1 + c1);  // keys binned (hi <= hhi)
     hist[2 * tid] = st0;
     hist[2 * tid + 1] = st1;
     __syncthreads();
@@ -358,8 +359,9 @@ __device__ inline void emit_sorted_prefix(uint64_t* keys, int c, int nw, uint64_
     __syncthreads();  // every thread has read s_bend before the next round
   }
   const int b_end = s_bend;
-  // keys of bins [0, b_end) fill grp[0 .. n_rel) after grouping
-  const int n_rel = b_end < kPrefixBins ? static_cast<int>(hist[b_end]) : c;
+  // keys of bins [0, b_end) fill grp[0 .. n_rel) after grouping (keys
+  // above hhi are in no bin)
+  const int n_rel = b_end < kPrefixBins ? static_cast<int>(hist[b_end]) : s_nbin;
   if (s_bmax <= kMaxBin) {
     // group the keys of bins before b_end; afterwards such a bin b spans
     // [end(b - 1), hist[b]) with end(-1) = 0
@@ -372,6 +374,7 @@ __device__ inline void emit_sorted_prefix(uint64_t* keys, int c, int nw, uint64_
     for (int p = tid; p < n_rel; p += 1024) {
       const uint64_t x = grp[p];
       const int b = bin(x);
+      if (b >= b_end) continue;  // (every grouped key is in a bin before b_end)
       const int lo = b == 0 ? 0 : static_cast<int>(hist[b - 1]);
       const int hi = static_cast<int>(hist[b]);
       int rk = lo;

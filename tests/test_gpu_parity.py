@@ -583,3 +583,41 @@ def test_refine_split_is_bitwise_undivided(T):
     for split in (0, 2, 5, 8):
         assert np.array_equal(res[split][0], ids1), f"split {split}: ids"
         assert np.array_equal(res[split][1].view(np.uint32), sc1.view(np.uint32)), f"split {split}: scores"
+
+
+def test_merge_topk_wide_score_range():
+    """The merge's ordering bins the scores of its keys; a few far-off
+    scores make the range wide, so the bins holding the first k keys are
+    binned once more over just their part of the range.  Here the k-th key
+    lies in the last of those finer bins (one top score, a block of 60
+    scores 2^21 order-key steps below it, 500 scores near -1e29): the
+    result is the exact top k in (score desc, id asc) order."""
+    from ivf_top_key_b200 import merge_topk
+    s0 = np.float32(1000.0)
+    blk = (np.uint32(s0.view(np.uint32) - (1 << 21) + 10) + np.arange(5, dtype=np.uint32)).view(np.float32)
+    sc = np.concatenate([[s0], np.repeat(blk, 12), np.float32(-1e29) + np.arange(500, dtype=np.float32)])
+    sc = sc.astype(np.float32)
+    ids = np.random.default_rng(3).permutation(4000)[:sc.size].astype(np.int32)
+    for k in (30, 61, 200):
+        P_ = 2
+        half = (sc.size + 1) // 2
+        pid = np.full((P_, 1, 400), -1, np.int32)
+        psc = np.full((P_, 1, 400), -np.inf, np.float32)
+        pid[0, 0, :half], psc[0, 0, :half] = ids[:half], sc[:half]
+        pid[1, 0, :sc.size - half], psc[1, 0, :sc.size - half] = ids[half:], sc[half:]
+        # each part keeps its own top k (the merge's input contract)
+        for p in range(P_):
+            v = pid[p, 0] >= 0
+            o = np.lexsort((pid[p, 0][v], -psc[p, 0][v].astype(np.float64)))[:k]
+            i2, s2 = pid[p, 0][v][o], psc[p, 0][v][o]
+            pid[p, 0], psc[p, 0] = -1, -np.inf
+            pid[p, 0, :i2.size], psc[p, 0, :s2.size] = i2, s2
+        ids_d = torch.from_numpy(pid[:, :, :k].copy()).cuda()
+        sc_d = torch.from_numpy(psc[:, :, :k].copy()).cuda()
+        out = torch.full((1, k), -7, dtype=torch.int32, device="cuda")
+        osc = torch.zeros((1, k), dtype=torch.float32, device="cuda")
+        merge_topk(ids_d, sc_d, k, out=out, out_scores=osc)
+        torch.cuda.synchronize()
+        o = np.lexsort((ids, -sc.astype(np.float64)))[:k]
+        assert np.array_equal(out.cpu().numpy()[0], ids[o]), k
+        assert np.array_equal(osc.cpu().numpy()[0].view(np.uint32), sc[o].view(np.uint32)), k
