@@ -31,3 +31,27 @@ def test_library_exports_every_declared_symbol():
 def test_binding_wraps_every_declared_symbol():
     from ivf_top_key_b200 import _capi
     assert sorted(_capi.EXPORTED) == declared_symbols()
+
+
+def declared_arities():
+    """Parameter count of every entry point's prototype in the header."""
+    src = open(os.path.join(ROOT, "include", "ai_index.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(ai_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        p = " ".join(params.split())
+        out[name] = 0 if p in ("", "void") else p.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every ctypes prototype in the binding takes as many arguments as the
+    C declaration (a dropped or added parameter would shift every later
+    argument silently)."""
+    from ivf_top_key_b200 import _capi
+    ar = declared_arities()
+    assert sorted(ar) == declared_symbols()
+    for name, n in ar.items():
+        f = getattr(_capi._lib, name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == n, (name, len(f.argtypes), n)
