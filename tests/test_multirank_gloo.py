@@ -114,15 +114,18 @@ def _shard_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_ranks_sharded_exchange_gives_the_global_topk():
+@pytest.mark.parametrize("world", [2, 3])
+def test_ranks_sharded_exchange_gives_the_global_topk(world):
+    """2 ranks split the 8 tiles of each list evenly, 3 ranks unevenly
+    (2, 3 and 3 tiles)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    ps = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
     for p in ps:
         p.start()
     res = sorted(q.get(timeout=120) for _ in ps)
     for p in ps:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert res == [(0, True), (1, True)]
+    assert res == [(r, True) for r in range(world)]
